@@ -1,0 +1,9 @@
+"""The CPU oracle against its pins (no GPU)."""
+import pytest
+
+from oracle_pins import ALL_PINS
+
+
+@pytest.mark.parametrize("pin", ALL_PINS, ids=[p.__name__ for p in ALL_PINS])
+def test_pin(oracle, pin):
+    pin(oracle)

@@ -1,0 +1,34 @@
+"""Each planted mistake in the oracle must be caught by at least one pin (no GPU).
+
+The mistakes are compiled into separate copies of the oracle (``ORACLE_PLANT_*``); the
+real oracle is never modified.  A mistake that no pin catches would mean the pins do not
+tie that part of the oracle to the pages.
+"""
+import pytest
+
+from oracle import Oracle
+from oracle_pins import ALL_PINS
+
+PLANTS = [
+    "ORACLE_PLANT_Q2_MSB_FIRST",      # wrong bit order
+    "ORACLE_PLANT_Q2_NO_OFFSET",      # dropped the -1 in (q - 1) d
+    "ORACLE_PLANT_Q2_SIGN",           # (1 - q) d
+    "ORACLE_PLANT_Q2_SCALE_BLOCK64",  # scale indexed per 64 instead of per 128 weights
+    "ORACLE_PLANT_Q4_NIBBLE_SWAP",    # even index in the high nibble
+    "ORACLE_PLANT_Q4_ZERO_SIGN",      # (q + z) s
+    "ORACLE_PLANT_F16_TRUNCATE",      # f32 -> f16 truncates instead of rounding
+    "ORACLE_PLANT_GEMM_TRANSPOSED",   # transposed weight operand
+    "ORACLE_PLANT_LORA_DROPPED",      # side branch missing
+]
+
+
+@pytest.mark.parametrize("plant", PLANTS)
+def test_plant_is_caught(plant):
+    mutant = Oracle(defines=(plant,))
+    failed = []
+    for pin in ALL_PINS:
+        try:
+            pin(mutant)
+        except AssertionError:
+            failed.append(pin.__name__)
+    assert failed, f"no pin catches {plant}"
