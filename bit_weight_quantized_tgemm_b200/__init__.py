@@ -1,1 +1,12 @@
-"""B200 (sm_100a) ternary / 4-bit dequant-fused matmul library: Python binding."""
+"""B200 (sm_100a) ternary / 4-bit dequant-fused matmul library.
+
+The compute lives in ``libtgemm.so`` (hand-written CUDA, C ABI in ``include/tgemm.h``);
+this package is the Python binding (:mod:`.binding`) plus seeded synthetic workloads
+(:mod:`.synth`).  PyTorch supplies device memory and streams only.
+"""
+from .binding import (  # noqa: F401
+    DEVERR_TIMEOUT, EALIGN, EARCH, ECUDA, EINVAL, EWORKSPACE, OK, OP_Q2, OP_Q2_LORA, OP_Q4,
+    OUT_BF16, OUT_F32, PACK_BAD_CODE, PACK_INEXACT, PACK_NONFINITE, PATH_AUTO, PATH_SMALL_M,
+    PATH_TENSOR, TgemmError, device_error, gemm_q2, gemm_q2_lora, gemm_q4, lib, library_path,
+    q2_dequant, q2_pack, q4_dequant, q4_pack, set_path, version, workspace_size,
+)

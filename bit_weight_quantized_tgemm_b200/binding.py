@@ -1,0 +1,254 @@
+"""Thin ctypes binding over libtgemm.so (include/tgemm.h).
+
+Argument marshalling only: every function checks tensor dtype/device/contiguity, passes
+``data_ptr()`` values and the current CUDA stream to the C entry point of the same name,
+and raises :class:`TgemmError` on a nonzero status.  All computation happens in the CUDA
+kernels.  There is no fallback: if the shared library is missing or fails to load,
+every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+from typing import Optional
+
+import torch
+
+from . import build as _build
+
+OK, EINVAL, EALIGN, ECUDA, EARCH, EWORKSPACE = 0, -1, -2, -3, -4, -5
+OUT_F32, OUT_BF16 = 0, 1
+OP_Q2, OP_Q2_LORA, OP_Q4 = 0, 1, 2
+PATH_AUTO, PATH_SMALL_M, PATH_TENSOR = 0, 1, 2
+PACK_BAD_CODE, PACK_INEXACT, PACK_NONFINITE = 1, 2, 4
+DEVERR_TIMEOUT = 1
+
+_P = ctypes.c_void_p
+_i = ctypes.c_int
+_sz = ctypes.c_size_t
+
+_SIGS = {
+    "q2_pack": (_i, [_P, _P, _P, _P, _i, _i, _P, _P]),
+    "q4_pack": (_i, [_P, _P, _P, _P, _P, _i, _i, _P, _P]),
+    "q2_dequant": (_i, [_P, _P, _P, _i, _i, _P]),
+    "q4_dequant": (_i, [_P, _P, _P, _i, _i, _P]),
+    "tgemm_workspace_size": (_sz, [_i, _i, _i, _i, _i]),
+    "tgemm_q2": (_i, [_P, _P, _P, _P, _i, _i, _i, _i, _P, _sz, _P]),
+    "tgemm_q2_lora": (_i, [_P, _P, _P, _P, _P, _i, _P, _i, _i, _i, _i, _P, _sz, _P]),
+    "tgemm_q4": (_i, [_P, _P, _P, _P, _i, _i, _i, _i, _P, _sz, _P]),
+    "tgemm_strerror": (ctypes.c_char_p, [_i]),
+    "tgemm_set_path": (_i, [_i]),
+    "tgemm_device_error": (_i, [_P, _i]),
+    "tgemm_version": (_i, []),
+}
+
+
+class TgemmError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        try:
+            msg = lib().tgemm_strerror(status).decode()
+        except Exception:  # pragma: no cover - only if the library itself is unusable
+            msg = "?"
+        super().__init__(f"{where}: status {status} ({msg})")
+
+
+_lib = None
+_lock = threading.Lock()
+
+
+def library_path() -> str:
+    return _build.LIB
+
+
+def lib():
+    """Load libtgemm.so (building it first if the sources are newer)."""
+    global _lib
+    if _lib is None:
+        with _lock:
+            if _lib is None:
+                path = _build.LIB
+                if not os.path.exists(path) or _build.stale():
+                    _build.build()
+                handle = ctypes.CDLL(path)
+                for name, (res, args) in _SIGS.items():
+                    fn = getattr(handle, name)
+                    fn.restype = res
+                    fn.argtypes = args
+                _lib = handle
+    return _lib
+
+
+def _check(status: int, where: str):
+    if status != OK:
+        raise TgemmError(status, where)
+
+
+def _stream() -> int:
+    return torch.cuda.current_stream().cuda_stream
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else t.data_ptr()
+
+
+def _need(t: torch.Tensor, dtype, name: str):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+# ---- packing ----------------------------------------------------------------------------
+
+def q2_pack(codes: torch.Tensor, scale: torch.Tensor, status: Optional[torch.Tensor] = None):
+    """codes uint8 [N, K], scale f32 [N, K/128] -> (wq uint8 [N, K/4], d f16 [N, K/128], status)."""
+    _need(codes, torch.uint8, "codes")
+    _need(scale, torch.float32, "scale")
+    N, K = codes.shape
+    wq = torch.empty((N, K // 4), dtype=torch.uint8, device=codes.device)
+    d = torch.empty((N, K // 128), dtype=torch.float16, device=codes.device)
+    if status is None:
+        status = torch.zeros(1, dtype=torch.int32, device=codes.device)
+    _check(lib().q2_pack(_ptr(codes), _ptr(scale), _ptr(wq), _ptr(d), N, K, _ptr(status),
+                         _stream()), "q2_pack")
+    return wq, d, status
+
+
+def q4_pack(codes: torch.Tensor, s: torch.Tensor, z: torch.Tensor,
+            status: Optional[torch.Tensor] = None):
+    """codes uint8 [N, K], s, z f32 [N, K/64] -> (wq uint8 [N, K/2], sz f16 [N, K/64, 2], status)."""
+    _need(codes, torch.uint8, "codes")
+    _need(s, torch.float32, "s")
+    _need(z, torch.float32, "z")
+    N, K = codes.shape
+    wq = torch.empty((N, K // 2), dtype=torch.uint8, device=codes.device)
+    sz = torch.empty((N, K // 64, 2), dtype=torch.float16, device=codes.device)
+    if status is None:
+        status = torch.zeros(1, dtype=torch.int32, device=codes.device)
+    _check(lib().q4_pack(_ptr(codes), _ptr(s), _ptr(z), _ptr(wq), _ptr(sz), N, K, _ptr(status),
+                         _stream()), "q4_pack")
+    return wq, sz, status
+
+
+def q2_dequant(wq: torch.Tensor, d: torch.Tensor) -> torch.Tensor:
+    _need(wq, torch.uint8, "wq")
+    _need(d, torch.float16, "d")
+    N, K = wq.shape[0], wq.shape[1] * 4
+    w = torch.empty((N, K), dtype=torch.float32, device=wq.device)
+    _check(lib().q2_dequant(_ptr(wq), _ptr(d), _ptr(w), N, K, _stream()), "q2_dequant")
+    return w
+
+
+def q4_dequant(wq: torch.Tensor, sz: torch.Tensor) -> torch.Tensor:
+    _need(wq, torch.uint8, "wq")
+    _need(sz, torch.float16, "sz")
+    N, K = wq.shape[0], wq.shape[1] * 2
+    w = torch.empty((N, K), dtype=torch.float32, device=wq.device)
+    _check(lib().q4_dequant(_ptr(wq), _ptr(sz), _ptr(w), N, K, _stream()), "q4_dequant")
+    return w
+
+
+# ---- matmuls --------------------------------------------------------------------------------
+
+def workspace_size(op: int, M: int, N: int, K: int, r: int = 0) -> int:
+    return int(lib().tgemm_workspace_size(op, M, N, K, r))
+
+
+_ws_cache = {}
+
+
+def _workspace(op, M, N, K, r, device, workspace):
+    need = workspace_size(op, M, N, K, r)
+    if need == 0:
+        return None, 0
+    if workspace is not None:
+        _need(workspace, torch.uint8, "workspace")
+        return workspace, workspace.numel()
+    key = (device.index if device.index is not None else torch.cuda.current_device())
+    buf = _ws_cache.get(key)
+    if buf is None or buf.numel() < need:
+        buf = torch.empty(need, dtype=torch.uint8, device=device)
+        _ws_cache[key] = buf
+    return buf, buf.numel()
+
+
+def _out(y, M, N, out_dtype, device):
+    dt = torch.float32 if out_dtype == OUT_F32 else torch.bfloat16
+    if y is None:
+        return torch.empty((M, N), dtype=dt, device=device)
+    _need(y, dt, "y")
+    if tuple(y.shape) != (M, N):
+        raise ValueError(f"y must have shape {(M, N)}")
+    return y
+
+
+def gemm_q2(x: torch.Tensor, wq: torch.Tensor, d: torch.Tensor, *, out_dtype: int = OUT_BF16,
+            y: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None):
+    """y = x . W^T, x bf16 [M, K], W packed Q2_0 (wq uint8 [N, K/4], d f16 [N, K/128])."""
+    _need(x, torch.bfloat16, "x")
+    _need(wq, torch.uint8, "wq")
+    _need(d, torch.float16, "d")
+    M, K = x.shape
+    N = wq.shape[0]
+    y = _out(y, M, N, out_dtype, x.device)
+    ws, nbytes = _workspace(OP_Q2, M, N, K, 0, x.device, workspace)
+    _check(lib().tgemm_q2(_ptr(x), _ptr(wq), _ptr(d), _ptr(y), M, N, K, out_dtype, _ptr(ws),
+                          nbytes, _stream()), "tgemm_q2")
+    return y
+
+
+def gemm_q2_lora(x, wq, d, a, b, *, out_dtype: int = OUT_BF16, y=None, workspace=None):
+    """y = x . W^T + (x . A^T) . B^T with a bf16 [r, K], b bf16 [N, r]."""
+    _need(x, torch.bfloat16, "x")
+    _need(wq, torch.uint8, "wq")
+    _need(d, torch.float16, "d")
+    _need(a, torch.bfloat16, "a")
+    _need(b, torch.bfloat16, "b")
+    M, K = x.shape
+    N = wq.shape[0]
+    r = a.shape[0]
+    y = _out(y, M, N, out_dtype, x.device)
+    ws, nbytes = _workspace(OP_Q2_LORA, M, N, K, r, x.device, workspace)
+    _check(lib().tgemm_q2_lora(_ptr(x), _ptr(wq), _ptr(d), _ptr(a), _ptr(b), r, _ptr(y), M, N,
+                               K, out_dtype, _ptr(ws), nbytes, _stream()), "tgemm_q2_lora")
+    return y
+
+
+def gemm_q4(x, wq, sz, *, out_dtype: int = OUT_BF16, y=None, workspace=None):
+    """y = x . W^T for 4-bit weights (wq uint8 [N, K/2], sz f16 [N, K/64, 2])."""
+    _need(x, torch.bfloat16, "x")
+    _need(wq, torch.uint8, "wq")
+    _need(sz, torch.float16, "sz")
+    M, K = x.shape
+    N = wq.shape[0]
+    y = _out(y, M, N, out_dtype, x.device)
+    ws, nbytes = _workspace(OP_Q4, M, N, K, 0, x.device, workspace)
+    _check(lib().tgemm_q4(_ptr(x), _ptr(wq), _ptr(sz), _ptr(y), M, N, K, out_dtype, _ptr(ws),
+                          nbytes, _stream()), "tgemm_q4")
+    return y
+
+
+# ---- control -------------------------------------------------------------------------------
+
+def set_path(path: int) -> int:
+    prev = lib().tgemm_set_path(path)
+    if prev < 0:
+        raise TgemmError(prev, "tgemm_set_path")
+    return prev
+
+
+def device_error(clear: bool = False) -> int:
+    bits = ctypes.c_uint32(0)
+    _check(lib().tgemm_device_error(ctypes.addressof(bits), 1 if clear else 0),
+           "tgemm_device_error")
+    return int(bits.value)
+
+
+def version() -> int:
+    return int(lib().tgemm_version())

@@ -1,0 +1,508 @@
+// gemm_tc.cuh -- large-M path: persistent tcgen05 (5th-generation tensor core) kernel.
+//
+// Tile: 128 tokens (TMEM lanes) x 256 weight rows (accumulator columns) x 64 k per stage.
+// Warp roles (14 warps, one CTA per SM):
+//   warp 0      TMA producer: activation tile (f16, 128-byte swizzle) + packed weight tile
+//   warp 1      TMEM allocator and MMA issuer (one thread): 4 x tcgen05.mma 128x256x16
+//   warps 2-9   dequantizers: thread i owns weight row i of the tile; it unpacks its 64
+//               codes per stage, multiplies by the block scale in f16 and stores the row
+//               straight into the 128-byte-swizzled K-major operand layout
+//   warps 10-13 epilogue: tcgen05.ld of the f32 accumulator, convert, store y
+// The accumulator is double-buffered in TMEM (2 x 256 columns), so a tile's epilogue
+// overlaps the next tile's main loop.
+//
+// Operand precision: kind::f16 with both operands f16.  Q2_0 weights (q - 1) * d are
+// exact in f16; 4-bit weights are computed as ((q - z) * s) in f16, exact up to the
+// final rounding.  The activations arrive as an f16 copy (prep_x16_kernel) whose k order
+// inside each 16-group (Q2) or 8-group (4-bit) is permuted to match the order in which a
+// 32-bit word of packed codes unpacks with one shift and one mask per pair:
+//   Q2:    pair i of a 16-code word = codes (i, i+8),  i < 8
+//   4-bit: pair i of an 8-code word = codes (i, i+4),  i < 4
+// Both operands use the same permutation, so the contraction is unchanged.
+//
+// The low-rank branch y += (x A^T) B^T ("mindview-t2i-turbo", section "One step") runs as
+// extra pipeline stages after the main K loop: the A-operand stage holds u = x A^T as a
+// bf16 pair [hi | lo], the B-operand stage holds [B | B], and a bf16 MMA adds
+// u_hi B^T + u_lo B^T into the same accumulator.
+#pragma once
+
+#include "common.cuh"
+
+namespace tgemm {
+
+constexpr int kTcBM = 128;
+constexpr int kTcBN = 256;
+constexpr int kTcBK = 64;
+constexpr int kTcStages = 4;
+constexpr int kTcWStages = 3;
+constexpr int kTcThreads = 448;
+constexpr int kTcXBytes = kTcBM * kTcBK * 2;  // 16 KB
+constexpr int kTcWBytes = kTcBN * kTcBK * 2;  // 32 KB
+constexpr int kTcTmemCols = 512;
+
+template <int FMT>
+struct TcFmt {
+  static constexpr int kWqRowBytes = FMT == 0 ? 16 : 32;  // packed bytes per row per stage
+  static constexpr int kWqStageBytes = kTcBN * kWqRowBytes;
+  static constexpr int kXOff = 0;
+  static constexpr int kWOff = kXOff + kTcStages * kTcXBytes;
+  static constexpr int kWqOff = kWOff + kTcWStages * kTcWBytes;
+  static constexpr int kBarOff = kWqOff + kTcStages * kWqStageBytes;
+  static constexpr int kNumBars = 2 * kTcStages + 2 * kTcWStages + 4 + 1;
+  static constexpr int kMiscOff = kBarOff + kNumBars * 8;
+  static constexpr int kSmemBytes = kMiscOff + 16 + 1024;  // + alignment slack
+};
+
+struct TcParams {
+  int M, N, K;
+  int tiles_m, num_tiles;
+  int kt_main;     // K / 64
+  int kt_lora;     // extra stages for the low-rank branch (0 without it)
+  int lora_mmas;   // K=16 MMAs in those stages: 2 * round_up(r, 16) / 16
+  int R;           // round_up(r, 16): width of u_hi (and of u_lo) in the concatenation
+  int r;
+  int out_f32;
+  int vec_store;   // rows of y are 16-byte aligned
+  const uint16_t* scales;  // Q2: d [N][K/128]; 4-bit: sz [N][K/64][2]
+  const uint16_t* lb;      // low-rank B [N][r] (bf16)
+  void* y;
+};
+
+__device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      atomicOr(&g_device_error, kDevErrTimeout);
+      return false;
+    }
+  }
+  return true;
+}
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
+                                             uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
+               "r"(d)
+               : "memory");
+}
+
+__device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(addr)
+               : "memory");
+  return v;
+}
+
+// Q2: 16 codes -> 8 f16x2 pairs (codes i, i+8) of (q - 1) * d.
+__device__ __forceinline__ void q2_word_to_f16(uint32_t w, uint32_t d2, uint32_t (&o)[8]) {
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const uint32_t t = lop3_and_or(w >> (2 * i), 0x00030003u, 0x64006400u);  // 1024 + q
+    o[i] = hmul2_u32(hsub2_u32(t, 0x64016401u), d2);                           // (q-1)*d
+  }
+}
+
+// 4-bit: 8 codes -> 4 f16x2 pairs (codes i, i+4) of (q - z) * s.
+__device__ __forceinline__ void q4_word_to_f16(uint32_t w, uint32_t s2, uint32_t z2,
+                                               uint32_t (&o)[4]) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint32_t t = lop3_and_or(w >> (4 * i), 0x000F000Fu, 0x64006400u);  // 1024 + q
+    o[i] = hmul2_u32(hsub2_u32(hsub2_u32(t, 0x64006400u), z2), s2);           // (q-z)*s
+  }
+}
+
+template <int FMT, bool LORA>
+__global__ void __launch_bounds__(kTcThreads, 1)
+    tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x,
+                   const __grid_constant__ CUtensorMap tm_w,
+                   const __grid_constant__ CUtensorMap tm_u, const TcParams p) {
+  using F = TcFmt<FMT>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bar0 = sbase + F::kBarOff;
+  // barrier addresses
+  auto full_bar = [&](int s) { return bar0 + 8u * s; };
+  auto empty_bar = [&](int s) { return bar0 + 8u * (kTcStages + s); };
+  auto wfull_bar = [&](int s) { return bar0 + 8u * (2 * kTcStages + s); };
+  auto wfree_bar = [&](int s) { return bar0 + 8u * (2 * kTcStages + kTcWStages + s); };
+  auto accfull_bar = [&](int a) { return bar0 + 8u * (2 * kTcStages + 2 * kTcWStages + a); };
+  auto accempty_bar = [&](int a) { return bar0 + 8u * (2 * kTcStages + 2 * kTcWStages + 2 + a); };
+  const uint32_t drain_bar = bar0 + 8u * (2 * kTcStages + 2 * kTcWStages + 4);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + F::kMiscOff);
+  volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + F::kMiscOff + 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kTcStages; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1 + 8);  // MMA commit + 8 dequant warps
+    }
+    for (int s = 0; s < kTcWStages; ++s) {
+      mbar_init(wfull_bar(s), 8);      // 8 dequant warps
+      mbar_init(wfree_bar(s), 1);      // MMA commit
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(accfull_bar(a), 1);    // MMA commit
+      mbar_init(accempty_bar(a), 4);   // 4 epilogue warps
+    }
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0u;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tm_x);
+    tma_prefetch_desc(&tm_w);
+    if (LORA) tma_prefetch_desc(&tm_u);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), kTcTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int ksteps = p.kt_main + (LORA ? p.kt_lora : 0);
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      uint32_t it = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
+        const int tm = tile % p.tiles_m, tn = tile / p.tiles_m;
+        for (int ks = 0; ks < ksteps; ++ks, ++it) {
+          const uint32_t s = it % kTcStages, ph = (it / kTcStages) & 1u;
+          if (!mbar_wait(empty_bar(s), ph ^ 1u, abort_flag)) { ok = false; break; }
+          const uint32_t xdst = sbase + F::kXOff + s * kTcXBytes;
+          if (ks < p.kt_main) {
+            mbar_arrive_expect_tx(full_bar(s), kTcXBytes + F::kWqStageBytes);
+            tma_load_2d(xdst, &tm_x, full_bar(s), ks * kTcBK, tm * kTcBM);
+            tma_load_2d(sbase + F::kWqOff + s * F::kWqStageBytes, &tm_w, full_bar(s),
+                        ks * F::kWqRowBytes, tn * kTcBN);
+          } else {
+            mbar_arrive_expect_tx(full_bar(s), kTcXBytes);
+            tma_load_2d(xdst, &tm_u, full_bar(s), (ks - p.kt_main) * kTcBK, tm * kTcBM);
+          }
+        }
+      }
+      // every load issued must land before the CTA may exit
+      const uint32_t n_issued = it;
+      for (uint32_t j = (n_issued > kTcStages ? n_issued - kTcStages : 0); j < n_issued; ++j)
+        mbar_wait_drain(full_bar(j % kTcStages), (j / kTcStages) & 1u);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t kIdescMain = make_idesc_f16(0u, kTcBM, kTcBN);  // f16 x f16
+      constexpr uint32_t kIdescLora = make_idesc_f16(1u, kTcBM, kTcBN);  // bf16 x bf16
+      uint32_t it = 0, wit = 0, tcount = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x, ++tcount) {
+        const uint32_t a = tcount & 1u, aph = (tcount >> 1) & 1u;
+        if (!mbar_wait(accempty_bar(a), aph ^ 1u, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + a * kTcBN;
+        for (int ks = 0; ks < ksteps; ++ks, ++it, ++wit) {
+          const uint32_t s = it % kTcStages, ph = (it / kTcStages) & 1u;
+          const uint32_t ws = wit % kTcWStages, wph = (wit / kTcWStages) & 1u;
+          if (!mbar_wait(full_bar(s), ph, abort_flag)) { ok = false; break; }
+          if (!mbar_wait(wfull_bar(ws), wph, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          const uint64_t adesc = smem_desc_sw128(sbase + F::kXOff + s * kTcXBytes);
+          const uint64_t bdesc = smem_desc_sw128(sbase + F::kWOff + ws * kTcWBytes);
+          if (!LORA || ks < p.kt_main) {
+#pragma unroll
+            for (int kk = 0; kk < kTcBK / 16; ++kk)
+              mma_f16_ss(d_tmem, adesc + 2u * kk, bdesc + 2u * kk, kIdescMain,
+                         (ks > 0 || kk > 0) ? 1u : 0u);
+          } else {
+            const int done = (ks - p.kt_main) * (kTcBK / 16);
+            for (int kk = 0; kk < kTcBK / 16 && done + kk < p.lora_mmas; ++kk)
+              mma_f16_ss(d_tmem, adesc + 2u * kk, bdesc + 2u * kk, kIdescLora, 1u);
+          }
+          mma_commit(empty_bar(s));
+          mma_commit(wfree_bar(ws));
+        }
+        if (!ok) break;
+        mma_commit(accfull_bar(a));
+      }
+      // all MMAs this thread issued must finish before TMEM is released
+      mma_commit(drain_bar);
+      mbar_wait_drain(drain_bar, 0u);
+    }
+  } else if (warp < 10) {
+    // ------------------------------------------------------------ dequantizers
+    const int dt = threadIdx.x - 64;  // weight row within the tile
+    const int swz = dt & 7;
+    const uint32_t row_off = static_cast<uint32_t>((dt >> 3) * 1024 + (dt & 7) * 128);
+    const int nscale = FMT == 0 ? p.K / 128 : p.K / 64;
+    uint32_t it = 0, wit = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
+      const int tn = tile / p.tiles_m;
+      const int row = tn * kTcBN + dt;
+      const bool valid = row < p.N;
+      const uint16_t* srow = p.scales + static_cast<int64_t>(row) * nscale * (FMT == 0 ? 1 : 2);
+      // scale for the next block (Q2) / group (4-bit), loaded one step ahead
+      uint32_t nxt = 0;
+      if (valid) nxt = FMT == 0 ? static_cast<uint32_t>(srow[0])
+                                : *reinterpret_cast<const uint32_t*>(srow);
+      uint32_t cur = 0;
+      for (int ks = 0; ks < ksteps; ++ks, ++it, ++wit) {
+        const uint32_t s = it % kTcStages, ph = (it / kTcStages) & 1u;
+        if (!mbar_wait(full_bar(s), ph, abort_flag)) { ok = false; break; }
+        const bool main_stage = !LORA || ks < p.kt_main;
+        uint4 pk0 = make_uint4(0, 0, 0, 0), pk1 = make_uint4(0, 0, 0, 0);
+        if (main_stage) {
+          const uint32_t src = sbase + F::kWqOff + s * F::kWqStageBytes + dt * F::kWqRowBytes;
+          pk0 = ld_shared_v4(src);
+          if (FMT == 1) pk1 = ld_shared_v4(src + 16);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(empty_bar(s));
+        const uint32_t ws = wit % kTcWStages, wph = (wit / kTcWStages) & 1u;
+        if (!mbar_wait(wfree_bar(ws), wph ^ 1u, abort_flag)) { ok = false; break; }
+        const uint32_t wrow = sbase + F::kWOff + ws * kTcWBytes + row_off;
+        if (main_stage) {
+          if (FMT == 0) {
+            if ((ks & 1) == 0) {
+              cur = nxt;
+              const int nb = (ks >> 1) + 1;
+              if (valid && nb < nscale) nxt = srow[nb];
+            }
+            const uint32_t d2 = cur | (cur << 16);
+            const uint32_t words[4] = {pk0.x, pk0.y, pk0.z, pk0.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              uint32_t o[8];
+              q2_word_to_f16(words[j], d2, o);
+              st_shared_v4(wrow + (((2 * j) ^ swz) << 4), o[0], o[1], o[2], o[3]);
+              st_shared_v4(wrow + (((2 * j + 1) ^ swz) << 4), o[4], o[5], o[6], o[7]);
+            }
+          } else {
+            cur = nxt;
+            if (valid && ks + 1 < nscale) nxt = reinterpret_cast<const uint32_t*>(srow)[ks + 1];
+            const uint32_t s2 = (cur & 0xFFFFu) | (cur << 16);
+            const uint32_t z2 = (cur >> 16) | (cur & 0xFFFF0000u);
+            const uint32_t words[8] = {pk0.x, pk0.y, pk0.z, pk0.w, pk1.x, pk1.y, pk1.z, pk1.w};
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              uint32_t o[4];
+              q4_word_to_f16(words[j], s2, z2, o);
+              st_shared_v4(wrow + ((j ^ swz) << 4), o[0], o[1], o[2], o[3]);
+            }
+          }
+        } else {
+          // low-rank stage: B-operand columns [jb, jb + 64) of [B | B], zero beyond 2R
+          const int jb = (ks - p.kt_main) * kTcBK;
+#pragma unroll 1
+          for (int cc = 0; cc < 8; ++cc) {
+            uint32_t o[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              uint32_t v2 = 0;
+#pragma unroll
+              for (int h = 0; h < 2; ++h) {
+                const int j = jb + 8 * cc + 2 * e + h;
+                const int i = j < p.R ? j : j - p.R;
+                uint32_t v = 0;
+                if (valid && j < 2 * p.R && i < p.r) v = p.lb[static_cast<int64_t>(row) * p.r + i];
+                v2 |= v << (16 * h);
+              }
+              o[e] = v2;
+            }
+            st_shared_v4(wrow + ((cc ^ swz) << 4), o[0], o[1], o[2], o[3]);
+          }
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(wfull_bar(ws));
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    uint32_t tcount = 0;
+    for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++tcount) {
+      const int tm = tile % p.tiles_m, tn = tile / p.tiles_m;
+      const uint32_t a = tcount & 1u, aph = (tcount >> 1) & 1u;
+      if (!mbar_wait(accfull_bar(a), aph, abort_flag)) break;
+      tc_fence_after();
+      const int m = tm * kTcBM + q * 32 + lane;
+      const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + a * kTcBN;
+#pragma unroll 1
+      for (int cc = 0; cc < kTcBN / 32; ++cc) {
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(tbase + cc * 32, v);
+        tmem_wait_ld();
+        const int n0 = tn * kTcBN + cc * 32;
+        if (m < p.M && n0 < p.N) {
+          const int64_t off = static_cast<int64_t>(m) * p.N + n0;
+          if (p.out_f32) {
+            float* dst = reinterpret_cast<float*>(p.y) + off;
+            if (p.vec_store && n0 + 32 <= p.N) {
+#pragma unroll
+              for (int e = 0; e < 8; ++e)
+                reinterpret_cast<uint4*>(dst)[e] = make_uint4(v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]);
+            } else {
+#pragma unroll
+              for (int e = 0; e < 32; ++e)
+                if (n0 + e < p.N) dst[e] = __uint_as_float(v[e]);
+            }
+          } else {
+            uint32_t b[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e)
+              b[e] = pack_bf16x2(__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1]));
+            uint16_t* dst = reinterpret_cast<uint16_t*>(p.y) + off;
+            if (p.vec_store && n0 + 32 <= p.N) {
+#pragma unroll
+              for (int e = 0; e < 4; ++e)
+                reinterpret_cast<uint4*>(dst)[e] = make_uint4(b[4 * e], b[4 * e + 1], b[4 * e + 2], b[4 * e + 3]);
+            } else {
+#pragma unroll
+              for (int e = 0; e < 32; ++e)
+                if (n0 + e < p.N) dst[e] = static_cast<uint16_t>(b[e >> 1] >> (16 * (e & 1)));
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(accempty_bar(a));
+    }
+  }
+
+  // ------------------------------------------------------------ teardown
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kTcTmemCols);
+  }
+}
+
+// ---- activation preparation ---------------------------------------------------------
+
+// bf16 [M][K] -> f16 [M][K] with the pair permutation the dequantizers produce
+// (FMT 0: within each 16-group, position 2i <- i, 2i+1 <- i+8; FMT 1: within each
+// 8-group, 2i <- i, 2i+1 <- i+4).  One thread per 16 elements.
+template <int FMT>
+__global__ void __launch_bounds__(256) prep_x16_kernel(const uint16_t* __restrict__ x,
+                                                       uint16_t* __restrict__ x16,
+                                                       int64_t ngroups) {
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t gidx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; gidx < ngroups;
+       gidx += stride) {
+    const uint4* src = reinterpret_cast<const uint4*>(x) + 2 * gidx;
+    const uint4 a = __ldg(src), b = __ldg(src + 1);
+    const uint32_t v[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+    float f[16];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      f[2 * i] = __uint_as_float(v[i] << 16);
+      f[2 * i + 1] = __uint_as_float(v[i] & 0xFFFF0000u);
+    }
+    uint32_t o[8];
+    if (FMT == 0) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) o[i] = pack_f16x2(f[i], f[i + 8]);
+    } else {
+#pragma unroll
+      for (int e8 = 0; e8 < 2; ++e8)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) o[4 * e8 + i] = pack_f16x2(f[8 * e8 + i], f[8 * e8 + i + 4]);
+    }
+    uint4* dst = reinterpret_cast<uint4*>(x16) + 2 * gidx;
+    dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
+    dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
+  }
+}
+
+// u = x A^T for the low-rank branch, f32 accumulation on mma.sync.  CTA: 16 tokens x up
+// to 64 branch columns (blockIdx.y picks the column chunk); its 8 warps split K and
+// reduce through shared memory.  Writes u in f32 [M][r] (small-M path) and/or the
+// concatenation ucat [M][wcat] = [bf16(u) pad R | bf16(u - bf16(u)) pad R | 0].
+__global__ void __launch_bounds__(256) lora_down_kernel(const uint16_t* __restrict__ x,
+                                                        const uint16_t* __restrict__ a, int M,
+                                                        int K, int r, int R, int wcat,
+                                                        float* __restrict__ u32,
+                                                        uint16_t* __restrict__ ucat) {
+  __shared__ float red[8][16][65];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, c = lane & 3;
+  const int m0 = blockIdx.x * 16;
+  const int col0 = blockIdx.y * 64;
+  float acc[8][4];
+#pragma unroll
+  for (int t = 0; t < 8; ++t)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) acc[t][e] = 0.f;
+  const uint32_t* x32 = reinterpret_cast<const uint32_t*>(x);
+  const uint32_t* a32 = reinterpret_cast<const uint32_t*>(a);
+  const int kw = K / 2;  // 32-bit words per row
+  for (int kb = warp; kb < K / 16; kb += 8) {
+    const int k2 = kb * 8 + c;  // word index of (k = 16kb + 2c, +1)
+    const bool r0 = m0 + g < M, r1 = m0 + g + 8 < M;
+    const uint32_t a0 = r0 ? __ldg(x32 + static_cast<int64_t>(m0 + g) * kw + k2) : 0u;
+    const uint32_t a1 = r1 ? __ldg(x32 + static_cast<int64_t>(m0 + g + 8) * kw + k2) : 0u;
+    const uint32_t a2 = r0 ? __ldg(x32 + static_cast<int64_t>(m0 + g) * kw + k2 + 4) : 0u;
+    const uint32_t a3 = r1 ? __ldg(x32 + static_cast<int64_t>(m0 + g + 8) * kw + k2 + 4) : 0u;
+#pragma unroll
+    for (int t = 0; t < 8; ++t) {
+      const int col = col0 + 8 * t + g;
+      const bool cv = col < r;
+      const uint32_t b0 = cv ? __ldg(a32 + static_cast<int64_t>(col) * kw + k2) : 0u;
+      const uint32_t b1 = cv ? __ldg(a32 + static_cast<int64_t>(col) * kw + k2 + 4) : 0u;
+      asm volatile(
+          "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
+          "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+          : "+f"(acc[t][0]), "+f"(acc[t][1]), "+f"(acc[t][2]), "+f"(acc[t][3])
+          : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+    }
+  }
+#pragma unroll
+  for (int t = 0; t < 8; ++t) {
+    red[warp][g][8 * t + 2 * c] = acc[t][0];
+    red[warp][g][8 * t + 2 * c + 1] = acc[t][1];
+    red[warp][g + 8][8 * t + 2 * c] = acc[t][2];
+    red[warp][g + 8][8 * t + 2 * c + 1] = acc[t][3];
+  }
+  __syncthreads();
+  for (int o = threadIdx.x; o < 16 * 64; o += blockDim.x) {
+    const int mm = o >> 6, cc = o & 63;
+    const int m = m0 + mm, col = col0 + cc;
+    if (m >= M) continue;
+    float v = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) v += red[w][mm][cc];
+    if (u32 != nullptr && col < r) u32[static_cast<int64_t>(m) * r + col] = v;
+    if (ucat != nullptr && col < R) {
+      uint16_t hi = 0, lo = 0;
+      if (col < r) {
+        const __nv_bfloat16 h = __float2bfloat16_rn(v);
+        hi = __bfloat16_as_ushort(h);
+        lo = __bfloat16_as_ushort(__float2bfloat16_rn(v - __bfloat162float(h)));
+      }
+      ucat[static_cast<int64_t>(m) * wcat + col] = hi;
+      ucat[static_cast<int64_t>(m) * wcat + R + col] = lo;
+    }
+  }
+  // zero the concatenation's tail [2R, wcat)
+  if (ucat != nullptr && blockIdx.y == 0) {
+    const int tail = wcat - 2 * R;
+    for (int o = threadIdx.x; o < 16 * tail; o += blockDim.x) {
+      const int m = m0 + o / tail;
+      if (m < M) ucat[static_cast<int64_t>(m) * wcat + 2 * R + o % tail] = 0;
+    }
+  }
+}
+
+}  // namespace tgemm

@@ -1,0 +1,174 @@
+// pack.cuh -- load-time packing of Q2_0 and 4-bit weights, and the dequant test hooks.
+//
+// Q2_0 ("We're Teaching Your Browser to Paint...", section "The lucky break that wasn't
+// luck"): code k of a row lands in bits 2*(k%4) of byte k/4; the f32 block scale becomes
+// an f16 that must round-trip exactly.  4-bit ("You Can Now Just Ask for an Image...",
+// section "The bug that hid in one flipped bit"): code t lands in the low nibble of byte
+// t/2 when t is even, the high nibble when odd.  Problems are reported through the
+// caller's status word; nothing traps.
+#pragma once
+
+#include "common.cuh"
+
+namespace tgemm {
+
+constexpr uint32_t kPackBadCode = 1u;
+constexpr uint32_t kPackInexact = 2u;
+constexpr uint32_t kPackNonFinite = 4u;
+
+// OR `bits` into *status once per warp (only lanes with something to report take part).
+__device__ __forceinline__ void report_status(uint32_t* status, uint32_t bits) {
+  const uint32_t all = __reduce_or_sync(0xFFFFFFFFu, bits);
+  if (all && (threadIdx.x & 31u) == 0u) atomicOr(status, all);
+}
+
+// f32 -> f16 (nearest even) plus the round-trip classification.
+__device__ __forceinline__ uint16_t scale_to_f16(float v, uint32_t& flags) {
+  const __half h = __float2half_rn(v);
+  if (!isfinite(v)) {
+    flags |= kPackNonFinite;
+  } else if (__half2float(h) != v) {
+    flags |= kPackInexact;
+  }
+  return __half_as_ushort(h);
+}
+
+// One thread packs 64 codes (64 bytes in) into 16 bytes out.
+__global__ void __launch_bounds__(256) q2_pack_kernel(const uint8_t* __restrict__ codes,
+                                                      const float* __restrict__ scale,
+                                                      uint8_t* __restrict__ wq,
+                                                      uint16_t* __restrict__ d, int64_t n_units,
+                                                      int64_t n_scales, uint32_t* status) {
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  const int64_t tid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int64_t iters = (n_units > n_scales ? n_units : n_scales);
+  for (int64_t base = 0; base < iters; base += stride) {
+    const int64_t u = base + tid;
+    uint32_t flags = 0;
+    if (u < n_units) {
+      const uint4* src = reinterpret_cast<const uint4*>(codes + u * 64);
+      uint32_t out[4];
+#pragma unroll
+      for (int v = 0; v < 4; ++v) {
+        const uint4 c = __ldg(src + v);
+        const uint32_t cw[4] = {c.x, c.y, c.z, c.w};
+        uint32_t word = 0;
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+          // cw[b] holds codes 4b..4b+3 of this 16-code group, one per byte.
+          const uint32_t q0 = cw[b] & 0xFFu, q1 = (cw[b] >> 8) & 0xFFu;
+          const uint32_t q2 = (cw[b] >> 16) & 0xFFu, q3 = cw[b] >> 24;
+          if ((q0 > 2u) | (q1 > 2u) | (q2 > 2u) | (q3 > 2u)) flags |= kPackBadCode;
+          const uint32_t byte = (q0 & 3u) | ((q1 & 3u) << 2) | ((q2 & 3u) << 4) | ((q3 & 3u) << 6);
+          word |= byte << (8 * b);
+        }
+        out[v] = word;
+      }
+      reinterpret_cast<uint4*>(wq)[u] = make_uint4(out[0], out[1], out[2], out[3]);
+    }
+    if (u < n_scales) d[u] = scale_to_f16(scale[u], flags);
+    report_status(status, flags);
+  }
+}
+
+// One thread packs 32 codes (32 bytes in) into 16 bytes out.
+__global__ void __launch_bounds__(256) q4_pack_kernel(const uint8_t* __restrict__ codes,
+                                                      const float* __restrict__ s,
+                                                      const float* __restrict__ z,
+                                                      uint8_t* __restrict__ wq,
+                                                      uint16_t* __restrict__ sz, int64_t n_units,
+                                                      int64_t n_groups, uint32_t* status) {
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  const int64_t tid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int64_t iters = (n_units > n_groups ? n_units : n_groups);
+  for (int64_t base = 0; base < iters; base += stride) {
+    const int64_t u = base + tid;
+    uint32_t flags = 0;
+    if (u < n_units) {
+      const uint4* src = reinterpret_cast<const uint4*>(codes + u * 32);
+      uint32_t out[4];
+#pragma unroll
+      for (int v = 0; v < 2; ++v) {
+        const uint4 c = __ldg(src + v);
+        const uint32_t cw[4] = {c.x, c.y, c.z, c.w};
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint32_t word = 0;
+#pragma unroll
+          for (int b = 0; b < 2; ++b) {
+            const uint32_t w4 = cw[2 * h + b];  // codes 4j..4j+3 of the group, one per byte
+            const uint32_t q0 = w4 & 0xFFu, q1 = (w4 >> 8) & 0xFFu;
+            const uint32_t q2 = (w4 >> 16) & 0xFFu, q3 = w4 >> 24;
+            if ((q0 > 15u) | (q1 > 15u) | (q2 > 15u) | (q3 > 15u)) flags |= kPackBadCode;
+            // even index -> low nibble, odd index -> high nibble
+            const uint32_t b0 = (q0 & 15u) | ((q1 & 15u) << 4);
+            const uint32_t b1 = (q2 & 15u) | ((q3 & 15u) << 4);
+            word |= (b0 | (b1 << 8)) << (16 * b);
+          }
+          out[2 * v + h] = word;
+        }
+      }
+      reinterpret_cast<uint4*>(wq)[u] = make_uint4(out[0], out[1], out[2], out[3]);
+    }
+    if (u < n_groups) {
+      const uint16_t hs = scale_to_f16(s[u], flags);
+      const uint16_t hz = scale_to_f16(z[u], flags);
+      reinterpret_cast<uint32_t*>(sz)[u] = static_cast<uint32_t>(hs) | (static_cast<uint32_t>(hz) << 16);
+    }
+    report_status(status, flags);
+  }
+}
+
+// (q - 1) * d for every weight, f32 out; one thread per 16 weights (one 32-bit word).
+__global__ void __launch_bounds__(256) q2_dequant_kernel(const uint8_t* __restrict__ wq,
+                                                         const uint16_t* __restrict__ d,
+                                                         float* __restrict__ w, int64_t n_words,
+                                                         int K) {
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  const int64_t words_per_row = K / 16;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n_words;
+       i += stride) {
+    const int64_t row = i / words_per_row;
+    const int64_t kw = (i % words_per_row) * 16;  // first k of this word
+    const uint32_t word = reinterpret_cast<const uint32_t*>(wq)[i];
+    const float dd = __half2float(__ushort_as_half(d[row * (K / 128) + kw / 128]));
+    float out[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      const int q = static_cast<int>((word >> (2 * j)) & 3u);
+      out[j] = static_cast<float>(q - 1) * dd;
+    }
+    float4* dst = reinterpret_cast<float4*>(w + row * K + kw);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) dst[j] = make_float4(out[4 * j], out[4 * j + 1], out[4 * j + 2], out[4 * j + 3]);
+  }
+}
+
+// (q - z) * s for every weight, two rounded f32 operations; one thread per 8 weights.
+__global__ void __launch_bounds__(256) q4_dequant_kernel(const uint8_t* __restrict__ wq,
+                                                         const uint16_t* __restrict__ sz,
+                                                         float* __restrict__ w, int64_t n_words,
+                                                         int K) {
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  const int64_t words_per_row = K / 8;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n_words;
+       i += stride) {
+    const int64_t row = i / words_per_row;
+    const int64_t t0 = (i % words_per_row) * 8;
+    const uint32_t word = reinterpret_cast<const uint32_t*>(wq)[i];
+    const uint32_t szw = reinterpret_cast<const uint32_t*>(sz)[row * (K / 64) + t0 / 64];
+    const float sc = __half2float(__ushort_as_half(static_cast<uint16_t>(szw & 0xFFFFu)));
+    const float ze = __half2float(__ushort_as_half(static_cast<uint16_t>(szw >> 16)));
+    float out[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const float q = static_cast<float>((word >> (4 * j)) & 15u);
+      out[j] = __fmul_rn(__fsub_rn(q, ze), sc);
+    }
+    float4* dst = reinterpret_cast<float4*>(w + row * K + t0);
+    dst[0] = make_float4(out[0], out[1], out[2], out[3]);
+    dst[1] = make_float4(out[4], out[5], out[6], out[7]);
+  }
+}
+
+}  // namespace tgemm

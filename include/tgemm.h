@@ -1,0 +1,187 @@
+/*
+ * tgemm.h -- C ABI of the B200 (sm_100a) ternary / 4-bit dequant-fused matmul library
+ * (libtgemm.so).
+ *
+ * What is computed (page title, section):
+ *   Q2_0 ternary weights -- "We're Teaching Your Browser to Paint: A 4B Image Model on
+ *     WebGPU", section "The lucky break that wasn't luck": blocks of 128 weights along
+ *     the input axis with one f16 scale d; 2-bit codes q in {0,1,2}, four per byte,
+ *     least-significant bits first; w = (q - 1) * d.  The converter's only rounding is
+ *     the scale's f32 -> f16 conversion, and it must round-trip exactly.
+ *   4-bit group weights -- "You Can Now Just Ask for an Image -- and Your Browser Draws
+ *     It", section "The bug that hid in one flipped bit": two codes per byte, code t of
+ *     a row is (byte[t/2] >> ((t & 1) * 4)) & 0xF (even index in the low nibble);
+ *     "We're Teaching...", section "What's left": w = (q - z) * s.
+ *   Low-rank side branch -- "mindview-t2i-turbo", section "One step": y = W x + B (A x).
+ *   Row slicing -- "We're Teaching...", section "The GPU driver, and the bug that looked
+ *     like broken math": quantized rows are independent byte runs, so rows [n0, n1) of a
+ *     packed matrix are the pointers wq + n0*K/4, d + n0*K/128 (Q2) or wq + n0*K/2,
+ *     sz + n0*(K/64)*2 (4-bit), with N = n1 - n0.
+ *
+ * Layouts (all row-major, the input axis K innermost):
+ *   x      bf16 bit patterns [M][K]                 activations
+ *   Q2:    wq  uint8 [N][K/4]     d  f16 [N][K/128]   (K a multiple of 128)
+ *   4-bit: wq  uint8 [N][K/2]     sz f16 [N][K/64][2], (s, z) per group of 64 (K % 64 == 0)
+ *   a      bf16 [r][K], b bf16 [N][r]                side-branch factors, 1 <= r <= 256
+ *   y      [M][N], f32 (TGEMM_OUT_F32) or bf16 (TGEMM_OUT_BF16, round to nearest even)
+ *   y[m][n] = sum_k w[n][k] * x[m][k]  (+ sum_i b[n][i] * sum_k a[i][k] * x[m][k])
+ *
+ * Ownership and memory: every pointer argument is a DEVICE pointer owned by the caller;
+ * the library keeps no reference after a call returns and allocates no device memory.
+ * Scratch space the matmuls need (an f16 copy of x for the tensor-core path, the side
+ * branch's A x) lives in a caller-provided workspace whose size tgemm_workspace_size()
+ * returns.
+ *
+ * Execution and errors: every call is asynchronous on `stream` (a cudaStream_t, or NULL
+ * for the legacy default stream).  The return value reports only what can be known on
+ * the host: argument checks and launch failures.  Results, pack status words and the
+ * device error word are valid once the stream has been synchronized.  No kernel traps:
+ * pack problems are reported through a status word, and a device-side wait that runs
+ * out of time sets a bit in the device error word (tgemm_device_error) and returns.
+ *
+ * Accuracy: the matmuls accumulate in f32.  The tensor-core path multiplies f16
+ * operands: x is converted bf16 -> f16 (exact for |x| in f16's normal range; x must be
+ * finite with |x| < 65504), Q2 weights (q-1)*d are exact in f16, 4-bit weights are the
+ * f16 rounding of (q - z) * s.
+ */
+#ifndef TGEMM_H
+#define TGEMM_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- status codes (return values) ------------------------------------------------ */
+#define TGEMM_OK          0
+#define TGEMM_EINVAL     -1 /* null pointer, non-positive size, K not a multiple of the
+                               block, r outside [1,256], unknown out_dtype/op/path */
+#define TGEMM_EALIGN     -2 /* a pointer is not aligned as documented for its argument */
+#define TGEMM_ECUDA      -3 /* a CUDA runtime call or kernel launch failed */
+#define TGEMM_EARCH      -4 /* the current device is not compute capability 10.0 */
+#define TGEMM_EWORKSPACE -5 /* workspace missing or smaller than tgemm_workspace_size() */
+
+/* ---- output element types ---------------------------------------------------------- */
+#define TGEMM_OUT_F32  0
+#define TGEMM_OUT_BF16 1
+
+/* ---- pack status bits (OR-ed into the caller's device status word) ----------------- */
+#define TGEMM_PACK_BAD_CODE  1u /* a Q2 code > 2 or a 4-bit code > 15 (stored masked) */
+#define TGEMM_PACK_INEXACT   2u /* a scale/zero is not exactly representable in f16 */
+#define TGEMM_PACK_NONFINITE 4u /* a scale/zero is inf or NaN */
+
+/* ---- device error word bits (tgemm_device_error) ----------------------------------- */
+#define TGEMM_DEVERR_TIMEOUT 1u /* a pipeline wait in a matmul kernel ran out of time */
+
+/* ---- operations, for tgemm_workspace_size ----------------------------------------- */
+#define TGEMM_OP_Q2      0
+#define TGEMM_OP_Q2_LORA 1
+#define TGEMM_OP_Q4      2
+
+/* ---- kernel path selection (tgemm_set_path) --------------------------------------- */
+#define TGEMM_PATH_AUTO    0 /* M <= 16: small-M kernel; otherwise the tensor-core kernel */
+#define TGEMM_PATH_SMALL_M 1 /* always the small-M (HBM-bound, mma.sync) kernel */
+#define TGEMM_PATH_TENSOR  2 /* always the tcgen05 tensor-core kernel */
+
+/*
+ * q2_pack -- Q2_0 packing ("We're Teaching...", "The lucky break that wasn't luck").
+ *   codes  uint8 [N][K], each in {0,1,2}             (16-byte aligned)
+ *   scale  f32   [N][K/128], the block scales         (4-byte aligned)
+ *   wq     uint8 [N][K/4]  out: code k of a row goes to bits 2*(k%4) of byte k/4 (16-byte aligned)
+ *   d      f16   [N][K/128] out: scale rounded to f16 (nearest even)  (2-byte aligned)
+ *   status uint32 device word, zeroed by the caller; receives TGEMM_PACK_* bits.  A code
+ *          above 2 is stored as (code & 3) and sets BAD_CODE; a scale whose f16 value
+ *          differs from it sets INEXACT (NONFINITE for inf/NaN).  A caller following the
+ *          pages aborts on any nonzero status.
+ *   Requires N >= 1, K >= 128, K % 128 == 0.
+ */
+int q2_pack(const uint8_t* codes, const float* scale, uint8_t* wq, uint16_t* d, int N, int K,
+            uint32_t* status, void* stream);
+
+/*
+ * q4_pack -- 4-bit packing ("You Can Now Just Ask...", "The bug that hid in one flipped bit").
+ *   codes  uint8 [N][K], each in 0..15               (16-byte aligned)
+ *   s, z   f32   [N][K/64], per-group scale and zero (4-byte aligned)
+ *   wq     uint8 [N][K/2] out: code t in the low nibble of byte t/2 when t is even, the
+ *          high nibble when t is odd                  (16-byte aligned)
+ *   sz     f16   [N][K/64][2] out: (s, z) rounded to f16 (4-byte aligned)
+ *   status as for q2_pack (BAD_CODE for codes > 15, stored as code & 15).
+ *   Requires N >= 1, K >= 64, K % 64 == 0.
+ */
+int q4_pack(const uint8_t* codes, const float* s, const float* z, uint8_t* wq, uint16_t* sz,
+            int N, int K, uint32_t* status, void* stream);
+
+/*
+ * q2_dequant / q4_dequant -- the weights a packed matrix stands for, in f32 [N][K]
+ * (16-byte aligned): (q - 1) * d, or (q - z) * s computed as two rounded f32 operations.
+ * Test hooks: they use the same unpacking as the matmul kernels.
+ */
+int q2_dequant(const uint8_t* wq, const uint16_t* d, float* w, int N, int K, void* stream);
+int q4_dequant(const uint8_t* wq, const uint16_t* sz, float* w, int N, int K, void* stream);
+
+/*
+ * tgemm_workspace_size -- bytes of workspace the matmul `op` (TGEMM_OP_*) needs for
+ * these sizes under the current path setting (0 when none).  r is ignored unless op is
+ * TGEMM_OP_Q2_LORA.  Returns 0 for invalid arguments as well; the matmul call then
+ * reports the argument error.
+ */
+size_t tgemm_workspace_size(int op, int M, int N, int K, int r);
+
+/*
+ * tgemm_q2 -- y = x . W^T for Q2_0 weights.
+ *   x [M][K] bf16 (16-byte aligned), wq [N][K/4] (16-byte aligned), d [N][K/128] f16
+ *   (2-byte aligned), y [M][N] (16-byte aligned), out_dtype TGEMM_OUT_*.
+ *   workspace: device memory of at least tgemm_workspace_size(TGEMM_OP_Q2, M, N, K, 0)
+ *   bytes (256-byte aligned; may be NULL when that size is 0).  The call overwrites it;
+ *   calls sharing a workspace must not overlap on the GPU.
+ *   Requires M, N >= 1, K % 128 == 0.
+ */
+int tgemm_q2(const uint16_t* x, const uint8_t* wq, const uint16_t* d, void* y, int M, int N,
+             int K, int out_dtype, void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * tgemm_q2_lora -- y = x . W^T + (x . A^T) . B^T ("mindview-t2i-turbo", "One step").
+ *   As tgemm_q2, plus a [r][K] bf16 (4-byte aligned) and b [N][r] bf16 (2-byte aligned),
+ *   1 <= r <= 256, and workspace of tgemm_workspace_size(TGEMM_OP_Q2_LORA, M, N, K, r).
+ *   The branch has no extra scale factor.  u = x . A^T is accumulated in f32; the
+ *   tensor-core path feeds it to the MMA as a bf16 pair (hi + lo) so that its rounding
+ *   error stays near 2^-16 relative.
+ */
+int tgemm_q2_lora(const uint16_t* x, const uint8_t* wq, const uint16_t* d, const uint16_t* a,
+                  const uint16_t* b, int r, void* y, int M, int N, int K, int out_dtype,
+                  void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * tgemm_q4 -- y = x . W^T for 4-bit group weights.
+ *   x [M][K] bf16 (16-byte aligned), wq [N][K/2] (16-byte aligned), sz [N][K/64][2] f16
+ *   (4-byte aligned), y [M][N] (16-byte aligned), workspace as for tgemm_q2 with
+ *   TGEMM_OP_Q4.  Requires M, N >= 1, K % 64 == 0.
+ */
+int tgemm_q4(const uint16_t* x, const uint8_t* wq, const uint16_t* sz, void* y, int M, int N,
+             int K, int out_dtype, void* workspace, size_t ws_bytes, void* stream);
+
+/* tgemm_strerror -- a static string describing a TGEMM_* status code. */
+const char* tgemm_strerror(int status);
+
+/*
+ * tgemm_set_path -- choose which matmul kernel runs (TGEMM_PATH_*); returns the previous
+ * setting, or TGEMM_EINVAL.  Process-wide; meant for tests and benchmarks.
+ */
+int tgemm_set_path(int path);
+
+/*
+ * tgemm_device_error -- synchronize the current device, copy its device error word
+ * (TGEMM_DEVERR_* bits, accumulated since load or the last clear) to *bits, and clear
+ * it if `clear` is nonzero.
+ */
+int tgemm_device_error(uint32_t* bits, int clear);
+
+/* tgemm_version -- library version, major * 10000 + minor * 100 + patch. */
+int tgemm_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* TGEMM_H */

@@ -1,0 +1,104 @@
+"""The C-ABI library builds, loads and exports what include/tgemm.h declares (no GPU).
+
+Only host-side behaviour is exercised here: symbol table, status strings, path switch,
+workspace sizes and the argument checks that return before any CUDA call.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+import bit_weight_quantized_tgemm_b200 as tg
+from bit_weight_quantized_tgemm_b200 import binding
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "tgemm.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\*?\s*([A-Za-z_][A-Za-z0-9_]*)\s*\(",
+                       src, flags=re.M)
+    return sorted(set(names))
+
+
+def test_library_exports_every_declared_symbol():
+    lib = tg.lib()
+    names = declared_functions()
+    assert len(names) >= 12
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in tgemm.h but not exported"
+
+
+def test_binding_knows_every_symbol():
+    assert set(declared_functions()) <= set(binding._SIGS)
+
+
+def test_strerror_and_version():
+    lib = tg.lib()
+    assert lib.tgemm_strerror(0) == b"success"
+    assert lib.tgemm_strerror(-5) == b"workspace missing or too small"
+    assert tg.version() >= 100
+
+
+def test_set_path_roundtrip():
+    prev = tg.set_path(tg.PATH_TENSOR)
+    assert tg.set_path(tg.PATH_SMALL_M) == tg.PATH_TENSOR
+    assert tg.set_path(prev) == tg.PATH_SMALL_M
+    assert tg.lib().tgemm_set_path(7) == tg.EINVAL
+
+
+def test_workspace_sizes():
+    prev = tg.set_path(tg.PATH_AUTO)
+    try:
+        assert tg.workspace_size(tg.OP_Q2, 16, 3072, 3072) == 0          # small-M path
+        assert tg.workspace_size(tg.OP_Q2, 1536, 9216, 3072) == 1536 * 3072 * 2
+        lora = tg.workspace_size(tg.OP_Q2_LORA, 1536, 9216, 3072, 64)
+        assert lora == 1536 * 3072 * 2 + 1536 * 128 * 2
+        assert tg.workspace_size(tg.OP_Q2_LORA, 4, 9216, 3072, 64) == 4 * 64 * 4  # f32 u
+        assert tg.workspace_size(tg.OP_Q2_LORA, 1536, 9216, 3072, 0) == 0  # invalid r
+        assert tg.workspace_size(9, 1, 1, 128) == 0
+    finally:
+        tg.set_path(prev)
+
+
+P = ctypes.c_void_p
+
+
+@pytest.mark.parametrize("call", [
+    lambda L: L.tgemm_q2(None, P(16), P(16), P(16), 4, 4, 128, 0, None, 0, None),
+    lambda L: L.tgemm_q2(P(16), P(16), P(16), P(16), 0, 4, 128, 0, None, 0, None),
+    lambda L: L.tgemm_q2(P(16), P(16), P(16), P(16), 4, 4, 100, 0, None, 0, None),
+    lambda L: L.tgemm_q2(P(16), P(16), P(16), P(16), 4, 4, 128, 5, None, 0, None),
+    lambda L: L.tgemm_q4(P(16), P(16), P(16), P(16), 4, 4, 96, 0, None, 0, None),
+    lambda L: L.tgemm_q2_lora(P(16), P(16), P(16), P(16), P(16), 0, P(16), 4, 4, 128, 0, None, 0, None),
+    lambda L: L.tgemm_q2_lora(P(16), P(16), P(16), P(16), P(16), 257, P(16), 4, 4, 128, 0, None, 0, None),
+    lambda L: L.q2_pack(P(16), P(16), P(16), P(16), 4, 64, P(16), None),
+    lambda L: L.q4_pack(P(16), P(16), P(16), P(16), P(16), 4, 32, P(16), None),
+    lambda L: L.q2_dequant(None, P(16), P(16), 4, 128, None),
+])
+def test_argument_errors_return_einval(call):
+    assert call(tg.lib()) == tg.EINVAL
+
+
+@pytest.mark.parametrize("call", [
+    lambda L: L.tgemm_q2(P(17), P(16), P(16), P(16), 4, 4, 128, 0, None, 0, None),
+    lambda L: L.tgemm_q2(P(16), P(24), P(16), P(16), 4, 4, 128, 0, None, 0, None),
+    lambda L: L.tgemm_q2(P(16), P(16), P(17), P(16), 4, 4, 128, 0, None, 0, None),
+    lambda L: L.tgemm_q4(P(16), P(16), P(18), P(16), 4, 4, 128, 0, None, 0, None),
+    lambda L: L.q2_pack(P(8), P(16), P(16), P(16), 4, 128, P(16), None),
+])
+def test_misaligned_pointers_return_ealign(call):
+    assert call(tg.lib()) == tg.EALIGN
+
+
+def test_missing_workspace_is_reported():
+    prev = tg.set_path(tg.PATH_TENSOR)
+    try:
+        st = tg.lib().tgemm_q2(P(256), P(256), P(256), P(256), 64, 64, 128, 0, None, 0, None)
+        assert st == tg.EWORKSPACE
+        st = tg.lib().tgemm_q2(P(256), P(256), P(256), P(256), 64, 64, 128, 0, P(256), 100, None)
+        assert st == tg.EWORKSPACE
+    finally:
+        tg.set_path(prev)
