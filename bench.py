@@ -1,0 +1,594 @@
+#!/usr/bin/env python3
+"""Benchmark: ternary / 4-bit dequant-fused matmuls on B200, one JSON line on stdout.
+
+A *step* is one pass of every matmul row of the hot path over one batch of synthetic
+input, shaped like one denoising step of the pages' 4B MMDiT plus the text encoder's
+4-bit linears and the small-M ternary GEMV:
+
+  mmdit_9216x3072, mmdit_3072x12288, mmdit_12288x3072   Q2_0, 1536 tokens (tensor cores)
+  lora_r4, lora_r32, lora_r64                           Q2_0 9216x3072 + rank-r branch
+  encoder_up (9728x2560), encoder_down (2560x9728)      4-bit, 512 tokens
+  gemv_m1, gemv_m4, gemv_m16                            Q2_0 3072x3072, M <= 16 (HBM-bound)
+
+``value`` is the step's algorithmic FLOPs (2*M*N*K, plus 2*M*r*(K+N) for the branch) per
+second of device time, over all ranks (weak scaling: every rank runs its own step).  L2
+is flushed (256 MB write) before every timed step, outside the step's events.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+For N > 1 launch one process per GPU with torch.distributed.run.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "ternary GEMM TFLOP/s and weight GB/s at 1 B200; % of tensor/HBM roofline"
+UNIT = "TFLOP/s"
+STEP_ORDER = ["mmdit_9216x3072", "gemv_m1", "gemv_m4", "gemv_m16", "mmdit_3072x12288",
+              "lora_r4", "lora_r32", "lora_r64", "mmdit_12288x3072", "encoder_up",
+              "encoder_down"]
+DOMINANT = ["mmdit_9216x3072", "mmdit_3072x12288", "mmdit_12288x3072"]
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "tc_gemm_q2_mmdit.md")
+TC_SOURCE = os.path.join(ROOT, "bit_weight_quantized_tgemm_b200", "csrc", "gemm_tc.cuh")
+
+
+def parse_args():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="CPU work for the oracle baseline sample (rank 0, N=1 only)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--only", default="",
+                    help="comma-separated subset of the step's matmuls (profiling runs)")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the end-to-end leg, the small-M stream and the CPU baseline")
+    return ap.parse_args()
+
+
+# ---- distributed plumbing ----------------------------------------------------------------
+
+def dist_setup(args):
+    import torch
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+def max_over_ranks(v: float, world: int) -> float:
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def dist_done(world):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.destroy_process_group()
+
+
+# ---- clocks during the timed region ---------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.rows = []
+        self.proc = None
+        self.t0 = self.t1 = None
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(gpu_index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.rows.append((time.time(), line.strip()))
+
+    def mark_start(self):
+        self.t0 = time.time()
+
+    def mark_end(self):
+        self.t1 = time.time()
+
+    def summary(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        inside = [r for (t, r) in self.rows if self.t0 is not None and self.t0 <= t <= self.t1 + 0.06]
+        if not inside:
+            inside = [r for (_, r) in self.rows[-3:]]
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in inside:
+            parts = [p.strip() for p in r.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---- the workload ------------------------------------------------------------------------
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "tflops_burst": d["bf16_tflops"],
+                "tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "tflops_burst": 1590.0, "tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+def ncu_traffic():
+    """Per-launch DRAM bytes of the tensor-core Q2 kernel from the committed ncu summary,
+    or None if there is none or the kernel source changed since it was taken."""
+    if not os.path.exists(TRAFFIC_FILE):
+        return None, None
+    want_sha = None
+    traffic = None
+    with open(TRAFFIC_FILE) as f:
+        for line in f:
+            if line.startswith("kernel_source_sha256:"):
+                want_sha = line.split(":", 1)[1].strip()
+            if line.startswith("traffic_bytes_per_launch_full:"):
+                traffic = float(line.split(":", 1)[1].strip())
+    with open(TC_SOURCE, "rb") as f:
+        sha = hashlib.sha256(f.read()).hexdigest()
+    if want_sha != sha:
+        return None, "kernel changed since the ncu capture"
+    return traffic, None
+
+
+class Op:
+    """One matmul of the step, its device buffers and a direct C-ABI call."""
+
+    def __init__(self, w, rank: int, tg, torch):
+        self.w = w
+        self.name = w.name
+        prob = w.make() if rank == 0 else _reseed(w, rank).make()
+        self.prob = prob
+        dev = torch.device("cuda")
+        self.x = _to_dev(prob.x, torch.bfloat16, torch)
+        M, N, K = w.M, w.N, w.K
+        if w.kind == "q4":
+            wq, sz, st = tg.q4_pack(torch.from_numpy(prob.codes).to(dev),
+                                    torch.from_numpy(prob.s).to(dev), torch.from_numpy(prob.z).to(dev))
+            self.wq, self.sc = wq, sz
+            self.op = tg.OP_Q4
+        else:
+            wq, d, st = tg.q2_pack(torch.from_numpy(prob.codes).to(dev),
+                                   torch.from_numpy(prob.scale).to(dev))
+            self.wq, self.sc = wq, d
+            self.op = tg.OP_Q2_LORA if w.kind == "q2_lora" else tg.OP_Q2
+        torch.cuda.synchronize()
+        if int(st.item()) != 0:
+            raise RuntimeError(f"{w.name}: pack status {int(st.item())}")
+        self.a = self.b = None
+        if w.kind == "q2_lora":
+            self.a = _to_dev(prob.a, torch.bfloat16, torch)
+            self.b = _to_dev(prob.b, torch.bfloat16, torch)
+        self.y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        self.flops = w.flops
+        self.weight_bytes = w.weight_bytes
+        self.ws_need = tg.workspace_size(self.op, M, N, K, w.r)
+        # host copies for the end-to-end leg
+        self.x_host = self.x.cpu().pin_memory()
+        self.y_host = torch.empty_like(self.y, device="cpu").pin_memory()
+
+    def bind(self, tg, ws, stream):
+        """Pre-compute the C call so a step costs one ctypes call per op."""
+        L = tg.lib()
+        w = self.w
+        wsp = ws.data_ptr() if ws is not None else None
+        wsn = ws.numel() if ws is not None else 0
+        if w.kind == "q4":
+            fn = L.tgemm_q4
+            args = (self.x.data_ptr(), self.wq.data_ptr(), self.sc.data_ptr(), self.y.data_ptr(),
+                    w.M, w.N, w.K, tg.OUT_BF16, wsp, wsn, stream)
+        elif w.kind == "q2_lora":
+            fn = L.tgemm_q2_lora
+            args = (self.x.data_ptr(), self.wq.data_ptr(), self.sc.data_ptr(), self.a.data_ptr(),
+                    self.b.data_ptr(), w.r, self.y.data_ptr(), w.M, w.N, w.K, tg.OUT_BF16, wsp,
+                    wsn, stream)
+        else:
+            fn = L.tgemm_q2
+            args = (self.x.data_ptr(), self.wq.data_ptr(), self.sc.data_ptr(), self.y.data_ptr(),
+                    w.M, w.N, w.K, tg.OUT_BF16, wsp, wsn, stream)
+        self._fn, self._args = fn, args
+
+    def __call__(self):
+        st = self._fn(*self._args)
+        if st != 0:
+            raise RuntimeError(f"{self.name}: status {st}")
+
+
+def _reseed(w, rank):
+    import dataclasses
+
+    return dataclasses.replace(w, seed=(w.seed, "rank", rank))
+
+
+def _to_dev(bits, dtype, torch):
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(dtype).cuda()
+
+
+# ---- CPU oracle baseline -------------------------------------------------------------------
+
+class OracleSampler:
+    """The CPU oracle on sampled outputs of the step's matmuls.
+
+    Outputs y[m, n] are drawn from every matmul in proportion to its FLOPs and computed
+    one at a time from the packed row (oracle.*_gemm_at); each counts 2*K FLOPs (plus the
+    branch's 2*r*(K+1) for the low-rank ops)."""
+
+    def __init__(self, items):
+        import oracle as orc
+
+        self.o = orc.get()
+        self.packed = []
+        for item in items:
+            w = item.w if hasattr(item, "w") else item
+            prob = item.prob if hasattr(item, "prob") else w.make()
+            if w.kind == "q4":
+                wq, sc, _ = self.o.q4_pack(prob.codes, prob.s, prob.z)
+            else:
+                wq, sc, _ = self.o.q2_pack(prob.codes, prob.scale)
+            self.packed.append((w, prob, wq, sc))
+        self.total = sum(w.flops for (w, *_) in self.packed)
+        self.per_sample = None  # seconds per unit of `scale`, from calibration
+
+    def _run(self, scale, rng):
+        o = self.o
+        flops = 0
+        n_out = 0
+        t0 = time.perf_counter()
+        for (w, prob, wq, sc) in self.packed:
+            n = max(1, int(round(scale * w.flops / self.total)))
+            mi = rng.integers(0, w.M, n)
+            ni = rng.integers(0, w.N, n)
+            if w.kind == "q4":
+                o.q4_gemm_at(prob.x, wq, sc, w.N, mi, ni)
+            elif w.kind == "q2_lora":
+                o.q2_gemm_at(prob.x, wq, sc, w.N, mi, ni, prob.a, prob.b)
+            else:
+                o.q2_gemm_at(prob.x, wq, sc, w.N, mi, ni)
+            flops += n * (2 * w.K + (2 * w.r * (w.K + 1) if w.r else 0))
+            n_out += n
+        return flops, time.perf_counter() - t0, n_out
+
+    def run(self, seconds: float, seed: int = 0):
+        rng = np.random.default_rng(seed)
+        if self.per_sample is None:
+            _, t, _ = self._run(200, rng)
+            self.per_sample = max(t, 1e-4) / 200
+        scale = max(50.0, seconds / self.per_sample)
+        f, t, n = self._run(scale, rng)
+        return {"flops": f, "seconds": t, "samples": n, "cores": self.o.num_threads()}
+
+
+def oracle_sample(items, seconds: float, seed: int = 0):
+    return OracleSampler(items).run(seconds, seed)
+
+
+def reference_arm(args, world, rank):
+    """The oracle as the reference arm: K timed steps, each a bounded sample."""
+    if rank != 0:
+        return
+    from bit_weight_quantized_tgemm_b200 import synth
+
+    sampler = OracleSampler([synth.ALL[n] for n in STEP_ORDER])
+    per_step = max(0.2, 90.0 / max(1, args.steps + args.warmup))
+    for i in range(args.warmup):
+        sampler.run(per_step, seed=1000 + i)
+    fl, sec, samples, cores = 0, 0.0, 0, 1
+    for i in range(args.steps):
+        r = sampler.run(per_step, seed=i + 1)
+        fl += r["flops"]
+        sec += r["seconds"]
+        samples += r["samples"]
+        cores = r["cores"]
+    value = fl / sec / 1e12
+    sample = (f"{samples} outputs y[m,n] over {args.steps} steps, drawn from the step's 11 "
+              f"matmuls in proportion to their FLOPs, each computed on its own by the CPU oracle")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * sec / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "mmdit_step (see bench.py docstring)", "sample": sample},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---- our arm -------------------------------------------------------------------------------
+
+def ours(args, world, rank, local):
+    import torch
+
+    import bit_weight_quantized_tgemm_b200 as tg
+    from bit_weight_quantized_tgemm_b200 import synth
+
+    tg.set_path(tg.PATH_AUTO)
+    torch.manual_seed(0)
+    names = [n for n in args.only.split(",") if n] or STEP_ORDER
+    for n in names:
+        if n not in synth.ALL:
+            raise SystemExit(f"unknown matmul {n!r}; choose from {', '.join(STEP_ORDER)}")
+    extras = not args.no_extras and not args.only
+    ops = [Op(synth.ALL[n], rank, tg, torch) for n in names]
+    ws_bytes = max(o.ws_need for o in ops)
+    ws = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream().cuda_stream
+    for o in ops:
+        o.bind(tg, ws, stream)
+    flush_buf = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")
+    step_flops = sum(o.flops for o in ops)
+    step_wbytes = sum(o.weight_bytes for o in ops)
+
+    def step():
+        for o in ops:
+            o()
+
+    # warm-up (also loads kernels, encodes nothing persistent)
+    for _ in range(args.warmup):
+        flush_buf.zero_()
+        step()
+    torch.cuda.synchronize()
+    if tg.device_error():
+        raise RuntimeError("device error after warm-up")
+
+    # ---- timed region: K steps, events around each step, L2 flushed before each
+    K = args.steps
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(K)]
+    for kind in range(6):
+        tg.profile_read(kind, reset=True)
+    clocks = ClockSampler(local)
+    time.sleep(0.3)
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks.mark_start()
+    launches0 = tg.launch_count()
+    tg.profile_enable(True)
+    for i in range(K):
+        flush_buf.zero_()
+        evs[i][0].record()
+        step()
+        evs[i][1].record()
+    torch.cuda.synchronize()
+    barrier(world)
+    clocks.mark_end()
+    tg.profile_enable(False)
+    launches = tg.launch_count() - launches0
+    step_ms_local = sum(a.elapsed_time(b) for a, b in evs) / K
+    step_ms = max_over_ranks(step_ms_local, world)
+    clk = clocks.summary()
+    prof = {k: tg.profile_read(k, reset=True) for k in range(6)}
+
+    # ---- dominant kernel roofline (tensor-core Q2 kernel, FLOP-weighted over its launches)
+    tc_ms, tc_n = prof[tg.KIND_TC_Q2]
+    dom_flops = sum(o.flops for o in ops if o.name in DOMINANT)
+    peaks = load_peaks()
+    timed_s = step_ms * K * 1e-3
+    peak = peaks["tflops_sustained"] if timed_s > 1.0 else peaks["tflops_burst"]
+    achieved = (dom_flops * K) / (tc_ms * 1e-3) / 1e12 if tc_ms > 0 else None
+    traffic, traffic_note = ncu_traffic()
+    roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": (achieved / peak) if achieved else None, "traffic": traffic,
+                "kernel": "tc_gemm_kernel<Q2> (1536 tokens; 9216x3072, 3072x12288, 12288x3072)",
+                "launches": tc_n,
+                "peak_source": f"MEASURED_PEAKS.json bf16 "
+                               f"{'sustained' if timed_s > 1.0 else 'burst'} (of {peaks['source']}); "
+                               "f16 operands run at the bf16 rate"}
+    if traffic_note:
+        roofline["traffic_note"] = traffic_note
+    gv_ms, gv_n = prof[tg.KIND_GEMV_Q2]
+    gv_bytes = sum(o.weight_bytes for o in ops if o.name.startswith("gemv")) * K
+    roofline_small_m = {"bound": "hbm", "unit": "GB/s", "peak": peaks["hbm_gbs"],
+                        "kernel": "gemv_kernel<Q2> (M=1,4,16; 3072x3072), packed-weight bytes",
+                        "achieved": gv_bytes / (gv_ms * 1e-3) / 1e9 if gv_ms else None}
+    if roofline_small_m["achieved"]:
+        roofline_small_m["frac"] = roofline_small_m["achieved"] / peaks["hbm_gbs"]
+
+    # ---- per-kind kernel time shares in the timed region
+    kinds = ["tc_q2", "tc_q2_lora", "tc_q4", "gemv_q2", "gemv_q4", "prep"]
+    kernel_time = {kinds[k]: {"ms_total": prof[k][0], "launches": prof[k][1]} for k in range(6)}
+
+    # ---- end-to-end through the C ABI with host buffers (pinned), copies inside the region
+    h2d = sum(o.x.numel() * 2 for o in ops)
+    d2h = sum(o.y.numel() * 2 for o in ops)
+    e2e_steps = max(5, min(K, 50)) if extras else 1
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    e0.record()
+    for _ in range(e2e_steps):
+        for o in ops:
+            o.x.copy_(o.x_host, non_blocking=True)
+            o()
+            o.y_host.copy_(o.y, non_blocking=True)
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world)
+
+    # ---- small-M stream: 64 distinct 3072x3072 weights (160 MB > L2), one graph of 64 GEMVs
+    parts = {}
+    if extras:
+        try:
+            parts["gemv_stream"] = gemv_stream(tg, torch, stream)
+        except Exception as exc:  # report, do not hide
+            parts["gemv_stream"] = {"error": str(exc)}
+
+    dev_err = tg.device_error()
+    cpu = None
+    if rank == 0 and world == 1 and extras and not args.no_cpu_baseline:
+        r = oracle_sample(ops, args.cpu_seconds)
+        cpu = {"value": r["flops"] / r["seconds"] / 1e12, "unit": UNIT, "cores": r["cores"],
+               "kind": "oracle",
+               "sample": f"{r['samples']} outputs y[m,n] drawn from the step's 11 matmuls in "
+                         f"proportion to their FLOPs, each computed on its own "
+                         f"({r['seconds']:.1f} s of CPU time)"}
+
+    value = world * step_flops / (step_ms * 1e-3) / 1e12
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f16", "data": "synthetic",
+        "config": {
+            "workload": "mmdit_step: 1536-token ternary 9216x3072, 3072x12288, 12288x3072; "
+                        "rank 4/32/64 branch on 9216x3072; 512-token 4-bit 9728x2560, "
+                        "2560x9728; 3072x3072 ternary GEMV at M=1,4,16",
+            "tokens": 1536, "encoder_tokens": 512, "out_dtype": "bf16",
+            "step_gflop": step_flops / 1e9, "step_weight_mb": step_wbytes / 1e6,
+            "l2": "flushed before every timed step (256 MB write, outside the step events)",
+            "parallelism": f"independent replicas x{world} (weak scaling, no collective)",
+        },
+        "weight_gbs": world * step_wbytes / (step_ms * 1e-3) / 1e9,
+        "e2e": {"value": world * step_flops / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": e2e_ms,
+                "how": "tgemm_* C-ABI calls with x copied from pinned host memory before and y "
+                       "copied back after each call, device-timed"},
+        "gpu_launches": launches,
+        "clocks": clk,
+        "roofline": roofline,
+        "roofline_small_m": roofline_small_m,
+        "kernel_time": kernel_time,
+        "parts": parts,
+        "device_error": dev_err,
+        "cpu_baseline": cpu,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def gemv_stream(tg, torch, stream):
+    """Back-to-back small-M calls over 64 distinct weight copies, replayed from a CUDA graph."""
+    N = K = 3072
+    copies = []
+    g = torch.Generator(device="cuda").manual_seed(123)
+    for _ in range(64):
+        codes = torch.randint(0, 3, (N, K), dtype=torch.uint8, device="cuda", generator=g)
+        scale = (torch.rand(N, K // 128, device="cuda", generator=g) * 0.02).half().float()
+        wq, d, _ = tg.q2_pack(codes, scale)
+        copies.append((wq, d))
+    out = {}
+    L = tg.lib()
+    for M in (1, 4, 16):
+        x = torch.randn(M, K, device="cuda").bfloat16()
+        y = torch.empty(M, N, device="cuda", dtype=torch.bfloat16)
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            sh = s.cuda_stream
+            calls = [(x.data_ptr(), wq.data_ptr(), d.data_ptr(), y.data_ptr(), M, N, K,
+                      tg.OUT_BF16, None, 0, sh) for (wq, d) in copies]
+            for c in calls[:4]:
+                assert L.tgemm_q2(*c) == 0
+            s.synchronize()
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph, stream=s):
+                for c in calls:
+                    L.tgemm_q2(*c)
+        torch.cuda.synchronize()
+        for _ in range(3):
+            graph.replay()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        reps = 20
+        a.record()
+        for _ in range(reps):
+            graph.replay()
+        b.record()
+        torch.cuda.synchronize()
+        per_call = a.elapsed_time(b) / (reps * len(calls)) * 1e-3
+        wbytes = N * K // 4 + N * (K // 128) * 2
+        out[f"m{M}"] = {"us_per_call": per_call * 1e6, "weight_gbs": wbytes / per_call / 1e9}
+        del graph
+    return out
+
+
+def main():
+    args = parse_args()
+    world, rank, local = (1, 0, 0)
+    if args.impl == "reference":
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        rank = int(os.environ.get("RANK", "0"))
+        reference_arm(args, world, rank)
+        return 0
+    world, rank, local = dist_setup(args)
+    try:
+        ours(args, world, rank, local)
+    finally:
+        dist_done(world)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -23,6 +23,7 @@ OP_Q2, OP_Q2_LORA, OP_Q4 = 0, 1, 2
 PATH_AUTO, PATH_SMALL_M, PATH_TENSOR = 0, 1, 2
 PACK_BAD_CODE, PACK_INEXACT, PACK_NONFINITE = 1, 2, 4
 DEVERR_TIMEOUT = 1
+KIND_TC_Q2, KIND_TC_Q2_LORA, KIND_TC_Q4, KIND_GEMV_Q2, KIND_GEMV_Q4, KIND_PREP = range(6)
 
 _P = ctypes.c_void_p
 _i = ctypes.c_int
@@ -41,6 +42,9 @@ _SIGS = {
     "tgemm_set_path": (_i, [_i]),
     "tgemm_device_error": (_i, [_P, _i]),
     "tgemm_version": (_i, []),
+    "tgemm_profile_enable": (_i, [_i]),
+    "tgemm_profile_read": (_i, [_i, _P, _P, _i]),
+    "tgemm_launch_count": (ctypes.c_int64, []),
 }
 
 
@@ -252,3 +256,22 @@ def device_error(clear: bool = False) -> int:
 
 def version() -> int:
     return int(lib().tgemm_version())
+
+
+def profile_enable(on: bool) -> bool:
+    """Record CUDA events around every launch (see tgemm_profile_enable)."""
+    return bool(lib().tgemm_profile_enable(1 if on else 0))
+
+
+def profile_read(kind: int, reset: bool = True):
+    """(total device ms, launches) recorded for kernel kind `kind` (KIND_*)."""
+    ms = ctypes.c_double(0.0)
+    n = ctypes.c_int64(0)
+    _check(lib().tgemm_profile_read(kind, ctypes.addressof(ms), ctypes.addressof(n),
+                                    1 if reset else 0), "tgemm_profile_read")
+    return float(ms.value), int(n.value)
+
+
+def launch_count() -> int:
+    """Kernels launched by libtgemm.so since it was loaded."""
+    return int(lib().tgemm_launch_count())

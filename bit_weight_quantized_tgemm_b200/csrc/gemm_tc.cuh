@@ -1,13 +1,19 @@
 // gemm_tc.cuh -- large-M path: persistent tcgen05 (5th-generation tensor core) kernel.
 //
-// Tile: 128 tokens (TMEM lanes) x 256 weight rows (accumulator columns) x 64 k per stage.
+// Tile: 128 weight rows (MMA M, TMEM lanes) x 256 tokens (MMA N, accumulator columns),
+// 64 k per stage.  Putting the weights on the 128-row side halves the dequantization
+// work per MMA flop compared with a 128-token tile: each stage dequantizes 128 x 64
+// codes for a 128x256x64 product.
 // Warp roles (14 warps, one CTA per SM):
-//   warp 0      TMA producer: activation tile (f16, 128-byte swizzle) + packed weight tile
+//   warp 0      TMA producer: activation tile, 256 tokens x 64 k (f16, 128-byte swizzle)
 //   warp 1      TMEM allocator and MMA issuer (one thread): 4 x tcgen05.mma 128x256x16
-//   warps 2-9   dequantizers: thread i owns weight row i of the tile; it unpacks its 64
-//               codes per stage, multiplies by the block scale in f16 and stores the row
-//               straight into the 128-byte-swizzled K-major operand layout
-//   warps 10-13 epilogue: tcgen05.ld of the f32 accumulator, convert, store y
+//   warps 2-9   dequantizers: warp pair (w, w+4) owns rows 32*(w%4).. of the tile, each
+//               thread half a row (32 codes) per stage; codes come straight from global
+//               memory (16 or 8 bytes per thread per stage, four stages ahead), are
+//               unpacked and scaled in f16 and stored in the 128-byte-swizzled K-major
+//               operand layout the MMA reads
+//   warps 10-13 epilogue: tcgen05.ld of the f32 accumulator (lane = weight row), convert,
+//               store y (lanes write consecutive n of one token row: coalesced)
 // The accumulator is double-buffered in TMEM (2 x 256 columns), so a tile's epilogue
 // overlaps the next tile's main loop.
 //
@@ -21,8 +27,8 @@
 // Both operands use the same permutation, so the contraction is unchanged.
 //
 // The low-rank branch y += (x A^T) B^T ("mindview-t2i-turbo", section "One step") runs as
-// extra pipeline stages after the main K loop: the A-operand stage holds u = x A^T as a
-// bf16 pair [hi | lo], the B-operand stage holds [B | B], and a bf16 MMA adds
+// extra pipeline stages after the main K loop: the weight-side stage holds [B | B], the
+// token-side stage holds u = x A^T as a bf16 pair [hi | lo], and a bf16 MMA adds
 // u_hi B^T + u_lo B^T into the same accumulator.
 #pragma once
 
@@ -30,24 +36,22 @@
 
 namespace tgemm {
 
-constexpr int kTcBM = 128;
-constexpr int kTcBN = 256;
+constexpr int kTcRows = 128;   // weight rows per tile (MMA M)
+constexpr int kTcTok = 256;    // tokens per tile (MMA N)
 constexpr int kTcBK = 64;
-constexpr int kTcStages = 4;
-constexpr int kTcWStages = 3;
+constexpr int kTcStages = 4;   // activation stages (TMA)
+constexpr int kTcWStages = 3;  // dequantized-weight stages
 constexpr int kTcThreads = 448;
-constexpr int kTcXBytes = kTcBM * kTcBK * 2;  // 16 KB
-constexpr int kTcWBytes = kTcBN * kTcBK * 2;  // 32 KB
+constexpr int kTcXBytes = kTcTok * kTcBK * 2;   // 32 KB
+constexpr int kTcWBytes = kTcRows * kTcBK * 2;  // 16 KB
 constexpr int kTcTmemCols = 512;
 
 template <int FMT>
 struct TcFmt {
   static constexpr int kWqRowBytes = FMT == 0 ? 16 : 32;  // packed bytes per row per stage
-  static constexpr int kWqStageBytes = kTcBN * kWqRowBytes;
   static constexpr int kXOff = 0;
   static constexpr int kWOff = kXOff + kTcStages * kTcXBytes;
-  static constexpr int kWqOff = kWOff + kTcWStages * kTcWBytes;
-  static constexpr int kBarOff = kWqOff + kTcStages * kWqStageBytes;
+  static constexpr int kBarOff = kWOff + kTcWStages * kTcWBytes;
   static constexpr int kNumBars = 2 * kTcStages + 2 * kTcWStages + 4 + 1;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kSmemBytes = kMiscOff + 16 + 1024;  // + alignment slack
@@ -62,7 +66,7 @@ struct TcParams {
   int R;           // round_up(r, 16): width of u_hi (and of u_lo) in the concatenation
   int r;
   int out_f32;
-  int vec_store;   // rows of y are 16-byte aligned
+  const uint8_t* wq;       // packed codes [N][K/4] (Q2) or [N][K/2] (4-bit)
   const uint16_t* scales;  // Q2: d [N][K/128]; 4-bit: sz [N][K/64][2]
   const uint16_t* lb;      // low-rank B [N][r] (bf16)
   void* y;
@@ -84,15 +88,6 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
                "r"(d)
                : "memory");
-}
-
-__device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
-  uint4 v;
-  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "r"(addr)
-               : "memory");
-  return v;
 }
 
 // Q2: 16 codes -> 8 f16x2 pairs (codes i, i+8) of (q - 1) * d.
@@ -117,15 +112,14 @@ __device__ __forceinline__ void q4_word_to_f16(uint32_t w, uint32_t s2, uint32_t
 template <int FMT, bool LORA>
 __global__ void __launch_bounds__(kTcThreads, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x,
-                   const __grid_constant__ CUtensorMap tm_w,
                    const __grid_constant__ CUtensorMap tm_u, const TcParams p) {
   using F = TcFmt<FMT>;
+  static_assert(F::kSmemBytes <= 232448, "shared memory budget");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const uint32_t sbase = smem_u32(smem);
   const uint32_t bar0 = sbase + F::kBarOff;
-  // barrier addresses
   auto full_bar = [&](int s) { return bar0 + 8u * s; };
   auto empty_bar = [&](int s) { return bar0 + 8u * (kTcStages + s); };
   auto wfull_bar = [&](int s) { return bar0 + 8u * (2 * kTcStages + s); };
@@ -140,8 +134,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kTcStages; ++s) {
-      mbar_init(full_bar(s), 1);
-      mbar_init(empty_bar(s), 1 + 8);  // MMA commit + 8 dequant warps
+      mbar_init(full_bar(s), 1);       // producer's expect_tx
+      mbar_init(empty_bar(s), 1);      // MMA commit
     }
     for (int s = 0; s < kTcWStages; ++s) {
       mbar_init(wfull_bar(s), 8);      // 8 dequant warps
@@ -157,7 +151,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   }
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tm_x);
-    tma_prefetch_desc(&tm_w);
     if (LORA) tma_prefetch_desc(&tm_u);
   }
   if (warp == 1) {
@@ -176,20 +169,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       uint32_t it = 0;
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
-        const int tm = tile % p.tiles_m, tn = tile / p.tiles_m;
+        const int tm = tile % p.tiles_m;
         for (int ks = 0; ks < ksteps; ++ks, ++it) {
           const uint32_t s = it % kTcStages, ph = (it / kTcStages) & 1u;
           if (!mbar_wait(empty_bar(s), ph ^ 1u, abort_flag)) { ok = false; break; }
           const uint32_t xdst = sbase + F::kXOff + s * kTcXBytes;
-          if (ks < p.kt_main) {
-            mbar_arrive_expect_tx(full_bar(s), kTcXBytes + F::kWqStageBytes);
-            tma_load_2d(xdst, &tm_x, full_bar(s), ks * kTcBK, tm * kTcBM);
-            tma_load_2d(sbase + F::kWqOff + s * F::kWqStageBytes, &tm_w, full_bar(s),
-                        ks * F::kWqRowBytes, tn * kTcBN);
-          } else {
-            mbar_arrive_expect_tx(full_bar(s), kTcXBytes);
-            tma_load_2d(xdst, &tm_u, full_bar(s), (ks - p.kt_main) * kTcBK, tm * kTcBM);
-          }
+          mbar_arrive_expect_tx(full_bar(s), kTcXBytes);
+          if (ks < p.kt_main)
+            tma_load_2d(xdst, &tm_x, full_bar(s), ks * kTcBK, tm * kTcTok);
+          else
+            tma_load_2d(xdst, &tm_u, full_bar(s), (ks - p.kt_main) * kTcBK, tm * kTcTok);
         }
       }
       // every load issued must land before the CTA may exit
@@ -200,23 +189,23 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t kIdescMain = make_idesc_f16(0u, kTcBM, kTcBN);  // f16 x f16
-      constexpr uint32_t kIdescLora = make_idesc_f16(1u, kTcBM, kTcBN);  // bf16 x bf16
+      constexpr uint32_t kIdescMain = make_idesc_f16(0u, kTcRows, kTcTok);  // f16 x f16
+      constexpr uint32_t kIdescLora = make_idesc_f16(1u, kTcRows, kTcTok);  // bf16 x bf16
       uint32_t it = 0, wit = 0, tcount = 0;
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x, ++tcount) {
         const uint32_t a = tcount & 1u, aph = (tcount >> 1) & 1u;
         if (!mbar_wait(accempty_bar(a), aph ^ 1u, abort_flag)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + a * kTcBN;
+        const uint32_t d_tmem = tmem_base + a * kTcTok;
         for (int ks = 0; ks < ksteps; ++ks, ++it, ++wit) {
           const uint32_t s = it % kTcStages, ph = (it / kTcStages) & 1u;
           const uint32_t ws = wit % kTcWStages, wph = (wit / kTcWStages) & 1u;
-          if (!mbar_wait(full_bar(s), ph, abort_flag)) { ok = false; break; }
           if (!mbar_wait(wfull_bar(ws), wph, abort_flag)) { ok = false; break; }
+          if (!mbar_wait(full_bar(s), ph, abort_flag)) { ok = false; break; }
           tc_fence_after();
-          const uint64_t adesc = smem_desc_sw128(sbase + F::kXOff + s * kTcXBytes);
-          const uint64_t bdesc = smem_desc_sw128(sbase + F::kWOff + ws * kTcWBytes);
+          const uint64_t adesc = smem_desc_sw128(sbase + F::kWOff + ws * kTcWBytes);  // weights
+          const uint64_t bdesc = smem_desc_sw128(sbase + F::kXOff + s * kTcXBytes);   // tokens
           if (!LORA || ks < p.kt_main) {
 #pragma unroll
             for (int kk = 0; kk < kTcBK / 16; ++kk)
@@ -239,78 +228,107 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
   } else if (warp < 10) {
     // ------------------------------------------------------------ dequantizers
-    const int dt = threadIdx.x - 64;  // weight row within the tile
-    const int swz = dt & 7;
-    const uint32_t row_off = static_cast<uint32_t>((dt >> 3) * 1024 + (dt & 7) * 128);
+    const int dw = warp - 2;
+    const int rt = 32 * (dw & 3) + lane;  // weight row within the tile
+    const int half = dw >> 2;             // which 32 codes of the stage's 64
+    const int swz = rt & 7;
+    const uint32_t row_off = static_cast<uint32_t>((rt >> 3) * 1024 + (rt & 7) * 128);
     const int nscale = FMT == 0 ? p.K / 128 : p.K / 64;
-    uint32_t it = 0, wit = 0;
+    const int64_t wq_row = FMT == 0 ? p.K / 4 : p.K / 2;
+    constexpr int kHalfBytes = F::kWqRowBytes / 2;  // 8 (Q2) or 16 (4-bit) bytes per stage
+    uint32_t wit = 0;
     bool ok = true;
     for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
       const int tn = tile / p.tiles_m;
-      const int row = tn * kTcBN + dt;
+      const int row = tn * kTcRows + rt;
       const bool valid = row < p.N;
       const uint16_t* srow = p.scales + static_cast<int64_t>(row) * nscale * (FMT == 0 ? 1 : 2);
-      // scale for the next block (Q2) / group (4-bit), loaded one step ahead
-      uint32_t nxt = 0;
-      if (valid) nxt = FMT == 0 ? static_cast<uint32_t>(srow[0])
-                                : *reinterpret_cast<const uint32_t*>(srow);
-      uint32_t cur = 0;
-      for (int ks = 0; ks < ksteps; ++ks, ++it, ++wit) {
-        const uint32_t s = it % kTcStages, ph = (it / kTcStages) & 1u;
-        if (!mbar_wait(full_bar(s), ph, abort_flag)) { ok = false; break; }
-        const bool main_stage = !LORA || ks < p.kt_main;
-        uint4 pk0 = make_uint4(0, 0, 0, 0), pk1 = make_uint4(0, 0, 0, 0);
-        if (main_stage) {
-          const uint32_t src = sbase + F::kWqOff + s * F::kWqStageBytes + dt * F::kWqRowBytes;
-          pk0 = ld_shared_v4(src);
-          if (FMT == 1) pk1 = ld_shared_v4(src + 16);
+      const uint8_t* wrow_g = p.wq + static_cast<int64_t>(row) * wq_row + half * kHalfBytes;
+      // block (Q2) / group (4-bit) scales, loaded four blocks ahead of their use
+      auto load_scale = [&](int b) -> uint32_t {
+        if (!valid || b >= nscale) return 0u;
+        return FMT == 0 ? static_cast<uint32_t>(srow[b])
+                        : reinterpret_cast<const uint32_t*>(srow)[b];
+      };
+      // this thread's packed codes for stage ks, loaded four stages ahead through L1
+      auto load_codes = [&](int ks) -> uint4 {
+        if (!valid || ks >= p.kt_main) return make_uint4(0, 0, 0, 0);
+        const uint8_t* src = wrow_g + static_cast<int64_t>(ks) * F::kWqRowBytes;
+        if (FMT == 0) {
+          const uint2 v = __ldg(reinterpret_cast<const uint2*>(src));
+          return make_uint4(v.x, v.y, 0, 0);
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(empty_bar(s));
+        return __ldg(reinterpret_cast<const uint4*>(src));
+      };
+      uint32_t q0 = load_scale(0), q1 = load_scale(1), q2 = load_scale(2), q3 = load_scale(3);
+      uint4 c0 = load_codes(0), c1 = load_codes(1), c2 = load_codes(2), c3 = load_codes(3);
+      uint32_t cur = 0;
+      for (int ks = 0; ks < ksteps; ++ks, ++wit) {
+        const uint4 pk = c0;
+        c0 = c1;
+        c1 = c2;
+        c2 = c3;
+        c3 = load_codes(ks + 4);
+        const bool main_stage = !LORA || ks < p.kt_main;
+        if (main_stage) {
+          const bool new_scale = FMT == 1 || (ks & 1) == 0;
+          if (new_scale) {
+            cur = q0;
+            q0 = q1;
+            q1 = q2;
+            q2 = q3;
+            q3 = load_scale((FMT == 0 ? (ks >> 1) : ks) + 4);
+          }
+        }
         const uint32_t ws = wit % kTcWStages, wph = (wit / kTcWStages) & 1u;
         if (!mbar_wait(wfree_bar(ws), wph ^ 1u, abort_flag)) { ok = false; break; }
         const uint32_t wrow = sbase + F::kWOff + ws * kTcWBytes + row_off;
         if (main_stage) {
           if (FMT == 0) {
-            if ((ks & 1) == 0) {
-              cur = nxt;
-              const int nb = (ks >> 1) + 1;
-              if (valid && nb < nscale) nxt = srow[nb];
-            }
             const uint32_t d2 = cur | (cur << 16);
-            const uint32_t words[4] = {pk0.x, pk0.y, pk0.z, pk0.w};
+            const uint32_t words[2] = {pk.x, pk.y};
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
+            for (int j = 0; j < 2; ++j) {
               uint32_t o[8];
               q2_word_to_f16(words[j], d2, o);
-              st_shared_v4(wrow + (((2 * j) ^ swz) << 4), o[0], o[1], o[2], o[3]);
-              st_shared_v4(wrow + (((2 * j + 1) ^ swz) << 4), o[4], o[5], o[6], o[7]);
+              const int ch = 4 * half + 2 * j;  // 16-byte chunk of the 128-byte row
+              st_shared_v4(wrow + ((ch ^ swz) << 4), o[0], o[1], o[2], o[3]);
+              st_shared_v4(wrow + (((ch + 1) ^ swz) << 4), o[4], o[5], o[6], o[7]);
             }
           } else {
-            cur = nxt;
-            if (valid && ks + 1 < nscale) nxt = reinterpret_cast<const uint32_t*>(srow)[ks + 1];
             const uint32_t s2 = (cur & 0xFFFFu) | (cur << 16);
             const uint32_t z2 = (cur >> 16) | (cur & 0xFFFF0000u);
-            const uint32_t words[8] = {pk0.x, pk0.y, pk0.z, pk0.w, pk1.x, pk1.y, pk1.z, pk1.w};
+            const uint32_t words[4] = {pk.x, pk.y, pk.z, pk.w};
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
+            for (int j = 0; j < 4; ++j) {
               uint32_t o[4];
               q4_word_to_f16(words[j], s2, z2, o);
-              st_shared_v4(wrow + ((j ^ swz) << 4), o[0], o[1], o[2], o[3]);
+              st_shared_v4(wrow + (((4 * half + j) ^ swz) << 4), o[0], o[1], o[2], o[3]);
             }
           }
         } else {
-          // low-rank stage: B-operand columns [jb, jb + 64) of [B | B], zero beyond 2R
+          // low-rank stage: weight-side columns [jb, jb + 64) of [B | B], zero beyond 2R;
+          // this thread fills 16-byte chunks 4*half .. 4*half+3 of its row
           const int jb = (ks - p.kt_main) * kTcBK;
+          const bool vec = (p.r & 7) == 0 && (reinterpret_cast<uintptr_t>(p.lb) & 15) == 0;
 #pragma unroll 1
-          for (int cc = 0; cc < 8; ++cc) {
+          for (int cq = 0; cq < 4; ++cq) {
+            const int cc = 4 * half + cq;
+            const int j0 = jb + 8 * cc;
+            const int i0 = j0 < p.R ? j0 : j0 - p.R;
+            if (vec && j0 < 2 * p.R && i0 + 8 <= p.r) {
+              uint4 v = make_uint4(0, 0, 0, 0);
+              if (valid) v = *reinterpret_cast<const uint4*>(p.lb + static_cast<int64_t>(row) * p.r + i0);
+              st_shared_v4(wrow + ((cc ^ swz) << 4), v.x, v.y, v.z, v.w);
+              continue;
+            }
             uint32_t o[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
               uint32_t v2 = 0;
 #pragma unroll
               for (int h = 0; h < 2; ++h) {
-                const int j = jb + 8 * cc + 2 * e + h;
+                const int j = j0 + 2 * e + h;
                 const int i = j < p.R ? j : j - p.R;
                 uint32_t v = 0;
                 if (valid && j < 2 * p.R && i < p.r) v = p.lb[static_cast<int64_t>(row) * p.r + i];
@@ -335,42 +353,26 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const uint32_t a = tcount & 1u, aph = (tcount >> 1) & 1u;
       if (!mbar_wait(accfull_bar(a), aph, abort_flag)) break;
       tc_fence_after();
-      const int m = tm * kTcBM + q * 32 + lane;
-      const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + a * kTcBN;
+      const int n = tn * kTcRows + q * 32 + lane;  // this thread's weight row
+      const bool nv = n < p.N;
+      const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + a * kTcTok;
 #pragma unroll 1
-      for (int cc = 0; cc < kTcBN / 32; ++cc) {
+      for (int cc = 0; cc < kTcTok / 32; ++cc) {
         uint32_t v[32];
         tmem_ld_32x32b_x32(tbase + cc * 32, v);
         tmem_wait_ld();
-        const int n0 = tn * kTcBN + cc * 32;
-        if (m < p.M && n0 < p.N) {
-          const int64_t off = static_cast<int64_t>(m) * p.N + n0;
+        const int m0 = tm * kTcTok + cc * 32;
+        if (nv && m0 < p.M) {
           if (p.out_f32) {
-            float* dst = reinterpret_cast<float*>(p.y) + off;
-            if (p.vec_store && n0 + 32 <= p.N) {
+            float* dst = reinterpret_cast<float*>(p.y) + static_cast<int64_t>(m0) * p.N + n;
 #pragma unroll
-              for (int e = 0; e < 8; ++e)
-                reinterpret_cast<uint4*>(dst)[e] = make_uint4(v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]);
-            } else {
-#pragma unroll
-              for (int e = 0; e < 32; ++e)
-                if (n0 + e < p.N) dst[e] = __uint_as_float(v[e]);
-            }
+            for (int e = 0; e < 32; ++e)
+              if (m0 + e < p.M) dst[static_cast<int64_t>(e) * p.N] = __uint_as_float(v[e]);
           } else {
-            uint32_t b[16];
+            __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.y) + static_cast<int64_t>(m0) * p.N + n;
 #pragma unroll
-            for (int e = 0; e < 16; ++e)
-              b[e] = pack_bf16x2(__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1]));
-            uint16_t* dst = reinterpret_cast<uint16_t*>(p.y) + off;
-            if (p.vec_store && n0 + 32 <= p.N) {
-#pragma unroll
-              for (int e = 0; e < 4; ++e)
-                reinterpret_cast<uint4*>(dst)[e] = make_uint4(b[4 * e], b[4 * e + 1], b[4 * e + 2], b[4 * e + 3]);
-            } else {
-#pragma unroll
-              for (int e = 0; e < 32; ++e)
-                if (n0 + e < p.N) dst[e] = static_cast<uint16_t>(b[e >> 1] >> (16 * (e & 1)));
-            }
+            for (int e = 0; e < 32; ++e)
+              if (m0 + e < p.M) dst[static_cast<int64_t>(e) * p.N] = __float2bfloat16_rn(__uint_as_float(v[e]));
           }
         }
       }
@@ -426,20 +428,26 @@ __global__ void __launch_bounds__(256) prep_x16_kernel(const uint16_t* __restric
   }
 }
 
-// u = x A^T for the low-rank branch, f32 accumulation on mma.sync.  CTA: 16 tokens x up
-// to 64 branch columns (blockIdx.y picks the column chunk); its 8 warps split K and
-// reduce through shared memory.  Writes u in f32 [M][r] (small-M path) and/or the
-// concatenation ucat [M][wcat] = [bf16(u) pad R | bf16(u - bf16(u)) pad R | 0].
-__global__ void __launch_bounds__(256) lora_down_kernel(const uint16_t* __restrict__ x,
-                                                        const uint16_t* __restrict__ a, int M,
-                                                        int K, int r, int R, int wcat,
-                                                        float* __restrict__ u32,
-                                                        uint16_t* __restrict__ ucat) {
+// u = x A^T for the low-rank branch, in two deterministic phases (no atomics).
+// Phase 1 (lora_down_partial_kernel): CTA (token block of 16, K slice of kLoraKc, column
+// chunk of 64) accumulates its slice on mma.sync (bf16 in, f32 accumulate); its 8 warps
+// split the slice and reduce through shared memory; the partial lands in
+// part[slice][m][col] (f32, `rpad` columns per row).
+// Phase 2 (lora_finalize_kernel): sums the slices in a fixed order and writes u in f32
+// [M][r] (small-M path) and/or the concatenation ucat [M][wcat] =
+// [bf16(u) pad R | bf16(u - bf16(u)) pad R | 0] (tensor-core path).
+constexpr int kLoraKc = 512;
+
+__global__ void __launch_bounds__(256) lora_down_partial_kernel(
+    const uint16_t* __restrict__ x, const uint16_t* __restrict__ a, int M, int K, int r,
+    int rpad, float* __restrict__ part) {
   __shared__ float red[8][16][65];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, c = lane & 3;
   const int m0 = blockIdx.x * 16;
-  const int col0 = blockIdx.y * 64;
+  const int k_lo = blockIdx.y * kLoraKc;
+  const int k_hi = min(K, k_lo + kLoraKc);
+  const int col0 = blockIdx.z * 64;
   float acc[8][4];
 #pragma unroll
   for (int t = 0; t < 8; ++t)
@@ -448,25 +456,29 @@ __global__ void __launch_bounds__(256) lora_down_kernel(const uint16_t* __restri
   const uint32_t* x32 = reinterpret_cast<const uint32_t*>(x);
   const uint32_t* a32 = reinterpret_cast<const uint32_t*>(a);
   const int kw = K / 2;  // 32-bit words per row
-  for (int kb = warp; kb < K / 16; kb += 8) {
+  const bool r0 = m0 + g < M, r1 = m0 + g + 8 < M;
+#pragma unroll 2
+  for (int kb = k_lo / 16 + warp; kb < k_hi / 16; kb += 8) {
     const int k2 = kb * 8 + c;  // word index of (k = 16kb + 2c, +1)
-    const bool r0 = m0 + g < M, r1 = m0 + g + 8 < M;
     const uint32_t a0 = r0 ? __ldg(x32 + static_cast<int64_t>(m0 + g) * kw + k2) : 0u;
     const uint32_t a1 = r1 ? __ldg(x32 + static_cast<int64_t>(m0 + g + 8) * kw + k2) : 0u;
     const uint32_t a2 = r0 ? __ldg(x32 + static_cast<int64_t>(m0 + g) * kw + k2 + 4) : 0u;
     const uint32_t a3 = r1 ? __ldg(x32 + static_cast<int64_t>(m0 + g + 8) * kw + k2 + 4) : 0u;
+    uint32_t b[8][2];
 #pragma unroll
     for (int t = 0; t < 8; ++t) {
       const int col = col0 + 8 * t + g;
       const bool cv = col < r;
-      const uint32_t b0 = cv ? __ldg(a32 + static_cast<int64_t>(col) * kw + k2) : 0u;
-      const uint32_t b1 = cv ? __ldg(a32 + static_cast<int64_t>(col) * kw + k2 + 4) : 0u;
+      b[t][0] = cv ? __ldg(a32 + static_cast<int64_t>(col) * kw + k2) : 0u;
+      b[t][1] = cv ? __ldg(a32 + static_cast<int64_t>(col) * kw + k2 + 4) : 0u;
+    }
+#pragma unroll
+    for (int t = 0; t < 8; ++t)
       asm volatile(
           "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
           "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
           : "+f"(acc[t][0]), "+f"(acc[t][1]), "+f"(acc[t][2]), "+f"(acc[t][3])
-          : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-    }
+          : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b[t][0]), "r"(b[t][1]));
   }
 #pragma unroll
   for (int t = 0; t < 8; ++t) {
@@ -479,29 +491,44 @@ __global__ void __launch_bounds__(256) lora_down_kernel(const uint16_t* __restri
   for (int o = threadIdx.x; o < 16 * 64; o += blockDim.x) {
     const int mm = o >> 6, cc = o & 63;
     const int m = m0 + mm, col = col0 + cc;
-    if (m >= M) continue;
+    if (m >= M || col >= rpad) continue;
     float v = 0.f;
 #pragma unroll
     for (int w = 0; w < 8; ++w) v += red[w][mm][cc];
-    if (u32 != nullptr && col < r) u32[static_cast<int64_t>(m) * r + col] = v;
-    if (ucat != nullptr && col < R) {
-      uint16_t hi = 0, lo = 0;
-      if (col < r) {
-        const __nv_bfloat16 h = __float2bfloat16_rn(v);
-        hi = __bfloat16_as_ushort(h);
-        lo = __bfloat16_as_ushort(__float2bfloat16_rn(v - __bfloat162float(h)));
-      }
-      ucat[static_cast<int64_t>(m) * wcat + col] = hi;
-      ucat[static_cast<int64_t>(m) * wcat + R + col] = lo;
-    }
+    part[(static_cast<int64_t>(blockIdx.y) * M + m) * rpad + col] = v;
   }
-  // zero the concatenation's tail [2R, wcat)
-  if (ucat != nullptr && blockIdx.y == 0) {
-    const int tail = wcat - 2 * R;
-    for (int o = threadIdx.x; o < 16 * tail; o += blockDim.x) {
-      const int m = m0 + o / tail;
-      if (m < M) ucat[static_cast<int64_t>(m) * wcat + 2 * R + o % tail] = 0;
+}
+
+__global__ void __launch_bounds__(256) lora_finalize_kernel(const float* __restrict__ part,
+                                                            int slices, int M, int r, int rpad,
+                                                            int R, int wcat,
+                                                            float* __restrict__ u32,
+                                                            uint16_t* __restrict__ ucat) {
+  const int64_t total = static_cast<int64_t>(M) * wcat;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+       i < (ucat ? total : static_cast<int64_t>(M) * r); i += stride) {
+    if (ucat == nullptr) {
+      const int64_t m = i / r, col = i % r;
+      float v = 0.f;
+      for (int sl = 0; sl < slices; ++sl) v += part[(sl * static_cast<int64_t>(M) + m) * rpad + col];
+      u32[i] = v;
+      continue;
     }
+    const int64_t m = i / wcat;
+    const int j = static_cast<int>(i % wcat);
+    uint16_t out = 0;
+    if (j < 2 * R) {
+      const int col = j < R ? j : j - R;
+      if (col < r) {
+        float v = 0.f;
+        for (int sl = 0; sl < slices; ++sl) v += part[(sl * static_cast<int64_t>(M) + m) * rpad + col];
+        const __nv_bfloat16 h = __float2bfloat16_rn(v);
+        out = j < R ? __bfloat16_as_ushort(h)
+                    : __bfloat16_as_ushort(__float2bfloat16_rn(v - __bfloat162float(h)));
+      }
+    }
+    ucat[i] = out;
   }
 }
 

@@ -1,17 +1,24 @@
 // gemv.cuh -- small-M path (M <= 16 tokens per pass): HBM-bound on the packed weights.
 //
-// Each CTA owns 32 weight rows (four 8-row n-blocks) and all K; its 8 warps split K in
-// units of 128 weights.  Per unit, a lane loads its share of the packed rows straight
-// from HBM with 8- or 16-byte loads (all of a pass's loads are issued before any is
-// used), unpacks the codes in registers into bf16 mma.sync fragments and multiplies them
-// with the activations held in shared memory.  Block scales are applied to the f32
-// partial sums after each unit, so the tensor cores see small exact integers:
+// Each CTA owns 32 weight rows (four 8-row n-blocks); its 8 warps split K in units of
+// 128 weights.  Per pass of up to kGvKP weights along K:
+//   * one thread copies the pass's activation rows into shared memory with bulk async
+//     copies (cp.async.bulk, completion on an mbarrier), while
+//   * every lane issues all of its packed-weight loads for the pass (8- or 16-byte loads
+//     straight from HBM into registers),
+// so the pass costs one memory round trip.  Codes are unpacked in registers into bf16
+// mma.sync fragments and multiplied with the activations; block scales are applied to
+// the f32 partial sums after each block, so the tensor cores see small exact integers:
 //   Q2_0:  B = q - 1 in {-1, 0, 1}, then y += d * sum          (one 128-weight block)
 //   4-bit: B = q in 0..15, S = sum of x over the group (an extra mma against ones),
 //          then y += s * (sum - z * S)                          (two 64-weight groups)
 // which equals sum_k (q - 1) d x  and  sum_k (q - z) s x  with only f32 rounding.
 // The warps' partial sums are reduced through shared memory; the optional low-rank
-// branch adds sum_i B[n][i] u[m][i] (u = A x in f32, computed by lora_down_kernel).
+// branch adds sum_i B[n][i] u[m][i] (u = A x in f32, from the lora kernels).
+//
+// Fragment order: a 32-bit word of Q2 codes unpacks with one shift and mask per pair
+// into codes (i, i+8); a word of 4-bit codes into codes (i, i+4).  The matching
+// activation pairs are gathered from shared memory with two 16-bit loads.
 #pragma once
 
 #include "common.cuh"
@@ -21,9 +28,13 @@ namespace tgemm {
 constexpr int kGvRows = 32;         // weight rows per CTA
 constexpr int kGvWarps = 8;         // warps per CTA, splitting K
 constexpr int kGvUnit = 128;        // K per unit
-constexpr int kGvMaxU = 4;          // units per warp per pass (weights held in registers)
-constexpr int kGvSub = kGvWarps;    // units per X sub-chunk (one per warp)
-constexpr int kGvRowWords = kGvSub * 64 + 4;  // X words per token row in smem (+4 pad)
+constexpr int kGvKP = 4096;         // K per pass (activations staged in shared memory)
+constexpr int kGvMaxU = kGvKP / kGvUnit / kGvWarps;  // units per warp per pass (4)
+
+__host__ __device__ constexpr int gemv_row_stride_bytes(int kp) { return 2 * kp + 16; }
+__host__ __device__ constexpr int gemv_smem_bytes(int mrows, int kp) {
+  return mrows * gemv_row_stride_bytes(kp) + 16;
+}
 
 // mma.sync m16n8k16, bf16 inputs, f32 accumulate.
 __device__ __forceinline__ void mma_bf16_16816(float (&c)[4], uint32_t a0, uint32_t a1,
@@ -55,102 +66,88 @@ __device__ __forceinline__ uint32_t q4_pair_bf16(uint32_t w, int s) {
   return bsub2(t, 0x43004300u);                                       // - 128
 }
 
-// Activation staging.  For one unit (128 k) of one token row the 64 words hold bf16
-// pairs in the order the fragments want them, lane-minor so a warp's 32 loads of one
-// fragment register hit 32 different banks (row stride = 516 words = 4 mod 32):
-//   Q2:   word ((j*4 + p)*2 + h)*4 + c = (x[32c+16j+p+4h], x[32c+16j+p+4h+8])
-//   4-bit word (kb*2 + hh)*4 + c       = (x[k1+hh], x[k1+hh+4]),
-//         k1 = 64*(kb/4) + 16c + 8*((kb%4)/2) + 2*(kb%2)
-// (j, p: word and pair of a Q2 lane's codes; kb: mma k-block; c = lane % 4).
-template <int FMT>
-__device__ __forceinline__ void stage_x_subchunk(uint32_t* xs, const uint16_t* __restrict__ x,
-                                                 int M, int K, int m0, int k0) {
-  // 16 rows x (kGvSub*128) k; thread handles 16 consecutive k of one row per step
-  constexpr int kGroupsPerRow = kGvSub * kGvUnit / 16;
-  for (int it = threadIdx.x; it < 16 * kGroupsPerRow; it += blockDim.x) {
-    const int row = it / kGroupsPerRow;
-    const int gi = it % kGroupsPerRow;  // 16-k group within the sub-chunk
-    const int m = m0 + row;
-    const int k = k0 + gi * 16;
-    uint32_t v[8];
-    if (m < M && k < K) {
-      const uint4* src = reinterpret_cast<const uint4*>(x + static_cast<int64_t>(m) * K + k);
-      const uint4 a = __ldg(src), b = __ldg(src + 1);
-      v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
-      v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
-    } else {
-#pragma unroll
-      for (int i = 0; i < 8; ++i) v[i] = 0u;
-    }
-    // element e of the group = half (e & 1) of v[e >> 1]
-    auto el = [&](int e) -> uint32_t { return (v[e >> 1] >> (16 * (e & 1))) & 0xFFFFu; };
-    uint32_t* rowp = xs + row * kGvRowWords + (gi / 8) * 64;  // unit base
-    const int gu = gi % 8;                                     // 16-group within the unit
-    if (FMT == 0) {
-      const int c = gu >> 1, j = gu & 1;
-#pragma unroll
-      for (int p = 0; p < 4; ++p)
-#pragma unroll
-        for (int h = 0; h < 2; ++h)
-          rowp[((j * 4 + p) * 2 + h) * 4 + c] = el(p + 4 * h) | (el(p + 4 * h + 8) << 16);
-    } else {
-      // two 8-groups: 8-group index within the unit G8 = 2*gu + e8
-#pragma unroll
-      for (int e8 = 0; e8 < 2; ++e8) {
-        const int G8 = 2 * gu + e8;          // = 8*h2 + 2c + jj
-        const int h2 = G8 >> 3, c = (G8 >> 1) & 3, jj = G8 & 1;
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {   // kb % 2
-          const int kb = 4 * h2 + 2 * jj + half;
-          const int i0 = 2 * half;
-#pragma unroll
-          for (int hh = 0; hh < 2; ++hh)
-            rowp[(kb * 2 + hh) * 4 + c] =
-                el(8 * e8 + i0 + hh) | (el(8 * e8 + i0 + hh + 4) << 16);
-        }
-      }
-    }
-  }
+__device__ __forceinline__ uint32_t lds_u16(uint32_t addr) {
+  uint16_t v;
+  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(addr));
+  return v;
+}
+
+// (x[k_lo], x[k_hi]) of one staged row as a bf16x2 fragment register.
+__device__ __forceinline__ uint32_t x_pair(uint32_t row_addr, int k_lo, int k_hi) {
+  return lds_u16(row_addr + 2 * k_lo) | (lds_u16(row_addr + 2 * k_hi) << 16);
+}
+
+__device__ __forceinline__ void bulk_copy_g2s(uint32_t dst, const void* src, uint32_t bytes,
+                                              uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+      : "memory");
 }
 
 template <int FMT, bool LORA>
 __global__ void __launch_bounds__(256) gemv_kernel(
     const uint16_t* __restrict__ x, const uint8_t* __restrict__ wq,
     const uint16_t* __restrict__ scales, void* __restrict__ y, int M, int N, int K, int out_f32,
-    const float* __restrict__ u, const uint16_t* __restrict__ lb, int r) {
-  __shared__ uint32_t xs[16 * kGvRowWords];
-  // the warps' partial sums reuse the activation buffer once a token tile is done
-  static_assert(sizeof(float) * kGvWarps * 16 * (kGvRows + 1) <= sizeof(uint32_t) * 16 * kGvRowWords,
-                "reduction buffer must fit in the staging buffer");
-  auto red = reinterpret_cast<float (*)[16][kGvRows + 1]>(xs);
+    const float* __restrict__ u, const uint16_t* __restrict__ lb, int r, int mrows, int kp) {
+  extern __shared__ __align__(16) uint8_t gv_smem[];
+  __shared__ float red[kGvWarps][16][kGvRows + 1];
+  // scales of this CTA's rows for one pass: Q2 d per unit, 4-bit (s, z) per group
+  constexpr int kScl = FMT == 0 ? kGvKP / 128 : kGvKP / 64;
+  __shared__ uint32_t scl[kGvRows][kScl];
+  __shared__ uint32_t abort_flag;
+  const uint32_t xs = smem_u32(gv_smem);
+  const int rs = gemv_row_stride_bytes(kp);
+  const uint32_t bar = xs + mrows * rs;  // 8-byte aligned: rs and the base are 16-aligned
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, c = lane & 3;
   const int n0 = blockIdx.x * kGvRows;
-  const int nunits = (K + kGvUnit - 1) / kGvUnit;
+  const int nunits = K / kGvUnit + ((K % kGvUnit) ? 1 : 0);
   constexpr int kUnitBytes = FMT == 0 ? 32 : 64;   // packed bytes of one row per unit
   constexpr int kWords = FMT == 0 ? 2 : 4;         // 32-bit words a lane loads per row per unit
   const int64_t row_bytes = FMT == 0 ? K / 4 : K / 2;
   const int nscale = FMT == 0 ? K / 128 : K / 64;  // scale entries per row
 
+  if (threadIdx.x == 0) {
+    mbar_init(bar, 1);
+    abort_flag = 0u;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  uint32_t phase = 0;
+
   for (int m0 = 0; m0 < M; m0 += 16) {
+    const int mt = min(16, M - m0);  // tokens in this tile (<= mrows)
     float acc[4][4];
 #pragma unroll
     for (int j = 0; j < 4; ++j)
 #pragma unroll
       for (int e = 0; e < 4; ++e) acc[j][e] = 0.f;
 
-    for (int pass_u = 0; pass_u < nunits; pass_u += kGvSub * kGvMaxU) {
-      // ---- issue every weight load of this pass --------------------------------------
+    for (int k0 = 0; k0 < K; k0 += kp) {
+      const int kpass = min(kp, K - k0);
+      // ---- activations for this pass: one bulk copy per token row
+      if (threadIdx.x == 0) {
+        fence_proxy_async_smem();
+        mbar_arrive_expect_tx(bar, static_cast<uint32_t>(mt * kpass * 2));
+        for (int i = 0; i < mt; ++i)
+          bulk_copy_g2s(xs + i * rs, x + static_cast<int64_t>(m0 + i) * K + k0,
+                        static_cast<uint32_t>(kpass * 2), bar);
+      }
+      // ---- every packed-weight load of this pass
+      const int u_base = k0 / kGvUnit;
+      const int u_end = min(nunits, (k0 + kpass + kGvUnit - 1) / kGvUnit);
       uint32_t wreg[kGvMaxU][4][kWords];
 #pragma unroll
       for (int i = 0; i < kGvMaxU; ++i) {
-        const int unit = pass_u + i * kGvSub + warp;
+        const int unit = u_base + i * kGvWarps + warp;
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           const int row = n0 + 8 * j + g;
-          const bool ok = unit < nunits && row < N;
-          const uint8_t* base = wq + static_cast<int64_t>(row) * row_bytes + static_cast<int64_t>(unit) * kUnitBytes;
+          const bool ok = unit < u_end && row < N;
+          const uint8_t* base = wq + static_cast<int64_t>(row) * row_bytes +
+                                static_cast<int64_t>(unit) * kUnitBytes;
           if (FMT == 0) {
             uint2 v = make_uint2(0x55555555u, 0x55555555u);  // code 1 everywhere = weight 0
             if (ok) v = __ldg(reinterpret_cast<const uint2*>(base + 8 * c));
@@ -170,18 +167,33 @@ __global__ void __launch_bounds__(256) gemv_kernel(
           }
         }
       }
-      // ---- consume them sub-chunk by sub-chunk ---------------------------------------
+      // ---- this pass's scales for the CTA's rows, staged in shared memory
+      {
+        const int s_base = FMT == 0 ? u_base : 2 * u_base;
+        const int s_cnt = FMT == 0 ? (u_end - u_base) : min(nscale - s_base, 2 * (u_end - u_base));
+        for (int it = threadIdx.x; it < kGvRows * s_cnt; it += blockDim.x) {
+          const int rl = it / s_cnt, si = it % s_cnt;
+          const int n = n0 + rl;
+          uint32_t v = 0;
+          if (n < N) {
+            const int64_t idx = static_cast<int64_t>(n) * nscale + s_base + si;
+            v = FMT == 0 ? static_cast<uint32_t>(scales[idx])
+                         : reinterpret_cast<const uint32_t*>(scales)[idx];
+          }
+          scl[rl][si] = v;
+        }
+      }
+      // ---- wait for the activations (bounded; the CTA leaves together on a timeout)
+      const bool ok = mbar_wait(bar, phase, &abort_flag);
+      if (__syncthreads_or(!ok)) return;
+      phase ^= 1u;
+      const bool g0 = g < mt, g1 = g + 8 < mt;
+      const uint32_t row0 = xs + g * rs, row1 = xs + (g + 8) * rs;
 #pragma unroll
       for (int i = 0; i < kGvMaxU; ++i) {
-        const int sub_u = pass_u + i * kGvSub;
-        if (sub_u >= nunits) break;
-        __syncthreads();  // previous readers of xs are done
-        stage_x_subchunk<FMT>(xs, x, M, K, m0, sub_u * kGvUnit);
-        __syncthreads();
-        const int unit = sub_u + warp;
-        if (unit >= nunits) continue;
-        const uint32_t* xrow0 = xs + g * kGvRowWords + warp * 64;
-        const uint32_t* xrow1 = xs + (g + 8) * kGvRowWords + warp * 64;
+        const int unit = u_base + i * kGvWarps + warp;
+        if (unit >= u_end) break;
+        const int ku = (unit - u_base) * kGvUnit;  // unit offset within the pass
         if (FMT == 0) {
           float part[4][4];
 #pragma unroll
@@ -191,8 +203,11 @@ __global__ void __launch_bounds__(256) gemv_kernel(
 #pragma unroll
           for (int kb = 0; kb < 8; ++kb) {
             const int jw = kb >> 2, p = kb & 3;
-            const int w0 = ((jw * 4 + p) * 2 + 0) * 4 + c, w1 = w0 + 4;
-            const uint32_t a0 = xrow0[w0], a1 = xrow1[w0], a2 = xrow0[w1], a3 = xrow1[w1];
+            const int k1 = ku + 32 * c + 16 * jw + p;  // codes (k1, k1+8) and (k1+4, k1+12)
+            const uint32_t a0 = g0 ? x_pair(row0, k1, k1 + 8) : 0u;
+            const uint32_t a1 = g1 ? x_pair(row1, k1, k1 + 8) : 0u;
+            const uint32_t a2 = g0 ? x_pair(row0, k1 + 4, k1 + 12) : 0u;
+            const uint32_t a3 = g1 ? x_pair(row1, k1 + 4, k1 + 12) : 0u;
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
               const uint32_t wv = wreg[i][j][jw];
@@ -200,12 +215,11 @@ __global__ void __launch_bounds__(256) gemv_kernel(
                              q2_pair_bf16(wv, 2 * p + 8));
             }
           }
-          // block scale d[n][unit] for columns n = n0 + 8j + 2c, +1
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
-            const int n = n0 + 8 * j + 2 * c;
-            const float d0 = n < N ? __half2float(__ushort_as_half(scales[static_cast<int64_t>(n) * nscale + unit])) : 0.f;
-            const float d1 = n + 1 < N ? __half2float(__ushort_as_half(scales[static_cast<int64_t>(n + 1) * nscale + unit])) : 0.f;
+            const int rl = 8 * j + 2 * c, ui = unit - u_base;
+            const float d0 = __half2float(__ushort_as_half(static_cast<uint16_t>(scl[rl][ui])));
+            const float d1 = __half2float(__ushort_as_half(static_cast<uint16_t>(scl[rl + 1][ui])));
             acc[j][0] = fmaf(d0, part[j][0], acc[j][0]);
             acc[j][1] = fmaf(d1, part[j][1], acc[j][1]);
             acc[j][2] = fmaf(d0, part[j][2], acc[j][2]);
@@ -223,10 +237,12 @@ __global__ void __launch_bounds__(256) gemv_kernel(
               for (int e = 0; e < 4; ++e) part[j][e] = 0.f;
 #pragma unroll
             for (int kq = 0; kq < 4; ++kq) {
-              const int kb = 4 * h2 + kq;
               const int jj = kq >> 1, half = kq & 1;
-              const int w0 = (kb * 2 + 0) * 4 + c, w1 = w0 + 4;
-              const uint32_t a0 = xrow0[w0], a1 = xrow1[w0], a2 = xrow0[w1], a3 = xrow1[w1];
+              const int k1 = ku + 64 * h2 + 16 * c + 8 * jj + 2 * half;  // (k1, k1+4), (k1+1, k1+5)
+              const uint32_t a0 = g0 ? x_pair(row0, k1, k1 + 4) : 0u;
+              const uint32_t a1 = g1 ? x_pair(row1, k1, k1 + 4) : 0u;
+              const uint32_t a2 = g0 ? x_pair(row0, k1 + 1, k1 + 5) : 0u;
+              const uint32_t a3 = g1 ? x_pair(row1, k1 + 1, k1 + 5) : 0u;
               mma_bf16_16816(ssum, a0, a1, a2, a3, 0x3F803F80u, 0x3F803F80u);
 #pragma unroll
               for (int j = 0; j < 4; ++j) {
@@ -238,18 +254,12 @@ __global__ void __launch_bounds__(256) gemv_kernel(
             // ssum[0] = S for token g, ssum[2] = S for token g + 8
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-              const int n = n0 + 8 * j + 2 * c;
-              float s0 = 0.f, z0 = 0.f, s1 = 0.f, z1 = 0.f;
-              if (n < N) {
-                const uint32_t v = reinterpret_cast<const uint32_t*>(scales)[static_cast<int64_t>(n) * nscale + grp];
-                s0 = __half2float(__ushort_as_half(static_cast<uint16_t>(v & 0xFFFFu)));
-                z0 = __half2float(__ushort_as_half(static_cast<uint16_t>(v >> 16)));
-              }
-              if (n + 1 < N) {
-                const uint32_t v = reinterpret_cast<const uint32_t*>(scales)[static_cast<int64_t>(n + 1) * nscale + grp];
-                s1 = __half2float(__ushort_as_half(static_cast<uint16_t>(v & 0xFFFFu)));
-                z1 = __half2float(__ushort_as_half(static_cast<uint16_t>(v >> 16)));
-              }
+              const int rl = 8 * j + 2 * c, gi = grp - 2 * u_base;
+              const uint32_t v0 = scl[rl][gi], v1 = scl[rl + 1][gi];
+              const float s0 = __half2float(__ushort_as_half(static_cast<uint16_t>(v0 & 0xFFFFu)));
+              const float z0 = __half2float(__ushort_as_half(static_cast<uint16_t>(v0 >> 16)));
+              const float s1 = __half2float(__ushort_as_half(static_cast<uint16_t>(v1 & 0xFFFFu)));
+              const float z1 = __half2float(__ushort_as_half(static_cast<uint16_t>(v1 >> 16)));
               acc[j][0] = fmaf(s0, fmaf(-z0, ssum[0], part[j][0]), acc[j][0]);
               acc[j][1] = fmaf(s1, fmaf(-z1, ssum[0], part[j][1]), acc[j][1]);
               acc[j][2] = fmaf(s0, fmaf(-z0, ssum[2], part[j][2]), acc[j][2]);
@@ -258,10 +268,10 @@ __global__ void __launch_bounds__(256) gemv_kernel(
           }
         }
       }
+      __syncthreads();  // everyone is done with this pass's activations
     }
 
     // ---- reduce the warps' partial sums and write y ---------------------------------
-    __syncthreads();  // every warp is done reading xs
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       red[warp][g][8 * j + 2 * c] = acc[j][0];

@@ -8,6 +8,7 @@
 #include <cstdint>
 #include <cstdio>
 #include <mutex>
+#include <vector>
 
 #include "../../include/tgemm.h"
 #include "common.cuh"
@@ -60,6 +61,50 @@ inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s
 
 inline int launch_status() {
   return cudaGetLastError() == cudaSuccess ? TGEMM_OK : TGEMM_ECUDA;
+}
+
+// ---- launch accounting and optional per-launch event timing ---------------------------
+
+std::atomic<int64_t> g_launches{0};
+std::atomic<int> g_profile{0};
+struct ProfRecord {
+  int kind;
+  cudaEvent_t begin, end;
+};
+std::vector<ProfRecord> g_records;
+std::vector<cudaEvent_t> g_event_pool;
+std::mutex g_prof_mu;
+
+cudaEvent_t take_event() {
+  std::lock_guard<std::mutex> lock(g_prof_mu);
+  if (!g_event_pool.empty()) {
+    cudaEvent_t e = g_event_pool.back();
+    g_event_pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+  return e;
+}
+
+// Run `launch_fn` (one kernel launch on `st`), count it, and time it when profiling.
+template <typename Fn>
+int launch(int kind, cudaStream_t st, Fn&& launch_fn) {
+  cudaEvent_t b = nullptr, e = nullptr;
+  if (g_profile.load(std::memory_order_relaxed)) {
+    b = take_event();
+    e = take_event();
+    if (b && e) cudaEventRecord(b, st);
+  }
+  launch_fn();
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  const int status = launch_status();
+  if (b && e) {
+    cudaEventRecord(e, st);
+    std::lock_guard<std::mutex> lock(g_prof_mu);
+    g_records.push_back({kind, b, e});
+  }
+  return status;
 }
 
 int grid_for(int64_t work_items, int per_block, int sms) {
@@ -129,45 +174,85 @@ int choose_path(int M) {
 }
 
 struct LoraDims {
-  int R;     // round_up(r, 16)
-  int wcat;  // width of [u_hi | u_lo | 0], a multiple of 64
-  int L;     // pipeline stages for the branch
+  int R;       // round_up(r, 16)
+  int wcat;    // width of [u_hi | u_lo | 0], a multiple of 64
+  int L;       // pipeline stages for the branch
+  int rpad;    // round_up(r, 64): columns of the partial sums
+  int slices;  // K slices of the partial sums
 };
 
-LoraDims lora_dims(int r) {
+LoraDims lora_dims(int r, int K) {
   LoraDims d;
   d.R = (r + 15) / 16 * 16;
   d.wcat = (2 * d.R + 63) / 64 * 64;
   d.L = d.wcat / 64;
+  d.rpad = (r + 63) / 64 * 64;
+  d.slices = (K + kLoraKc - 1) / kLoraKc;
   return d;
 }
 
 struct Workspace {
-  size_t x16 = 0, x16_bytes = 0;  // f16 activations (tensor-core path)
-  size_t ucat = 0, ucat_bytes = 0;
-  size_t u32 = 0, u32_bytes = 0;  // f32 u (small-M path)
+  size_t x16 = 0, x16_bytes = 0;    // f16 activations (tensor-core path)
+  size_t ucat = 0, ucat_bytes = 0;  // [u_hi | u_lo] (tensor-core path)
+  size_t u32 = 0, u32_bytes = 0;    // f32 u (small-M path)
+  size_t part = 0, part_bytes = 0;  // f32 partial sums of u
   size_t total = 0;
 };
 
 Workspace workspace_layout(int op, int M, int K, int r, int path) {
   Workspace w;
   size_t off = 0;
+  const bool lora = op == TGEMM_OP_Q2_LORA;
   if (path == TGEMM_PATH_TENSOR) {
     w.x16 = off;
     w.x16_bytes = static_cast<size_t>(M) * K * 2;
     off = round_up(off + w.x16_bytes, 256);
-    if (op == TGEMM_OP_Q2_LORA) {
+    if (lora) {
       w.ucat = off;
-      w.ucat_bytes = static_cast<size_t>(M) * lora_dims(r).wcat * 2;
+      w.ucat_bytes = static_cast<size_t>(M) * lora_dims(r, K).wcat * 2;
       off = round_up(off + w.ucat_bytes, 256);
     }
-  } else if (op == TGEMM_OP_Q2_LORA) {
+  } else if (lora) {
     w.u32 = off;
     w.u32_bytes = static_cast<size_t>(M) * r * 4;
     off = round_up(off + w.u32_bytes, 256);
   }
+  if (lora) {
+    const LoraDims ld = lora_dims(r, K);
+    w.part = off;
+    w.part_bytes = static_cast<size_t>(ld.slices) * M * ld.rpad * 4;
+    off = round_up(off + w.part_bytes, 256);
+  }
   w.total = off;
   return w;
+}
+
+// u = x A^T into u32 (f32 [M][r]) and/or ucat, through the partial-sum workspace.
+int launch_lora_down(const uint16_t* x, const uint16_t* la, int M, int K, int r,
+                     const LoraDims& ld, float* part, float* u32, uint16_t* ucat,
+                     cudaStream_t st, int sms) {
+  const dim3 grid((M + 15) / 16, ld.slices, ld.rpad / 64);
+  if (int e = launch(TGEMM_KIND_PREP, st, [&] {
+        lora_down_partial_kernel<<<grid, 256, 0, st>>>(x, la, M, K, r, ld.rpad, part);
+      }))
+    return e;
+  const int64_t items = ucat ? static_cast<int64_t>(M) * ld.wcat : static_cast<int64_t>(M) * r;
+  const int fgrid = grid_for(items, 256, sms);
+  return launch(TGEMM_KIND_PREP, st, [&] {
+    lora_finalize_kernel<<<fgrid, 256, 0, st>>>(part, ld.slices, M, r, ld.rpad, ld.R, ld.wcat,
+                                                u32, ucat);
+  });
+}
+
+template <int FMT, bool LORA>
+int gemv_prepare() {
+  static std::once_flag once;
+  static cudaError_t err = cudaSuccess;
+  std::call_once(once, [] {
+    err = cudaFuncSetAttribute(gemv_kernel<FMT, LORA>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               gemv_smem_bytes(16, kGvKP));
+  });
+  return err == cudaSuccess ? TGEMM_OK : TGEMM_ECUDA;
 }
 
 // ---- the matmul driver ---------------------------------------------------------------
@@ -196,52 +281,60 @@ int run_gemm(int fmt, const uint16_t* x, const uint8_t* wq, const uint16_t* scal
   const cudaStream_t st = as_stream(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   const int out_f32 = out_dtype == TGEMM_OUT_F32 ? 1 : 0;
-  const LoraDims ld = lora ? lora_dims(r) : LoraDims{0, 0, 0};
+  const LoraDims ld = lora ? lora_dims(r, K) : LoraDims{0, 0, 0, 0, 0};
+  float* part = lora ? reinterpret_cast<float*>(ws + wl.part) : nullptr;
 
   if (path == TGEMM_PATH_SMALL_M) {
     float* u32 = nullptr;
     if (lora) {
       u32 = reinterpret_cast<float*>(ws + wl.u32);
-      const dim3 grid((M + 15) / 16, (r + 63) / 64);
-      lora_down_kernel<<<grid, 256, 0, st>>>(x, la, M, K, r, ld.R, ld.wcat, u32, nullptr);
+      if (int e = launch_lora_down(x, la, M, K, r, ld, part, u32, nullptr, st, di.sms)) return e;
     }
     const int grid = (N + kGvRows - 1) / kGvRows;
-    if (fmt == 0) {
-      if (lora)
-        gemv_kernel<0, true><<<grid, 256, 0, st>>>(x, wq, scales, y, M, N, K, out_f32, u32, lb, r);
-      else
-        gemv_kernel<0, false><<<grid, 256, 0, st>>>(x, wq, scales, y, M, N, K, out_f32, nullptr, nullptr, 0);
-    } else {
-      gemv_kernel<1, false><<<grid, 256, 0, st>>>(x, wq, scales, y, M, N, K, out_f32, nullptr, nullptr, 0);
+    const int mrows = M < 16 ? M : 16;
+    const int kp = K < kGvKP ? K : kGvKP;
+    const size_t smem = gemv_smem_bytes(mrows, kp);
+    if (fmt == 0 && lora) {
+      if (int e = gemv_prepare<0, true>()) return e;
+      return launch(TGEMM_KIND_GEMV_Q2, st, [&] {
+        gemv_kernel<0, true><<<grid, 256, smem, st>>>(x, wq, scales, y, M, N, K, out_f32, u32, lb, r, mrows, kp);
+      });
     }
-    return launch_status();
+    if (fmt == 0) {
+      if (int e = gemv_prepare<0, false>()) return e;
+      return launch(TGEMM_KIND_GEMV_Q2, st, [&] {
+        gemv_kernel<0, false><<<grid, 256, smem, st>>>(x, wq, scales, y, M, N, K, out_f32, nullptr, nullptr, 0, mrows, kp);
+      });
+    }
+    if (int e = gemv_prepare<1, false>()) return e;
+    return launch(TGEMM_KIND_GEMV_Q4, st, [&] {
+      gemv_kernel<1, false><<<grid, 256, smem, st>>>(x, wq, scales, y, M, N, K, out_f32, nullptr, nullptr, 0, mrows, kp);
+    });
   }
 
   // ---- tensor-core path
   uint16_t* x16 = reinterpret_cast<uint16_t*>(ws + wl.x16);
   const int64_t ngroups = static_cast<int64_t>(M) * K / 16;
-  if (fmt == 0)
-    prep_x16_kernel<0><<<grid_for(ngroups, 256, di.sms), 256, 0, st>>>(x, x16, ngroups);
-  else
-    prep_x16_kernel<1><<<grid_for(ngroups, 256, di.sms), 256, 0, st>>>(x, x16, ngroups);
+  const int pgrid = grid_for(ngroups, 256, di.sms);
+  if (int e = launch(TGEMM_KIND_PREP, st, [&] {
+        if (fmt == 0)
+          prep_x16_kernel<0><<<pgrid, 256, 0, st>>>(x, x16, ngroups);
+        else
+          prep_x16_kernel<1><<<pgrid, 256, 0, st>>>(x, x16, ngroups);
+      }))
+    return e;
   uint16_t* ucat = nullptr;
   if (lora) {
     ucat = reinterpret_cast<uint16_t*>(ws + wl.ucat);
-    const dim3 grid((M + 15) / 16, (ld.R + 63) / 64);
-    lora_down_kernel<<<grid, 256, 0, st>>>(x, la, M, K, r, ld.R, ld.wcat, nullptr, ucat);
+    if (int e = launch_lora_down(x, la, M, K, r, ld, part, nullptr, ucat, st, di.sms)) return e;
   }
-  CUtensorMap tm_x, tm_w, tm_u;
-  if (int e = make_map_2d(&tm_x, x16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, K, M, kTcBK, kTcBM,
+  CUtensorMap tm_x, tm_u;
+  if (int e = make_map_2d(&tm_x, x16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, K, M, kTcBK, kTcTok,
                           CU_TENSOR_MAP_SWIZZLE_128B))
-    return e;
-  const int wq_row_bytes = fmt == 0 ? 16 : 32;
-  const uint64_t wq_cols = fmt == 0 ? K / 4 : K / 2;
-  if (int e = make_map_2d(&tm_w, wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, wq_cols, N, wq_row_bytes,
-                          kTcBN, CU_TENSOR_MAP_SWIZZLE_NONE))
     return e;
   if (lora) {
     if (int e = make_map_2d(&tm_u, ucat, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ld.wcat, M, kTcBK,
-                            kTcBM, CU_TENSOR_MAP_SWIZZLE_128B))
+                            kTcTok, CU_TENSOR_MAP_SWIZZLE_128B))
       return e;
   } else {
     tm_u = tm_x;  // unused
@@ -250,8 +343,8 @@ int run_gemm(int fmt, const uint16_t* x, const uint8_t* wq, const uint16_t* scal
   p.M = M;
   p.N = N;
   p.K = K;
-  p.tiles_m = (M + kTcBM - 1) / kTcBM;
-  const int tiles_n = (N + kTcBN - 1) / kTcBN;
+  p.tiles_m = (M + kTcTok - 1) / kTcTok;
+  const int tiles_n = (N + kTcRows - 1) / kTcRows;
   p.num_tiles = p.tiles_m * tiles_n;
   p.kt_main = K / kTcBK;
   p.kt_lora = lora ? ld.L : 0;
@@ -259,23 +352,27 @@ int run_gemm(int fmt, const uint16_t* x, const uint8_t* wq, const uint16_t* scal
   p.R = ld.R;
   p.r = r;
   p.out_f32 = out_f32;
-  const int esize = out_f32 ? 4 : 2;
-  p.vec_store = (static_cast<int64_t>(N) * esize) % 16 == 0 ? 1 : 0;
+  p.wq = wq;
   p.scales = scales;
   p.lb = lb;
   p.y = y;
   const int grid = p.num_tiles < di.sms ? p.num_tiles : di.sms;
   if (fmt == 0 && !lora) {
     if (int e = tc_prepare<0, false>()) return e;
-    tc_gemm_kernel<0, false><<<grid, kTcThreads, TcFmt<0>::kSmemBytes, st>>>(tm_x, tm_w, tm_u, p);
-  } else if (fmt == 0) {
-    if (int e = tc_prepare<0, true>()) return e;
-    tc_gemm_kernel<0, true><<<grid, kTcThreads, TcFmt<0>::kSmemBytes, st>>>(tm_x, tm_w, tm_u, p);
-  } else {
-    if (int e = tc_prepare<1, false>()) return e;
-    tc_gemm_kernel<1, false><<<grid, kTcThreads, TcFmt<1>::kSmemBytes, st>>>(tm_x, tm_w, tm_u, p);
+    return launch(TGEMM_KIND_TC_Q2, st, [&] {
+      tc_gemm_kernel<0, false><<<grid, kTcThreads, TcFmt<0>::kSmemBytes, st>>>(tm_x, tm_u, p);
+    });
   }
-  return launch_status();
+  if (fmt == 0) {
+    if (int e = tc_prepare<0, true>()) return e;
+    return launch(TGEMM_KIND_TC_Q2_LORA, st, [&] {
+      tc_gemm_kernel<0, true><<<grid, kTcThreads, TcFmt<0>::kSmemBytes, st>>>(tm_x, tm_u, p);
+    });
+  }
+  if (int e = tc_prepare<1, false>()) return e;
+  return launch(TGEMM_KIND_TC_Q4, st, [&] {
+    tc_gemm_kernel<1, false><<<grid, kTcThreads, TcFmt<1>::kSmemBytes, st>>>(tm_x, tm_u, p);
+  });
 }
 
 }  // namespace
@@ -296,8 +393,10 @@ int q2_pack(const uint8_t* codes, const float* scale, uint8_t* wq, uint16_t* d, 
   if (int st = current_device_info(&di)) return st;
   const int64_t units = static_cast<int64_t>(N) * K / 64;
   const int64_t scales = static_cast<int64_t>(N) * K / 128;
-  q2_pack_kernel<<<grid_for(units, 256, di.sms), 256, 0, as_stream(stream)>>>(codes, scale, wq, d, units, scales, status);
-  return launch_status();
+  const cudaStream_t st = as_stream(stream);
+  return launch(TGEMM_KIND_PREP, st, [&] {
+    q2_pack_kernel<<<grid_for(units, 256, di.sms), 256, 0, st>>>(codes, scale, wq, d, units, scales, status);
+  });
 }
 
 int q4_pack(const uint8_t* codes, const float* s, const float* z, uint8_t* wq, uint16_t* sz,
@@ -311,8 +410,10 @@ int q4_pack(const uint8_t* codes, const float* s, const float* z, uint8_t* wq, u
   if (int st = current_device_info(&di)) return st;
   const int64_t units = static_cast<int64_t>(N) * K / 32;
   const int64_t groups = static_cast<int64_t>(N) * K / 64;
-  q4_pack_kernel<<<grid_for(units, 256, di.sms), 256, 0, as_stream(stream)>>>(codes, s, z, wq, sz, units, groups, status);
-  return launch_status();
+  const cudaStream_t st = as_stream(stream);
+  return launch(TGEMM_KIND_PREP, st, [&] {
+    q4_pack_kernel<<<grid_for(units, 256, di.sms), 256, 0, st>>>(codes, s, z, wq, sz, units, groups, status);
+  });
 }
 
 int q2_dequant(const uint8_t* wq, const uint16_t* d, float* w, int N, int K, void* stream) {
@@ -322,8 +423,10 @@ int q2_dequant(const uint8_t* wq, const uint16_t* d, float* w, int N, int K, voi
   DeviceInfo di;
   if (int st = current_device_info(&di)) return st;
   const int64_t words = static_cast<int64_t>(N) * K / 16;
-  q2_dequant_kernel<<<grid_for(words, 256, di.sms), 256, 0, as_stream(stream)>>>(wq, d, w, words, K);
-  return launch_status();
+  const cudaStream_t st = as_stream(stream);
+  return launch(TGEMM_KIND_PREP, st, [&] {
+    q2_dequant_kernel<<<grid_for(words, 256, di.sms), 256, 0, st>>>(wq, d, w, words, K);
+  });
 }
 
 int q4_dequant(const uint8_t* wq, const uint16_t* sz, float* w, int N, int K, void* stream) {
@@ -333,8 +436,10 @@ int q4_dequant(const uint8_t* wq, const uint16_t* sz, float* w, int N, int K, vo
   DeviceInfo di;
   if (int st = current_device_info(&di)) return st;
   const int64_t words = static_cast<int64_t>(N) * K / 8;
-  q4_dequant_kernel<<<grid_for(words, 256, di.sms), 256, 0, as_stream(stream)>>>(wq, sz, w, words, K);
-  return launch_status();
+  const cudaStream_t st = as_stream(stream);
+  return launch(TGEMM_KIND_PREP, st, [&] {
+    q4_dequant_kernel<<<grid_for(words, 256, di.sms), 256, 0, st>>>(wq, sz, w, words, K);
+  });
 }
 
 size_t tgemm_workspace_size(int op, int M, int N, int K, int r) {
@@ -396,5 +501,40 @@ int tgemm_device_error(uint32_t* bits, int clear) {
 }
 
 int tgemm_version(void) { return 100; }
+
+int tgemm_profile_enable(int on) { return g_profile.exchange(on ? 1 : 0); }
+
+int tgemm_profile_read(int kind, double* total_ms, int64_t* launches, int reset) {
+  if (kind < 0 || kind >= TGEMM_NUM_KINDS || !total_ms || !launches) return TGEMM_EINVAL;
+  std::lock_guard<std::mutex> lock(g_prof_mu);
+  double sum = 0.0;
+  int64_t n = 0;
+  int status = TGEMM_OK;
+  std::vector<ProfRecord> keep;
+  for (const ProfRecord& rec : g_records) {
+    if (rec.kind != kind) {
+      keep.push_back(rec);
+      continue;
+    }
+    float ms = 0.f;
+    if (cudaEventSynchronize(rec.end) != cudaSuccess ||
+        cudaEventElapsedTime(&ms, rec.begin, rec.end) != cudaSuccess)
+      status = TGEMM_ECUDA;
+    sum += ms;
+    ++n;
+    if (reset) {
+      g_event_pool.push_back(rec.begin);
+      g_event_pool.push_back(rec.end);
+    } else {
+      keep.push_back(rec);
+    }
+  }
+  g_records.swap(keep);
+  *total_ms = sum;
+  *launches = n;
+  return status;
+}
+
+int64_t tgemm_launch_count(void) { return g_launches.load(); }
 
 }  // extern "C"

@@ -181,6 +181,33 @@ int tgemm_device_error(uint32_t* bits, int clear);
 /* tgemm_version -- library version, major * 10000 + minor * 100 + patch. */
 int tgemm_version(void);
 
+/* ---- measurement hooks ------------------------------------------------------------ */
+/* Kernel kinds for tgemm_profile_read. */
+#define TGEMM_KIND_TC_Q2       0 /* tensor-core Q2_0 matmul kernel */
+#define TGEMM_KIND_TC_Q2_LORA  1 /* tensor-core Q2_0 matmul + low-rank branch kernel */
+#define TGEMM_KIND_TC_Q4       2 /* tensor-core 4-bit matmul kernel */
+#define TGEMM_KIND_GEMV_Q2     3 /* small-M Q2_0 kernel (with or without the branch) */
+#define TGEMM_KIND_GEMV_Q4     4 /* small-M 4-bit kernel */
+#define TGEMM_KIND_PREP        5 /* activation conversion and u = x A^T kernels */
+#define TGEMM_NUM_KINDS        6
+
+/*
+ * tgemm_profile_enable -- when `on` is nonzero, every subsequent launch records a pair of
+ * CUDA events around itself on the call's stream (host cost: two event records per
+ * launch; do not enable while capturing a CUDA graph).  Returns the previous setting.
+ */
+int tgemm_profile_enable(int on);
+
+/*
+ * tgemm_profile_read -- wait for the recorded events of `kind` (TGEMM_KIND_*), store the
+ * summed device time in *total_ms and the number of launches in *launches; forget them
+ * if `reset` is nonzero.
+ */
+int tgemm_profile_read(int kind, double* total_ms, int64_t* launches, int reset);
+
+/* tgemm_launch_count -- kernels launched by this library since it was loaded. */
+int64_t tgemm_launch_count(void);
+
 #ifdef __cplusplus
 }
 #endif
