@@ -89,14 +89,22 @@ def barrier(world):
 
 
 def max_over_ranks(v: float, world: int) -> float:
+    """The slowest rank's value (device times are compared as the max over ranks)."""
     if world == 1:
         return v
     import torch
     import torch.distributed as dist
 
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def aggregate_value(world: int, step_flops: float, step_ms: float) -> float:
+    """Whole-job TFLOP/s: every rank runs one step of `step_flops`; the job takes the
+    slowest rank's `step_ms`."""
+    return world * step_flops / (step_ms * 1e-3) / 1e12
 
 
 def dist_done(world):
@@ -266,9 +274,11 @@ class Op:
 
 
 def _reseed(w, rank):
+    """The same workload with rank-specific data (weak scaling: every rank its own batch)."""
     import dataclasses
 
-    return dataclasses.replace(w, seed=(w.seed, "rank", rank))
+    base = tuple(w.seed) if isinstance(w.seed, tuple) else (w.seed,)
+    return dataclasses.replace(w, seed=base + (7919, rank))
 
 
 def _to_dev(bits, dtype, torch):
@@ -495,7 +505,7 @@ def ours(args, world, rank, local):
                          f"proportion to their FLOPs, each computed on its own "
                          f"({r['seconds']:.1f} s of CPU time)"}
 
-    value = world * step_flops / (step_ms * 1e-3) / 1e12
+    value = aggregate_value(world, step_flops, step_ms)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True,
