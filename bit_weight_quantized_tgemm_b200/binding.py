@@ -17,7 +17,8 @@ import torch
 
 from . import build as _build
 
-OK, EINVAL, EALIGN, ECUDA, EARCH, EWORKSPACE = 0, -1, -2, -3, -4, -5
+OK, EINVAL, EALIGN, ECUDA, EARCH, EWORKSPACE, ETOOLARGE = 0, -1, -2, -3, -4, -5, -6
+NOALLOC_SCRATCH_BYTES = 40 * 1024 * 1024
 OUT_F32, OUT_BF16 = 0, 1
 OP_Q2, OP_Q2_LORA, OP_Q4 = 0, 1, 2
 PATH_AUTO, PATH_SMALL_M, PATH_TENSOR = 0, 1, 2
@@ -38,6 +39,7 @@ _SIGS = {
     "tgemm_q2": (_i, [_P, _P, _P, _P, _i, _i, _i, _i, _P, _sz, _P]),
     "tgemm_q2_lora": (_i, [_P, _P, _P, _P, _P, _i, _P, _i, _i, _i, _i, _P, _sz, _P]),
     "tgemm_q4": (_i, [_P, _P, _P, _P, _i, _i, _i, _i, _P, _sz, _P]),
+    "tgemm_q2_noalloc": (_i, [_P, _P, _P, _P, _i, _i, _i, _i, _P]),
     "tgemm_strerror": (ctypes.c_char_p, [_i]),
     "tgemm_set_path": (_i, [_i]),
     "tgemm_device_error": (_i, [_P, _i]),
@@ -204,6 +206,23 @@ def gemm_q2(x: torch.Tensor, wq: torch.Tensor, d: torch.Tensor, *, out_dtype: in
     ws, nbytes = _workspace(OP_Q2, M, N, K, 0, x.device, workspace)
     _check(lib().tgemm_q2(_ptr(x), _ptr(wq), _ptr(d), _ptr(y), M, N, K, out_dtype, _ptr(ws),
                           nbytes, _stream()), "tgemm_q2")
+    return y
+
+
+def gemm_q2_noalloc(x: torch.Tensor, wq: torch.Tensor, d: torch.Tensor, *,
+                    out_dtype: int = OUT_BF16, y: Optional[torch.Tensor] = None):
+    """gemm_q2 through tgemm_q2_noalloc: scratch comes from the library's built-in buffer.
+
+    For callers that cannot allocate device memory (pass a preallocated ``y``).  Calls
+    that overlap on the GPU share that buffer and race; see include/tgemm.h."""
+    _need(x, torch.bfloat16, "x")
+    _need(wq, torch.uint8, "wq")
+    _need(d, torch.float16, "d")
+    M, K = x.shape
+    N = wq.shape[0]
+    y = _out(y, M, N, out_dtype, x.device)
+    _check(lib().tgemm_q2_noalloc(_ptr(x), _ptr(wq), _ptr(d), _ptr(y), M, N, K, out_dtype,
+                                  _stream()), "tgemm_q2_noalloc")
     return y
 
 

@@ -378,6 +378,32 @@ int run_gemm(int fmt, const uint16_t* x, const uint8_t* wq, const uint16_t* scal
 }  // namespace
 }  // namespace tgemm
 
+// ---- scratch for tgemm_q2_noalloc ------------------------------------------------------
+// Compiled into the library so that tgemm_q2_noalloc never allocates.  In host code the
+// name is only a stand-in for the symbol; the device address comes from
+// cudaGetSymbolAddress, once per device.
+static __device__ __align__(256) uint8_t g_noalloc_scratch[TGEMM_NOALLOC_SCRATCH_BYTES];
+
+namespace tgemm {
+namespace {
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+int noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return TGEMM_ECUDA;
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
+      return TGEMM_ECUDA;
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return TGEMM_OK;
+}
+}  // namespace
+}  // namespace tgemm
+
 using namespace tgemm;
 
 extern "C" {
@@ -463,6 +489,20 @@ int tgemm_q2_lora(const uint16_t* x, const uint8_t* wq, const uint16_t* d, const
   return run_gemm(0, x, wq, d, a, b, r, y, M, N, K, out_dtype, workspace, ws_bytes, stream);
 }
 
+int tgemm_q2_noalloc(const uint16_t* x, const uint8_t* wq, const uint16_t* d, void* y, int M,
+                     int N, int K, int out_dtype, void* stream) {
+  if (!x || !wq || !d || !y) return TGEMM_EINVAL;
+  if (M < 1 || N < 1 || K < 128 || K % 128) return TGEMM_EINVAL;
+  const size_t need = workspace_layout(TGEMM_OP_Q2, M, K, 0, choose_path(M)).total;
+  if (need > TGEMM_NOALLOC_SCRATCH_BYTES) return TGEMM_ETOOLARGE;
+  void* scratch = nullptr;
+  if (need > 0) {
+    if (int e = noalloc_scratch(&scratch)) return e;
+  }
+  return run_gemm(0, x, wq, d, nullptr, nullptr, 0, y, M, N, K, out_dtype, scratch,
+                  need > 0 ? static_cast<size_t>(TGEMM_NOALLOC_SCRATCH_BYTES) : 0, stream);
+}
+
 int tgemm_q4(const uint16_t* x, const uint8_t* wq, const uint16_t* sz, void* y, int M, int N,
              int K, int out_dtype, void* workspace, size_t ws_bytes, void* stream) {
   return run_gemm(1, x, wq, sz, nullptr, nullptr, 0, y, M, N, K, out_dtype, workspace, ws_bytes,
@@ -477,6 +517,7 @@ const char* tgemm_strerror(int status) {
     case TGEMM_ECUDA: return "CUDA runtime or launch failure";
     case TGEMM_EARCH: return "device is not compute capability 10.0 (sm_100)";
     case TGEMM_EWORKSPACE: return "workspace missing or too small";
+    case TGEMM_ETOOLARGE: return "problem needs more scratch than the built-in buffer holds";
     default: return "unknown status";
   }
 }

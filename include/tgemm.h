@@ -62,6 +62,8 @@ extern "C" {
 #define TGEMM_ECUDA      -3 /* a CUDA runtime call or kernel launch failed */
 #define TGEMM_EARCH      -4 /* the current device is not compute capability 10.0 */
 #define TGEMM_EWORKSPACE -5 /* workspace missing or smaller than tgemm_workspace_size() */
+#define TGEMM_ETOOLARGE  -6 /* tgemm_q2_noalloc: the problem needs more scratch than its
+                               built-in buffer (TGEMM_NOALLOC_SCRATCH_BYTES) holds */
 
 /* ---- output element types ---------------------------------------------------------- */
 #define TGEMM_OUT_F32  0
@@ -152,6 +154,29 @@ int tgemm_q2(const uint16_t* x, const uint8_t* wq, const uint16_t* d, void* y, i
 int tgemm_q2_lora(const uint16_t* x, const uint8_t* wq, const uint16_t* d, const uint16_t* a,
                   const uint16_t* b, int r, void* y, int M, int N, int K, int out_dtype,
                   void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * tgemm_q2_noalloc -- tgemm_q2 for callers that cannot allocate device memory.
+ *   The pages have no counterpart to this call; it exists for code that may not call
+ *   cudaMalloc or any allocator: plugins inside hosts that own all device memory, code
+ *   paths that run while a stream is being captured, real-time loops that must not
+ *   allocate.  It computes exactly what tgemm_q2 computes (same kernels), but instead of
+ *   a caller workspace it uses one scratch buffer compiled into the library: a
+ *   file-scope device array of TGEMM_NOALLOC_SCRATCH_BYTES (40 MiB), which every GPU
+ *   that loads the library holds until the process exits.
+ *   Limit: the tensor-core path needs M*K*2 bytes of scratch (an f16 copy of x), so
+ *   M*K may be at most 20 Mi elements (e.g. 1536 x 12288); larger problems return
+ *   TGEMM_ETOOLARGE before launching anything.  The small-M path (M <= 16) needs none.
+ *   The first call on a device looks up that device's address of the buffer
+ *   (cudaGetSymbolAddress, with that device current); make that first call before any
+ *   stream capture.  All calls share the one buffer and it keeps the last call's
+ *   contents (nothing in it has to start at zero: every call rewrites what it reads).
+ *   Calls that overlap on the GPU -- on different streams, or from different threads --
+ *   race on the buffer: serialize them.  Arguments, layouts and errors as tgemm_q2.
+ */
+#define TGEMM_NOALLOC_SCRATCH_BYTES (40u * 1024u * 1024u)
+int tgemm_q2_noalloc(const uint16_t* x, const uint8_t* wq, const uint16_t* d, void* y, int M,
+                     int N, int K, int out_dtype, void* stream);
 
 /*
  * tgemm_q4 -- y = x . W^T for 4-bit group weights.
