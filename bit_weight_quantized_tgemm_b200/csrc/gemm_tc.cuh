@@ -1,21 +1,30 @@
 // gemm_tc.cuh -- large-M path: persistent tcgen05 (5th-generation tensor core) kernel.
 //
 // Tile: 128 weight rows (MMA M, TMEM lanes) x 256 tokens (MMA N, accumulator columns),
-// 64 k per stage.  Putting the weights on the 128-row side halves the dequantization
-// work per MMA flop compared with a 128-token tile: each stage dequantizes 128 x 64
-// codes for a 128x256x64 product.
-// Warp roles (14 warps, one CTA per SM):
+// 64 k per stage (an M=128 MMA costs the same time for any N up to 256, so N is 256).  The dequantized weights never touch shared memory: dequant warps write
+// them straight into tensor memory (tcgen05.st) and the MMA reads its A operand from
+// there (tcgen05.mma ... [a_tmem]).  Shared memory then carries only the activation
+// tiles (TMA in, MMA out), which keeps its traffic at 128 bytes per MMA cycle.
+//
+// Tensor memory (512 columns x 128 lanes of 32 bits):
+//   columns [0, 256)             the f32 accumulator
+//   columns [256 + 32 s, +32)    A stage s (s < 8): 128 rows x 64 k of f16, element k of a
+//                                row in column k/2 (low half for even k)
+// With one accumulator the MMA waits while a finished tile is read out; eight epilogue
+// warps keep that short, and the eight A stages and the TMA stages keep filling
+// meanwhile, so the next tile starts with full queues.
+//
+// Warp roles (18 warps, one CTA per SM):
 //   warp 0      TMA producer: activation tile, 256 tokens x 64 k (f16, 128-byte swizzle)
 //   warp 1      TMEM allocator and MMA issuer (one thread): 4 x tcgen05.mma 128x256x16
-//   warps 2-9   dequantizers: warp pair (w, w+4) owns rows 32*(w%4).. of the tile, each
-//               thread half a row (32 codes) per stage; codes come straight from global
-//               memory (16 or 8 bytes per thread per stage, four stages ahead), are
-//               unpacked and scaled in f16 and stored in the 128-byte-swizzled K-major
-//               operand layout the MMA reads
-//   warps 10-13 epilogue: tcgen05.ld of the f32 accumulator (lane = weight row), convert,
-//               store y (lanes write consecutive n of one token row: coalesced)
-// The accumulator is double-buffered in TMEM (2 x 256 columns), so a tile's epilogue
-// overlaps the next tile's main loop.
+//   warps 2-9   dequantizers: warp w handles TMEM lanes 32*(w%4).. (weight rows), warps
+//               2-5 the first 32 k of a stage and warps 6-9 the second; codes come
+//               straight from global memory (8 or 16 bytes per thread per stage, four
+//               stages ahead), are unpacked and scaled in f16 and stored with one
+//               tcgen05.st of 16 columns
+//   warps 10-17 epilogue: warp w reads TMEM lanes 32*(w%4).. and half of the columns
+//               (tcgen05.ld), converts and stores y (lanes write consecutive n of one
+//               token row: coalesced)
 //
 // Operand precision: kind::f16 with both operands f16.  Q2_0 weights (q - 1) * d are
 // exact in f16; 4-bit weights are computed as ((q - z) * s) in f16, exact up to the
@@ -36,23 +45,29 @@
 
 namespace tgemm {
 
+#ifndef TGEMM_TC_STAGES
+#define TGEMM_TC_STAGES 4
+#endif
 constexpr int kTcRows = 128;   // weight rows per tile (MMA M)
 constexpr int kTcTok = 256;    // tokens per tile (MMA N)
 constexpr int kTcBK = 64;
-constexpr int kTcStages = 4;   // activation stages (TMA)
-constexpr int kTcWStages = 3;  // dequantized-weight stages
-constexpr int kTcThreads = 448;
+constexpr int kTcStages = TGEMM_TC_STAGES;  // activation stages (TMA)
+constexpr int kTcAStages = 8;               // dequantized-weight stages in TMEM
+constexpr int kTcEpiWarps = 8;
+constexpr int kTcThreads = (2 + 8 + kTcEpiWarps) * 32;
 constexpr int kTcXBytes = kTcTok * kTcBK * 2;   // 32 KB
-constexpr int kTcWBytes = kTcRows * kTcBK * 2;  // 16 KB
 constexpr int kTcTmemCols = 512;
+constexpr int kTcAccCols = kTcTok;              // f32 accumulator columns
+constexpr int kTcACol0 = kTcAccCols;            // first A-stage column
+constexpr int kTcACols = kTcBK / 2;             // columns per A stage (2 f16 per column)
+static_assert(kTcACol0 + kTcAStages * kTcACols <= kTcTmemCols, "TMEM budget");
 
 template <int FMT>
 struct TcFmt {
   static constexpr int kWqRowBytes = FMT == 0 ? 16 : 32;  // packed bytes per row per stage
   static constexpr int kXOff = 0;
-  static constexpr int kWOff = kXOff + kTcStages * kTcXBytes;
-  static constexpr int kBarOff = kWOff + kTcWStages * kTcWBytes;
-  static constexpr int kNumBars = 2 * kTcStages + 2 * kTcWStages + 4 + 1;
+  static constexpr int kBarOff = kXOff + kTcStages * kTcXBytes;
+  static constexpr int kNumBars = 2 * kTcStages + 2 * kTcAStages + 4 + 1;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kSmemBytes = kMiscOff + 16 + 1024;  // + alignment slack
 };
@@ -83,15 +98,15 @@ __device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity) {
   return true;
 }
 
-__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
-                                             uint32_t d) {
-  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
-               "r"(d)
-               : "memory");
+// A warp-uniform bounded wait: every lane gets the same answer, so the .sync.aligned
+// tcgen05 instructions that follow never run with part of a warp.
+__device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity,
+                                               volatile uint32_t* abort_flag) {
+  return __all_sync(0xFFFFFFFFu, mbar_wait(bar, parity, abort_flag));
 }
 
 // Q2: 16 codes -> 8 f16x2 pairs (codes i, i+8) of (q - 1) * d.
-__device__ __forceinline__ void q2_word_to_f16(uint32_t w, uint32_t d2, uint32_t (&o)[8]) {
+__device__ __forceinline__ void q2_word_to_f16(uint32_t w, uint32_t d2, uint32_t* o) {
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     const uint32_t t = lop3_and_or(w >> (2 * i), 0x00030003u, 0x64006400u);  // 1024 + q
@@ -101,7 +116,7 @@ __device__ __forceinline__ void q2_word_to_f16(uint32_t w, uint32_t d2, uint32_t
 
 // 4-bit: 8 codes -> 4 f16x2 pairs (codes i, i+4) of (q - z) * s.
 __device__ __forceinline__ void q4_word_to_f16(uint32_t w, uint32_t s2, uint32_t z2,
-                                               uint32_t (&o)[4]) {
+                                               uint32_t* o) {
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const uint32_t t = lop3_and_or(w >> (4 * i), 0x000F000Fu, 0x64006400u);  // 1024 + q
@@ -123,10 +138,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   auto full_bar = [&](int s) { return bar0 + 8u * s; };
   auto empty_bar = [&](int s) { return bar0 + 8u * (kTcStages + s); };
   auto wfull_bar = [&](int s) { return bar0 + 8u * (2 * kTcStages + s); };
-  auto wfree_bar = [&](int s) { return bar0 + 8u * (2 * kTcStages + kTcWStages + s); };
-  auto accfull_bar = [&](int a) { return bar0 + 8u * (2 * kTcStages + 2 * kTcWStages + a); };
-  auto accempty_bar = [&](int a) { return bar0 + 8u * (2 * kTcStages + 2 * kTcWStages + 2 + a); };
-  const uint32_t drain_bar = bar0 + 8u * (2 * kTcStages + 2 * kTcWStages + 4);
+  auto wfree_bar = [&](int s) { return bar0 + 8u * (2 * kTcStages + kTcAStages + s); };
+  const uint32_t accfull_bar = bar0 + 8u * (2 * kTcStages + 2 * kTcAStages);
+  const uint32_t accempty_bar = bar0 + 8u * (2 * kTcStages + 2 * kTcAStages + 1);
+  const uint32_t drain_bar = bar0 + 8u * (2 * kTcStages + 2 * kTcAStages + 4);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + F::kMiscOff);
   volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + F::kMiscOff + 4);
 
@@ -137,14 +152,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       mbar_init(full_bar(s), 1);       // producer's expect_tx
       mbar_init(empty_bar(s), 1);      // MMA commit
     }
-    for (int s = 0; s < kTcWStages; ++s) {
+    for (int s = 0; s < kTcAStages; ++s) {
       mbar_init(wfull_bar(s), 8);      // 8 dequant warps
       mbar_init(wfree_bar(s), 1);      // MMA commit
     }
-    for (int a = 0; a < 2; ++a) {
-      mbar_init(accfull_bar(a), 1);    // MMA commit
-      mbar_init(accempty_bar(a), 4);   // 4 epilogue warps
-    }
+    mbar_init(accfull_bar, 1);             // MMA commit
+    mbar_init(accempty_bar, kTcEpiWarps);  // epilogue warps
     mbar_init(drain_bar, 1);
     *abort_flag = 0u;
     fence_mbar_init();
@@ -194,33 +207,32 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       uint32_t it = 0, wit = 0, tcount = 0;
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x, ++tcount) {
-        const uint32_t a = tcount & 1u, aph = (tcount >> 1) & 1u;
-        if (!mbar_wait(accempty_bar(a), aph ^ 1u, abort_flag)) { ok = false; break; }
+        if (!mbar_wait(accempty_bar, (tcount & 1u) ^ 1u, abort_flag)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + a * kTcTok;
+        const uint32_t d_tmem = tmem_base;
         for (int ks = 0; ks < ksteps; ++ks, ++it, ++wit) {
           const uint32_t s = it % kTcStages, ph = (it / kTcStages) & 1u;
-          const uint32_t ws = wit % kTcWStages, wph = (wit / kTcWStages) & 1u;
+          const uint32_t ws = wit % kTcAStages, wph = (wit / kTcAStages) & 1u;
           if (!mbar_wait(wfull_bar(ws), wph, abort_flag)) { ok = false; break; }
           if (!mbar_wait(full_bar(s), ph, abort_flag)) { ok = false; break; }
           tc_fence_after();
-          const uint64_t adesc = smem_desc_sw128(sbase + F::kWOff + ws * kTcWBytes);  // weights
-          const uint64_t bdesc = smem_desc_sw128(sbase + F::kXOff + s * kTcXBytes);   // tokens
+          const uint32_t a_tmem = tmem_base + kTcACol0 + ws * kTcACols;             // weights
+          const uint64_t bdesc = smem_desc_sw128(sbase + F::kXOff + s * kTcXBytes);  // tokens
           if (!LORA || ks < p.kt_main) {
 #pragma unroll
             for (int kk = 0; kk < kTcBK / 16; ++kk)
-              mma_f16_ss(d_tmem, adesc + 2u * kk, bdesc + 2u * kk, kIdescMain,
+              mma_f16_ts(d_tmem, a_tmem + 8u * kk, bdesc + 2u * kk, kIdescMain,
                          (ks > 0 || kk > 0) ? 1u : 0u);
           } else {
             const int done = (ks - p.kt_main) * (kTcBK / 16);
             for (int kk = 0; kk < kTcBK / 16 && done + kk < p.lora_mmas; ++kk)
-              mma_f16_ss(d_tmem, adesc + 2u * kk, bdesc + 2u * kk, kIdescLora, 1u);
+              mma_f16_ts(d_tmem, a_tmem + 8u * kk, bdesc + 2u * kk, kIdescLora, 1u);
           }
           mma_commit(empty_bar(s));
           mma_commit(wfree_bar(ws));
         }
         if (!ok) break;
-        mma_commit(accfull_bar(a));
+        mma_commit(accfull_bar);
       }
       // all MMAs this thread issued must finish before TMEM is released
       mma_commit(drain_bar);
@@ -228,14 +240,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
   } else if (warp < 10) {
     // ------------------------------------------------------------ dequantizers
-    const int dw = warp - 2;
-    const int rt = 32 * (dw & 3) + lane;  // weight row within the tile
-    const int half = dw >> 2;             // which 32 codes of the stage's 64
-    const int swz = rt & 7;
-    const uint32_t row_off = static_cast<uint32_t>((rt >> 3) * 1024 + (rt & 7) * 128);
+    const int q = warp & 3;               // TMEM lane quarter this warp may access
+    const int rt = 32 * q + lane;         // weight row within the tile
+    const int half = (warp - 2) >> 2;     // which 32 codes of the stage's 64
     const int nscale = FMT == 0 ? p.K / 128 : p.K / 64;
     const int64_t wq_row = FMT == 0 ? p.K / 4 : p.K / 2;
     constexpr int kHalfBytes = F::kWqRowBytes / 2;  // 8 (Q2) or 16 (4-bit) bytes per stage
+    const uint32_t a_lane = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + kTcACol0 +
+                            16u * half;
     uint32_t wit = 0;
     bool ok = true;
     for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
@@ -270,98 +282,94 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         c2 = c3;
         c3 = load_codes(ks + 4);
         const bool main_stage = !LORA || ks < p.kt_main;
-        if (main_stage) {
-          const bool new_scale = FMT == 1 || (ks & 1) == 0;
-          if (new_scale) {
-            cur = q0;
-            q0 = q1;
-            q1 = q2;
-            q2 = q3;
-            q3 = load_scale((FMT == 0 ? (ks >> 1) : ks) + 4);
-          }
+        if (main_stage && (FMT == 1 || (ks & 1) == 0)) {
+          cur = q0;
+          q0 = q1;
+          q1 = q2;
+          q2 = q3;
+          q3 = load_scale((FMT == 0 ? (ks >> 1) : ks) + 4);
         }
-        const uint32_t ws = wit % kTcWStages, wph = (wit / kTcWStages) & 1u;
-        if (!mbar_wait(wfree_bar(ws), wph ^ 1u, abort_flag)) { ok = false; break; }
-        const uint32_t wrow = sbase + F::kWOff + ws * kTcWBytes + row_off;
+        uint32_t o[16];
         if (main_stage) {
           if (FMT == 0) {
             const uint32_t d2 = cur | (cur << 16);
-            const uint32_t words[2] = {pk.x, pk.y};
-#pragma unroll
-            for (int j = 0; j < 2; ++j) {
-              uint32_t o[8];
-              q2_word_to_f16(words[j], d2, o);
-              const int ch = 4 * half + 2 * j;  // 16-byte chunk of the 128-byte row
-              st_shared_v4(wrow + ((ch ^ swz) << 4), o[0], o[1], o[2], o[3]);
-              st_shared_v4(wrow + (((ch + 1) ^ swz) << 4), o[4], o[5], o[6], o[7]);
-            }
+            q2_word_to_f16(pk.x, d2, o);
+            q2_word_to_f16(pk.y, d2, o + 8);
           } else {
             const uint32_t s2 = (cur & 0xFFFFu) | (cur << 16);
             const uint32_t z2 = (cur >> 16) | (cur & 0xFFFF0000u);
-            const uint32_t words[4] = {pk.x, pk.y, pk.z, pk.w};
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              uint32_t o[4];
-              q4_word_to_f16(words[j], s2, z2, o);
-              st_shared_v4(wrow + (((4 * half + j) ^ swz) << 4), o[0], o[1], o[2], o[3]);
-            }
+            q4_word_to_f16(pk.x, s2, z2, o);
+            q4_word_to_f16(pk.y, s2, z2, o + 4);
+            q4_word_to_f16(pk.z, s2, z2, o + 8);
+            q4_word_to_f16(pk.w, s2, z2, o + 12);
           }
         } else {
-          // low-rank stage: weight-side columns [jb, jb + 64) of [B | B], zero beyond 2R;
-          // this thread fills 16-byte chunks 4*half .. 4*half+3 of its row
-          const int jb = (ks - p.kt_main) * kTcBK;
+          // low-rank stage: weight-side columns [j0, j0 + 32) of [B | B], zero beyond 2R
+          const int j0 = (ks - p.kt_main) * kTcBK + 32 * half;
           const bool vec = (p.r & 7) == 0 && (reinterpret_cast<uintptr_t>(p.lb) & 15) == 0;
-#pragma unroll 1
+#pragma unroll
           for (int cq = 0; cq < 4; ++cq) {
-            const int cc = 4 * half + cq;
-            const int j0 = jb + 8 * cc;
-            const int i0 = j0 < p.R ? j0 : j0 - p.R;
-            if (vec && j0 < 2 * p.R && i0 + 8 <= p.r) {
+            const int jc = j0 + 8 * cq;
+            const int ic = jc < p.R ? jc : jc - p.R;
+            if (vec && jc < 2 * p.R && ic + 8 <= p.r) {
               uint4 v = make_uint4(0, 0, 0, 0);
-              if (valid) v = *reinterpret_cast<const uint4*>(p.lb + static_cast<int64_t>(row) * p.r + i0);
-              st_shared_v4(wrow + ((cc ^ swz) << 4), v.x, v.y, v.z, v.w);
+              if (valid) v = *reinterpret_cast<const uint4*>(p.lb + static_cast<int64_t>(row) * p.r + ic);
+              o[4 * cq] = v.x;
+              o[4 * cq + 1] = v.y;
+              o[4 * cq + 2] = v.z;
+              o[4 * cq + 3] = v.w;
               continue;
             }
-            uint32_t o[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
               uint32_t v2 = 0;
 #pragma unroll
               for (int h = 0; h < 2; ++h) {
-                const int j = j0 + 2 * e + h;
+                const int j = jc + 2 * e + h;
                 const int i = j < p.R ? j : j - p.R;
                 uint32_t v = 0;
                 if (valid && j < 2 * p.R && i < p.r) v = p.lb[static_cast<int64_t>(row) * p.r + i];
                 v2 |= v << (16 * h);
               }
-              o[e] = v2;
+              o[4 * cq + e] = v2;
             }
-            st_shared_v4(wrow + ((cc ^ swz) << 4), o[0], o[1], o[2], o[3]);
           }
         }
-        fence_proxy_async_smem();
+        const uint32_t ws = wit % kTcAStages, wph = (wit / kTcAStages) & 1u;
+        if (!mbar_wait_warp(wfree_bar(ws), wph ^ 1u, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        tmem_st_32x32b_x16(a_lane + ws * kTcACols, o);
+        tmem_wait_st();
+        tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(wfull_bar(ws));
       }
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    const int q = warp & 3;                // TMEM lane quarter this warp may access
+    const int eh = (warp - 10) >> 2;       // which half of the accumulator's columns
+    constexpr int kChunks = kTcTok / 32 / 2;
     uint32_t tcount = 0;
     for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++tcount) {
       const int tm = tile % p.tiles_m, tn = tile / p.tiles_m;
-      const uint32_t a = tcount & 1u, aph = (tcount >> 1) & 1u;
-      if (!mbar_wait(accfull_bar(a), aph, abort_flag)) break;
+      if (!mbar_wait_warp(accfull_bar, tcount & 1u, abort_flag)) break;
       tc_fence_after();
       const int n = tn * kTcRows + q * 32 + lane;  // this thread's weight row
       const bool nv = n < p.N;
-      const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + a * kTcTok;
+      const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + eh * (kTcTok / 2);
 #pragma unroll 1
-      for (int cc = 0; cc < kTcTok / 32; ++cc) {
+      for (int cc = 0; cc < kChunks; ++cc) {
         uint32_t v[32];
         tmem_ld_32x32b_x32(tbase + cc * 32, v);
         tmem_wait_ld();
-        const int m0 = tm * kTcTok + cc * 32;
+        if (cc == kChunks - 1) {
+          // the accumulator is read out: let the next tile's MMAs start
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(accempty_bar);
+        }
+        const int m0 = tm * kTcTok + eh * (kTcTok / 2) + cc * 32;
         if (nv && m0 < p.M) {
           if (p.out_f32) {
             float* dst = reinterpret_cast<float*>(p.y) + static_cast<int64_t>(m0) * p.N + n;
@@ -376,9 +384,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           }
         }
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(accempty_bar(a));
     }
   }
 
