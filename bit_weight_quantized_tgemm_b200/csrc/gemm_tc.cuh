@@ -8,20 +8,23 @@
 //
 // Tensor memory (512 columns x 128 lanes of 32 bits):
 //   columns [0, 256)             the f32 accumulator
-//   columns [256 + 32 s, +32)    A stage s (s < 8): 128 rows x 64 k of f16, element k of a
+//   columns [256 + 32 s, +32)    A stage s (s < 6): 128 rows x 64 k of f16, element k of a
 //                                row in column k/2 (low half for even k)
+// Stage s of the pipeline is the activation tile in shared memory plus A stage s; one
+// mbarrier says it is full (TMA bytes + the eight dequant warps) and one says it is
+// free (the MMA's commit), so the MMA thread waits once and commits once per stage.
 // With one accumulator the MMA waits while a finished tile is read out; eight epilogue
-// warps keep that short, and the eight A stages and the TMA stages keep filling
-// meanwhile, so the next tile starts with full queues.
+// warps keep that short, and the stages keep filling meanwhile, so the next tile starts
+// with full queues.
 //
 // Warp roles (18 warps, one CTA per SM):
 //   warp 0      TMA producer: activation tile, 256 tokens x 64 k (f16, 128-byte swizzle)
 //   warp 1      TMEM allocator and MMA issuer (one thread): 4 x tcgen05.mma 128x256x16
 //   warps 2-9   dequantizers: warp w handles TMEM lanes 32*(w%4).. (weight rows), warps
-//               2-5 the first 32 k of a stage and warps 6-9 the second; codes come
-//               straight from global memory (8 or 16 bytes per thread per stage, four
-//               stages ahead), are unpacked and scaled in f16 and stored with one
-//               tcgen05.st of 16 columns
+//               2-5 the first 32 k of a stage and warps 6-9 the second; codes and
+//               scales come straight from global memory (8 or 16 bytes per thread per
+//               stage, issued four stages ahead into alternating register sets), are
+//               unpacked and scaled in f16 and stored with one tcgen05.st of 16 columns
 //   warps 10-17 epilogue: warp w reads TMEM lanes 32*(w%4).. and half of the columns
 //               (tcgen05.ld), converts and stores y (lanes write consecutive n of one
 //               token row: coalesced)
@@ -46,13 +49,14 @@
 namespace tgemm {
 
 #ifndef TGEMM_TC_STAGES
-#define TGEMM_TC_STAGES 4
+#define TGEMM_TC_STAGES 6
 #endif
 constexpr int kTcRows = 128;   // weight rows per tile (MMA M)
 constexpr int kTcTok = 256;    // tokens per tile (MMA N)
 constexpr int kTcBK = 64;
-constexpr int kTcStages = TGEMM_TC_STAGES;  // activation stages (TMA)
-constexpr int kTcAStages = 8;               // dequantized-weight stages in TMEM
+// One ring of stages: stage s is an activation tile in shared memory plus an A tile in
+// TMEM, filled by the TMA producer and the dequant warps and released together.
+constexpr int kTcStages = TGEMM_TC_STAGES;
 constexpr int kTcEpiWarps = 8;
 constexpr int kTcThreads = (2 + 8 + kTcEpiWarps) * 32;
 constexpr int kTcXBytes = kTcTok * kTcBK * 2;   // 32 KB
@@ -60,14 +64,14 @@ constexpr int kTcTmemCols = 512;
 constexpr int kTcAccCols = kTcTok;              // f32 accumulator columns
 constexpr int kTcACol0 = kTcAccCols;            // first A-stage column
 constexpr int kTcACols = kTcBK / 2;             // columns per A stage (2 f16 per column)
-static_assert(kTcACol0 + kTcAStages * kTcACols <= kTcTmemCols, "TMEM budget");
+static_assert(kTcACol0 + kTcStages * kTcACols <= kTcTmemCols, "TMEM budget");
 
 template <int FMT>
 struct TcFmt {
   static constexpr int kWqRowBytes = FMT == 0 ? 16 : 32;  // packed bytes per row per stage
   static constexpr int kXOff = 0;
   static constexpr int kBarOff = kXOff + kTcStages * kTcXBytes;
-  static constexpr int kNumBars = 2 * kTcStages + 2 * kTcAStages + 4 + 1;
+  static constexpr int kNumBars = 2 * kTcStages + 2 + 1;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kSmemBytes = kMiscOff + 16 + 1024;  // + alignment slack
 };
@@ -137,11 +141,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const uint32_t bar0 = sbase + F::kBarOff;
   auto full_bar = [&](int s) { return bar0 + 8u * s; };
   auto empty_bar = [&](int s) { return bar0 + 8u * (kTcStages + s); };
-  auto wfull_bar = [&](int s) { return bar0 + 8u * (2 * kTcStages + s); };
-  auto wfree_bar = [&](int s) { return bar0 + 8u * (2 * kTcStages + kTcAStages + s); };
-  const uint32_t accfull_bar = bar0 + 8u * (2 * kTcStages + 2 * kTcAStages);
-  const uint32_t accempty_bar = bar0 + 8u * (2 * kTcStages + 2 * kTcAStages + 1);
-  const uint32_t drain_bar = bar0 + 8u * (2 * kTcStages + 2 * kTcAStages + 4);
+  const uint32_t accfull_bar = bar0 + 8u * (2 * kTcStages);
+  const uint32_t accempty_bar = bar0 + 8u * (2 * kTcStages + 1);
+  const uint32_t drain_bar = bar0 + 8u * (2 * kTcStages + 2);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + F::kMiscOff);
   volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + F::kMiscOff + 4);
 
@@ -149,12 +151,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kTcStages; ++s) {
-      mbar_init(full_bar(s), 1);       // producer's expect_tx
+      mbar_init(full_bar(s), 1 + 8);   // producer's expect_tx + 8 dequant warps
       mbar_init(empty_bar(s), 1);      // MMA commit
-    }
-    for (int s = 0; s < kTcAStages; ++s) {
-      mbar_init(wfull_bar(s), 8);      // 8 dequant warps
-      mbar_init(wfree_bar(s), 1);      // MMA commit
     }
     mbar_init(accfull_bar, 1);             // MMA commit
     mbar_init(accempty_bar, kTcEpiWarps);  // epilogue warps
@@ -204,19 +202,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     if (lane == 0) {
       constexpr uint32_t kIdescMain = make_idesc_f16(0u, kTcRows, kTcTok);  // f16 x f16
       constexpr uint32_t kIdescLora = make_idesc_f16(1u, kTcRows, kTcTok);  // bf16 x bf16
-      uint32_t it = 0, wit = 0, tcount = 0;
+      uint32_t it = 0, tcount = 0;
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x, ++tcount) {
         if (!mbar_wait(accempty_bar, (tcount & 1u) ^ 1u, abort_flag)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base;
-        for (int ks = 0; ks < ksteps; ++ks, ++it, ++wit) {
+        for (int ks = 0; ks < ksteps; ++ks, ++it) {
           const uint32_t s = it % kTcStages, ph = (it / kTcStages) & 1u;
-          const uint32_t ws = wit % kTcAStages, wph = (wit / kTcAStages) & 1u;
-          if (!mbar_wait(wfull_bar(ws), wph, abort_flag)) { ok = false; break; }
           if (!mbar_wait(full_bar(s), ph, abort_flag)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t a_tmem = tmem_base + kTcACol0 + ws * kTcACols;             // weights
+          const uint32_t a_tmem = tmem_base + kTcACol0 + s * kTcACols;              // weights
           const uint64_t bdesc = smem_desc_sw128(sbase + F::kXOff + s * kTcXBytes);  // tokens
           if (!LORA || ks < p.kt_main) {
 #pragma unroll
@@ -229,7 +225,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
               mma_f16_ts(d_tmem, a_tmem + 8u * kk, bdesc + 2u * kk, kIdescLora, 1u);
           }
           mma_commit(empty_bar(s));
-          mma_commit(wfree_bar(ws));
         }
         if (!ok) break;
         mma_commit(accfull_bar);
@@ -250,100 +245,121 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                             16u * half;
     uint32_t wit = 0;
     bool ok = true;
-    for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
-      const int tn = tile / p.tiles_m;
-      const int row = tn * kTcRows + rt;
-      const bool valid = row < p.N;
-      const uint16_t* srow = p.scales + static_cast<int64_t>(row) * nscale * (FMT == 0 ? 1 : 2);
-      const uint8_t* wrow_g = p.wq + static_cast<int64_t>(row) * wq_row + half * kHalfBytes;
-      // block (Q2) / group (4-bit) scales, loaded four blocks ahead of their use
-      auto load_scale = [&](int b) -> uint32_t {
-        if (!valid || b >= nscale) return 0u;
-        return FMT == 0 ? static_cast<uint32_t>(srow[b])
-                        : reinterpret_cast<const uint32_t*>(srow)[b];
-      };
-      // this thread's packed codes for stage ks, loaded four stages ahead through L1
-      auto load_codes = [&](int ks) -> uint4 {
-        if (!valid || ks >= p.kt_main) return make_uint4(0, 0, 0, 0);
-        const uint8_t* src = wrow_g + static_cast<int64_t>(ks) * F::kWqRowBytes;
-        if (FMT == 0) {
-          const uint2 v = __ldg(reinterpret_cast<const uint2*>(src));
-          return make_uint4(v.x, v.y, 0, 0);
-        }
-        return __ldg(reinterpret_cast<const uint4*>(src));
-      };
-      uint32_t q0 = load_scale(0), q1 = load_scale(1), q2 = load_scale(2), q3 = load_scale(3);
-      uint4 c0 = load_codes(0), c1 = load_codes(1), c2 = load_codes(2), c3 = load_codes(3);
-      uint32_t cur = 0;
-      for (int ks = 0; ks < ksteps; ++ks, ++wit) {
-        const uint4 pk = c0;
-        c0 = c1;
-        c1 = c2;
-        c2 = c3;
-        c3 = load_codes(ks + 4);
-        const bool main_stage = !LORA || ks < p.kt_main;
-        if (main_stage && (FMT == 1 || (ks & 1) == 0)) {
-          cur = q0;
-          q0 = q1;
-          q1 = q2;
-          q2 = q3;
-          q3 = load_scale((FMT == 0 ? (ks >> 1) : ks) + 4);
-        }
-        uint32_t o[16];
-        if (main_stage) {
-          if (FMT == 0) {
-            const uint32_t d2 = cur | (cur << 16);
-            q2_word_to_f16(pk.x, d2, o);
-            q2_word_to_f16(pk.y, d2, o + 8);
-          } else {
-            const uint32_t s2 = (cur & 0xFFFFu) | (cur << 16);
-            const uint32_t z2 = (cur >> 16) | (cur & 0xFFFF0000u);
-            q4_word_to_f16(pk.x, s2, z2, o);
-            q4_word_to_f16(pk.y, s2, z2, o + 4);
-            q4_word_to_f16(pk.z, s2, z2, o + 8);
-            q4_word_to_f16(pk.w, s2, z2, o + 12);
-          }
-        } else {
-          // low-rank stage: weight-side columns [j0, j0 + 32) of [B | B], zero beyond 2R
-          const int j0 = (ks - p.kt_main) * kTcBK + 32 * half;
-          const bool vec = (p.r & 7) == 0 && (reinterpret_cast<uintptr_t>(p.lb) & 15) == 0;
-#pragma unroll
-          for (int cq = 0; cq < 4; ++cq) {
-            const int jc = j0 + 8 * cq;
-            const int ic = jc < p.R ? jc : jc - p.R;
-            if (vec && jc < 2 * p.R && ic + 8 <= p.r) {
-              uint4 v = make_uint4(0, 0, 0, 0);
-              if (valid) v = *reinterpret_cast<const uint4*>(p.lb + static_cast<int64_t>(row) * p.r + ic);
-              o[4 * cq] = v.x;
-              o[4 * cq + 1] = v.y;
-              o[4 * cq + 2] = v.z;
-              o[4 * cq + 3] = v.w;
-              continue;
-            }
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              uint32_t v2 = 0;
-#pragma unroll
-              for (int h = 0; h < 2; ++h) {
-                const int j = jc + 2 * e + h;
-                const int i = j < p.R ? j : j - p.R;
-                uint32_t v = 0;
-                if (valid && j < 2 * p.R && i < p.r) v = p.lb[static_cast<int64_t>(row) * p.r + i];
-                v2 |= v << (16 * h);
-              }
-              o[4 * cq + e] = v2;
-            }
-          }
-        }
-        const uint32_t ws = wit % kTcAStages, wph = (wit / kTcAStages) & 1u;
-        if (!mbar_wait_warp(wfree_bar(ws), wph ^ 1u, abort_flag)) { ok = false; break; }
-        tc_fence_after();
-        tmem_st_32x32b_x16(a_lane + ws * kTcACols, o);
-        tmem_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(wfull_bar(ws));
+    // This CTA's work is one stream of (tile, stage) items, item i being stage i % ksteps
+    // of its (i / ksteps)-th tile; prefetching runs across tile boundaries, so a new
+    // tile's first stages are already loaded when the previous tile ends.
+    const int my_tiles = p.num_tiles > static_cast<int>(blockIdx.x)
+                             ? (p.num_tiles - 1 - static_cast<int>(blockIdx.x)) / static_cast<int>(gridDim.x) + 1
+                             : 0;
+    const int n_items = my_tiles * ksteps;
+    struct Item {
+      int ks;
+      int row;
+      bool valid;
+    };
+    auto decode = [&](int i) -> Item {
+      const int ti = i / ksteps;
+      const int tile = static_cast<int>(blockIdx.x) + ti * static_cast<int>(gridDim.x);
+      const int row = (tile / p.tiles_m) * kTcRows + rt;
+      return Item{i - ti * ksteps, row, i < n_items && row < p.N};
+    };
+    // Codes and scale of one item, issued four items before their use into two register
+    // sets used in turn (A for items 8j..8j+3, B for 8j+4..8j+7), so no register that a
+    // load is still filling is ever touched early.
+    auto fetch = [&](int i, uint4& c, uint32_t& sc) {
+      c = make_uint4(0, 0, 0, 0);
+      sc = 0u;
+      const Item it = decode(i);
+      if (!it.valid || it.ks >= p.kt_main) return;
+      const uint8_t* src = p.wq + static_cast<int64_t>(it.row) * wq_row + half * kHalfBytes +
+                           static_cast<int64_t>(it.ks) * F::kWqRowBytes;
+      const uint16_t* srow = p.scales + static_cast<int64_t>(it.row) * nscale * (FMT == 0 ? 1 : 2);
+      if (FMT == 0) {
+        const uint2 v = __ldg(reinterpret_cast<const uint2*>(src));
+        c = make_uint4(v.x, v.y, 0, 0);
+        sc = static_cast<uint32_t>(srow[it.ks >> 1]);
+      } else {
+        c = __ldg(reinterpret_cast<const uint4*>(src));
+        sc = reinterpret_cast<const uint32_t*>(srow)[it.ks];
       }
+    };
+    // Dequantize item i into the next A stage of TMEM.
+    auto process = [&](int i, const uint4& pk, uint32_t cur) {
+      if (!ok || i >= n_items) return;
+      const Item it = decode(i);
+      const int ks = it.ks;
+      uint32_t o[16];
+      if (!LORA || ks < p.kt_main) {
+        if (FMT == 0) {
+          const uint32_t d2 = cur | (cur << 16);
+          q2_word_to_f16(pk.x, d2, o);
+          q2_word_to_f16(pk.y, d2, o + 8);
+        } else {
+          const uint32_t s2 = (cur & 0xFFFFu) | (cur << 16);
+          const uint32_t z2 = (cur >> 16) | (cur & 0xFFFF0000u);
+          q4_word_to_f16(pk.x, s2, z2, o);
+          q4_word_to_f16(pk.y, s2, z2, o + 4);
+          q4_word_to_f16(pk.z, s2, z2, o + 8);
+          q4_word_to_f16(pk.w, s2, z2, o + 12);
+        }
+      } else {
+        // low-rank stage: weight-side columns [j0, j0 + 32) of [B | B], zero beyond 2R
+        const int j0 = (ks - p.kt_main) * kTcBK + 32 * half;
+        const bool vec = (p.r & 7) == 0 && (reinterpret_cast<uintptr_t>(p.lb) & 15) == 0;
+#pragma unroll
+        for (int cq = 0; cq < 4; ++cq) {
+          const int jc = j0 + 8 * cq;
+          const int ic = jc < p.R ? jc : jc - p.R;
+          if (vec && jc < 2 * p.R && ic + 8 <= p.r) {
+            uint4 v = make_uint4(0, 0, 0, 0);
+            if (it.valid) v = *reinterpret_cast<const uint4*>(p.lb + static_cast<int64_t>(it.row) * p.r + ic);
+            o[4 * cq] = v.x;
+            o[4 * cq + 1] = v.y;
+            o[4 * cq + 2] = v.z;
+            o[4 * cq + 3] = v.w;
+            continue;
+          }
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            uint32_t v2 = 0;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const int j = jc + 2 * e + h;
+              const int ii = j < p.R ? j : j - p.R;
+              uint32_t v = 0;
+              if (it.valid && j < 2 * p.R && ii < p.r) v = p.lb[static_cast<int64_t>(it.row) * p.r + ii];
+              v2 |= v << (16 * h);
+            }
+            o[4 * cq + e] = v2;
+          }
+        }
+      }
+      const uint32_t ws = wit % kTcStages, wph = (wit / kTcStages) & 1u;
+      if (!mbar_wait_warp(empty_bar(ws), wph ^ 1u, abort_flag)) {
+        ok = false;
+        return;
+      }
+      tc_fence_after();
+      tmem_st_32x32b_x16(a_lane + ws * kTcACols, o);
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(full_bar(ws));
+      ++wit;
+    };
+    uint4 ca[4], cb[4];
+    uint32_t sa[4], sb[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) fetch(j, ca[j], sa[j]);
+    for (int g = 0; ok && g < n_items; g += 8) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) fetch(g + 4 + j, cb[j], sb[j]);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) process(g + j, ca[j], sa[j]);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) fetch(g + 8 + j, ca[j], sa[j]);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) process(g + 4 + j, cb[j], sb[j]);
     }
   } else {
     // ------------------------------------------------------------ epilogue
@@ -358,6 +374,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const int n = tn * kTcRows + q * 32 + lane;  // this thread's weight row
       const bool nv = n < p.N;
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + eh * (kTcTok / 2);
+      const int mbase = tm * kTcTok + eh * (kTcTok / 2);
 #pragma unroll 1
       for (int cc = 0; cc < kChunks; ++cc) {
         uint32_t v[32];
@@ -369,7 +386,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           __syncwarp();
           if (lane == 0) mbar_arrive(accempty_bar);
         }
-        const int m0 = tm * kTcTok + eh * (kTcTok / 2) + cc * 32;
+        const int m0 = mbase + cc * 32;
         if (nv && m0 < p.M) {
           if (p.out_f32) {
             float* dst = reinterpret_cast<float*>(p.y) + static_cast<int64_t>(m0) * p.N + n;
