@@ -1,15 +1,17 @@
 // gemm_tc.cuh -- large-M path: persistent tcgen05 (5th-generation tensor core) kernel.
 //
 // Tile: 128 weight rows (MMA M, TMEM lanes) x 256 tokens (MMA N, accumulator columns),
-// 64 k per stage (an M=128 MMA costs the same time for any N up to 256, so N is 256).  The dequantized weights never touch shared memory: dequant warps write
+// 128 k per stage (an M=128 MMA costs the same time for any N up to 256, so N is 256;
+// a stage of eight K=16 MMAs keeps the single issuing thread's per-stage wait and commit
+// small next to the tensor core's work).  The dequantized weights never touch shared memory: dequant warps write
 // them straight into tensor memory (tcgen05.st) and the MMA reads its A operand from
 // there (tcgen05.mma ... [a_tmem]).  Shared memory then carries only the activation
 // tiles (TMA in, MMA out), which keeps its traffic at 128 bytes per MMA cycle.
 //
 // Tensor memory (512 columns x 128 lanes of 32 bits):
 //   columns [0, 256)             the f32 accumulator
-//   columns [256 + 32 s, +32)    A stage s (s < 6): 128 rows x 64 k of f16, element k of a
-//                                row in column k/2 (low half for even k)
+//   columns [256 + 64 s, +64)    A stage s (s < 3): 128 rows x 128 k of f16, element k of
+//                                a row in column k/2 (low half for even k)
 // Stage s of the pipeline is the activation tile in shared memory plus A stage s; one
 // mbarrier says it is full (TMA bytes + the eight dequant warps) and one says it is
 // free (the MMA's commit), so the MMA thread waits once and commits once per stage.
@@ -18,13 +20,14 @@
 // with full queues.
 //
 // Warp roles (18 warps, one CTA per SM):
-//   warp 0      TMA producer: activation tile, 256 tokens x 64 k (f16, 128-byte swizzle)
-//   warp 1      TMEM allocator and MMA issuer (one thread): 4 x tcgen05.mma 128x256x16
+//   warp 0      TMA producer: activation tile, 256 tokens x 128 k as two 64-k boxes (f16,
+//               128-byte swizzle)
+//   warp 1      TMEM allocator and MMA issuer (one thread): 8 x tcgen05.mma 128x256x16
 //   warps 2-9   dequantizers: warp w handles TMEM lanes 32*(w%4).. (weight rows), warps
-//               2-5 the first 32 k of a stage and warps 6-9 the second; codes and
-//               scales come straight from global memory (8 or 16 bytes per thread per
-//               stage, issued four stages ahead into alternating register sets), are
-//               unpacked and scaled in f16 and stored with one tcgen05.st of 16 columns
+//               2-5 the first 64 k of a stage and warps 6-9 the second; codes and
+//               scales come straight from global memory (16 or 32 bytes per thread per
+//               stage, issued ahead into alternating register sets), are unpacked and
+//               scaled in f16 and stored with one tcgen05.st of 32 columns
 //   warps 10-17 epilogue: warp w reads TMEM lanes 32*(w%4).. and half of the columns
 //               (tcgen05.ld), converts and stores y (lanes write consecutive n of one
 //               token row: coalesced)
@@ -49,17 +52,19 @@
 namespace tgemm {
 
 #ifndef TGEMM_TC_STAGES
-#define TGEMM_TC_STAGES 6
+#define TGEMM_TC_STAGES 3
 #endif
 constexpr int kTcRows = 128;   // weight rows per tile (MMA M)
 constexpr int kTcTok = 256;    // tokens per tile (MMA N)
-constexpr int kTcBK = 64;
+constexpr int kTcBK = 128;     // k per stage
+constexpr int kTcBox = 64;     // k per TMA box (one 128-byte swizzle row of f16)
 // One ring of stages: stage s is an activation tile in shared memory plus an A tile in
 // TMEM, filled by the TMA producer and the dequant warps and released together.
 constexpr int kTcStages = TGEMM_TC_STAGES;
 constexpr int kTcEpiWarps = 8;
 constexpr int kTcThreads = (2 + 8 + kTcEpiWarps) * 32;
-constexpr int kTcXBytes = kTcTok * kTcBK * 2;   // 32 KB
+constexpr int kTcXBytes = kTcTok * kTcBK * 2;   // 64 KB: two 32 KB boxes
+constexpr int kTcXBoxBytes = kTcTok * kTcBox * 2;
 constexpr int kTcTmemCols = 512;
 constexpr int kTcAccCols = kTcTok;              // f32 accumulator columns
 constexpr int kTcACol0 = kTcAccCols;            // first A-stage column
@@ -68,7 +73,7 @@ static_assert(kTcACol0 + kTcStages * kTcACols <= kTcTmemCols, "TMEM budget");
 
 template <int FMT>
 struct TcFmt {
-  static constexpr int kWqRowBytes = FMT == 0 ? 16 : 32;  // packed bytes per row per stage
+  static constexpr int kWqRowBytes = FMT == 0 ? 32 : 64;  // packed bytes per row per stage
   static constexpr int kXOff = 0;
   static constexpr int kBarOff = kXOff + kTcStages * kTcXBytes;
   static constexpr int kNumBars = 2 * kTcStages + 2 + 1;
@@ -79,7 +84,7 @@ struct TcFmt {
 struct TcParams {
   int M, N, K;
   int tiles_m, num_tiles;
-  int kt_main;     // K / 64
+  int kt_main;     // ceil(K / 128)
   int kt_lora;     // extra stages for the low-rank branch (0 without it)
   int lora_mmas;   // K=16 MMAs in those stages: 2 * round_up(r, 16) / 16
   int R;           // round_up(r, 16): width of u_hi (and of u_lo) in the concatenation
@@ -186,10 +191,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           if (!mbar_wait(empty_bar(s), ph ^ 1u, abort_flag)) { ok = false; break; }
           const uint32_t xdst = sbase + F::kXOff + s * kTcXBytes;
           mbar_arrive_expect_tx(full_bar(s), kTcXBytes);
-          if (ks < p.kt_main)
-            tma_load_2d(xdst, &tm_x, full_bar(s), ks * kTcBK, tm * kTcTok);
-          else
-            tma_load_2d(xdst, &tm_u, full_bar(s), (ks - p.kt_main) * kTcBK, tm * kTcTok);
+          const CUtensorMap* map = ks < p.kt_main ? &tm_x : &tm_u;
+          const int k0 = (ks < p.kt_main ? ks : ks - p.kt_main) * kTcBK;
+          tma_load_2d(xdst, map, full_bar(s), k0, tm * kTcTok);
+          tma_load_2d(xdst + kTcXBoxBytes, map, full_bar(s), k0 + kTcBox, tm * kTcTok);
         }
       }
       // every load issued must land before the CTA may exit
@@ -213,16 +218,21 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           if (!mbar_wait(full_bar(s), ph, abort_flag)) { ok = false; break; }
           tc_fence_after();
           const uint32_t a_tmem = tmem_base + kTcACol0 + s * kTcACols;              // weights
-          const uint64_t bdesc = smem_desc_sw128(sbase + F::kXOff + s * kTcXBytes);  // tokens
+          const uint32_t xs = sbase + F::kXOff + s * kTcXBytes;                      // tokens
+          // K=16 step kk reads columns 8kk.. of the A stage and 32-byte offset (kk % 4) in
+          // the (kk / 4)-th 64-k box of the activation tile
+          auto bdesc = [&](int kk) {
+            return smem_desc_sw128(xs + (kk >> 2) * kTcXBoxBytes) + 2u * (kk & 3);
+          };
           if (!LORA || ks < p.kt_main) {
 #pragma unroll
             for (int kk = 0; kk < kTcBK / 16; ++kk)
-              mma_f16_ts(d_tmem, a_tmem + 8u * kk, bdesc + 2u * kk, kIdescMain,
+              mma_f16_ts(d_tmem, a_tmem + 8u * kk, bdesc(kk), kIdescMain,
                          (ks > 0 || kk > 0) ? 1u : 0u);
           } else {
             const int done = (ks - p.kt_main) * (kTcBK / 16);
             for (int kk = 0; kk < kTcBK / 16 && done + kk < p.lora_mmas; ++kk)
-              mma_f16_ts(d_tmem, a_tmem + 8u * kk, bdesc + 2u * kk, kIdescLora, 1u);
+              mma_f16_ts(d_tmem, a_tmem + 8u * kk, bdesc(kk), kIdescLora, 1u);
           }
           mma_commit(empty_bar(s));
         }
@@ -237,12 +247,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     // ------------------------------------------------------------ dequantizers
     const int q = warp & 3;               // TMEM lane quarter this warp may access
     const int rt = 32 * q + lane;         // weight row within the tile
-    const int half = (warp - 2) >> 2;     // which 32 codes of the stage's 64
+    const int half = (warp - 2) >> 2;     // which 64 codes of the stage's 128
     const int nscale = FMT == 0 ? p.K / 128 : p.K / 64;
     const int64_t wq_row = FMT == 0 ? p.K / 4 : p.K / 2;
-    constexpr int kHalfBytes = F::kWqRowBytes / 2;  // 8 (Q2) or 16 (4-bit) bytes per stage
+    constexpr int kHalfBytes = F::kWqRowBytes / 2;  // 16 (Q2) or 32 (4-bit) bytes per stage
+    constexpr int kPf = FMT == 0 ? 3 : 2;           // items per prefetch register set
     const uint32_t a_lane = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + kTcACol0 +
-                            16u * half;
+                            32u * half;
     uint32_t wit = 0;
     bool ok = true;
     // This CTA's work is one stream of (tile, stage) items, item i being stage i % ksteps
@@ -263,51 +274,62 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const int row = (tile / p.tiles_m) * kTcRows + rt;
       return Item{i - ti * ksteps, row, i < n_items && row < p.N};
     };
-    // Codes and scale of one item, issued four items before their use into two register
-    // sets used in turn (A for items 8j..8j+3, B for 8j+4..8j+7), so no register that a
-    // load is still filling is ever touched early.
-    auto fetch = [&](int i, uint4& c, uint32_t& sc) {
-      c = make_uint4(0, 0, 0, 0);
-      sc = 0u;
+    struct Codes {
+      uint4 a, b;    // Q2 uses a (64 codes); 4-bit uses a and b (64 codes)
+      uint32_t sc;   // Q2 block scale d, or the 4-bit group's (s, z)
+    };
+    // Codes and scale of one item, issued ahead of their use into two register sets used
+    // in turn, so no register that a load is still filling is ever touched early.
+    auto fetch = [&](int i, Codes& c) {
+      c.a = make_uint4(0, 0, 0, 0);
+      c.b = c.a;
+      c.sc = 0u;
       const Item it = decode(i);
       if (!it.valid || it.ks >= p.kt_main) return;
-      const uint8_t* src = p.wq + static_cast<int64_t>(it.row) * wq_row + half * kHalfBytes +
-                           static_cast<int64_t>(it.ks) * F::kWqRowBytes;
+      const int k_first = it.ks * kTcBK + 64 * half;  // first k of this thread's 64
+      if (k_first >= p.K) return;                     // a 4-bit row ending mid-stage
+      const uint8_t* src = p.wq + static_cast<int64_t>(it.row) * wq_row +
+                           static_cast<int64_t>(it.ks) * F::kWqRowBytes + half * kHalfBytes;
       const uint16_t* srow = p.scales + static_cast<int64_t>(it.row) * nscale * (FMT == 0 ? 1 : 2);
+      c.a = __ldg(reinterpret_cast<const uint4*>(src));
       if (FMT == 0) {
-        const uint2 v = __ldg(reinterpret_cast<const uint2*>(src));
-        c = make_uint4(v.x, v.y, 0, 0);
-        sc = static_cast<uint32_t>(srow[it.ks >> 1]);
+        c.sc = static_cast<uint32_t>(srow[it.ks]);
       } else {
-        c = __ldg(reinterpret_cast<const uint4*>(src));
-        sc = reinterpret_cast<const uint32_t*>(srow)[it.ks];
+        c.b = __ldg(reinterpret_cast<const uint4*>(src) + 1);
+        c.sc = reinterpret_cast<const uint32_t*>(srow)[k_first / 64];
       }
     };
-    // Dequantize item i into the next A stage of TMEM.
-    auto process = [&](int i, const uint4& pk, uint32_t cur) {
+    // Dequantize item i into its A stage of TMEM.
+    auto process = [&](int i, const Codes& c) {
       if (!ok || i >= n_items) return;
       const Item it = decode(i);
       const int ks = it.ks;
-      uint32_t o[16];
+      uint32_t o[32];
       if (!LORA || ks < p.kt_main) {
         if (FMT == 0) {
-          const uint32_t d2 = cur | (cur << 16);
-          q2_word_to_f16(pk.x, d2, o);
-          q2_word_to_f16(pk.y, d2, o + 8);
+          const uint32_t d2 = c.sc | (c.sc << 16);
+          q2_word_to_f16(c.a.x, d2, o);
+          q2_word_to_f16(c.a.y, d2, o + 8);
+          q2_word_to_f16(c.a.z, d2, o + 16);
+          q2_word_to_f16(c.a.w, d2, o + 24);
         } else {
-          const uint32_t s2 = (cur & 0xFFFFu) | (cur << 16);
-          const uint32_t z2 = (cur >> 16) | (cur & 0xFFFF0000u);
-          q4_word_to_f16(pk.x, s2, z2, o);
-          q4_word_to_f16(pk.y, s2, z2, o + 4);
-          q4_word_to_f16(pk.z, s2, z2, o + 8);
-          q4_word_to_f16(pk.w, s2, z2, o + 12);
+          const uint32_t s2 = (c.sc & 0xFFFFu) | (c.sc << 16);
+          const uint32_t z2 = (c.sc >> 16) | (c.sc & 0xFFFF0000u);
+          q4_word_to_f16(c.a.x, s2, z2, o);
+          q4_word_to_f16(c.a.y, s2, z2, o + 4);
+          q4_word_to_f16(c.a.z, s2, z2, o + 8);
+          q4_word_to_f16(c.a.w, s2, z2, o + 12);
+          q4_word_to_f16(c.b.x, s2, z2, o + 16);
+          q4_word_to_f16(c.b.y, s2, z2, o + 20);
+          q4_word_to_f16(c.b.z, s2, z2, o + 24);
+          q4_word_to_f16(c.b.w, s2, z2, o + 28);
         }
       } else {
-        // low-rank stage: weight-side columns [j0, j0 + 32) of [B | B], zero beyond 2R
-        const int j0 = (ks - p.kt_main) * kTcBK + 32 * half;
+        // low-rank stage: weight-side columns [j0, j0 + 64) of [B | B], zero beyond 2R
+        const int j0 = (ks - p.kt_main) * kTcBK + 64 * half;
         const bool vec = (p.r & 7) == 0 && (reinterpret_cast<uintptr_t>(p.lb) & 15) == 0;
 #pragma unroll
-        for (int cq = 0; cq < 4; ++cq) {
+        for (int cq = 0; cq < 8; ++cq) {
           const int jc = j0 + 8 * cq;
           const int ic = jc < p.R ? jc : jc - p.R;
           if (vec && jc < 2 * p.R && ic + 8 <= p.r) {
@@ -340,26 +362,25 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         return;
       }
       tc_fence_after();
-      tmem_st_32x32b_x16(a_lane + ws * kTcACols, o);
+      tmem_st_32x32b_x32(a_lane + ws * kTcACols, o);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(full_bar(ws));
       ++wit;
     };
-    uint4 ca[4], cb[4];
-    uint32_t sa[4], sb[4];
+    Codes ca[kPf], cb[kPf];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) fetch(j, ca[j], sa[j]);
-    for (int g = 0; ok && g < n_items; g += 8) {
+    for (int j = 0; j < kPf; ++j) fetch(j, ca[j]);
+    for (int g = 0; ok && g < n_items; g += 2 * kPf) {
 #pragma unroll
-      for (int j = 0; j < 4; ++j) fetch(g + 4 + j, cb[j], sb[j]);
+      for (int j = 0; j < kPf; ++j) fetch(g + kPf + j, cb[j]);
 #pragma unroll
-      for (int j = 0; j < 4; ++j) process(g + j, ca[j], sa[j]);
+      for (int j = 0; j < kPf; ++j) process(g + j, ca[j]);
 #pragma unroll
-      for (int j = 0; j < 4; ++j) fetch(g + 8 + j, ca[j], sa[j]);
+      for (int j = 0; j < kPf; ++j) fetch(g + 2 * kPf + j, ca[j]);
 #pragma unroll
-      for (int j = 0; j < 4; ++j) process(g + 4 + j, cb[j], sb[j]);
+      for (int j = 0; j < kPf; ++j) process(g + kPf + j, cb[j]);
     }
   } else {
     // ------------------------------------------------------------ epilogue

@@ -175,7 +175,7 @@ int choose_path(int M) {
 
 struct LoraDims {
   int R;       // round_up(r, 16)
-  int wcat;    // width of [u_hi | u_lo | 0], a multiple of 64
+  int wcat;    // width of [u_hi | u_lo | 0], a multiple of the tensor-core stage (128)
   int L;       // pipeline stages for the branch
   int rpad;    // round_up(r, 64): columns of the partial sums
   int slices;  // K slices of the partial sums
@@ -184,8 +184,8 @@ struct LoraDims {
 LoraDims lora_dims(int r, int K) {
   LoraDims d;
   d.R = (r + 15) / 16 * 16;
-  d.wcat = (2 * d.R + 63) / 64 * 64;
-  d.L = d.wcat / 64;
+  d.wcat = (2 * d.R + kTcBK - 1) / kTcBK * kTcBK;
+  d.L = d.wcat / kTcBK;
   d.rpad = (r + 63) / 64 * 64;
   d.slices = (K + kLoraKc - 1) / kLoraKc;
   return d;
@@ -329,11 +329,11 @@ int run_gemm(int fmt, const uint16_t* x, const uint8_t* wq, const uint16_t* scal
     if (int e = launch_lora_down(x, la, M, K, r, ld, part, nullptr, ucat, st, di.sms)) return e;
   }
   CUtensorMap tm_x, tm_u;
-  if (int e = make_map_2d(&tm_x, x16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, K, M, kTcBK, kTcTok,
+  if (int e = make_map_2d(&tm_x, x16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, K, M, kTcBox, kTcTok,
                           CU_TENSOR_MAP_SWIZZLE_128B))
     return e;
   if (lora) {
-    if (int e = make_map_2d(&tm_u, ucat, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ld.wcat, M, kTcBK,
+    if (int e = make_map_2d(&tm_u, ucat, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ld.wcat, M, kTcBox,
                             kTcTok, CU_TENSOR_MAP_SWIZZLE_128B))
       return e;
   } else {
@@ -346,7 +346,7 @@ int run_gemm(int fmt, const uint16_t* x, const uint8_t* wq, const uint16_t* scal
   p.tiles_m = (M + kTcTok - 1) / kTcTok;
   const int tiles_n = (N + kTcRows - 1) / kTcRows;
   p.num_tiles = p.tiles_m * tiles_n;
-  p.kt_main = K / kTcBK;
+  p.kt_main = (K + kTcBK - 1) / kTcBK;
   p.kt_lora = lora ? ld.L : 0;
   p.lora_mmas = lora ? 2 * ld.R / 16 : 0;
   p.R = ld.R;
