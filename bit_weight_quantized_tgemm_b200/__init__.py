@@ -9,6 +9,7 @@ from .binding import (  # noqa: F401
     OUT_BF16, OUT_F32, PACK_BAD_CODE, PACK_INEXACT, PACK_NONFINITE, PATH_AUTO, PATH_SMALL_M,
     PATH_TENSOR, TgemmError, device_error, gemm_q2, gemm_q2_lora, gemm_q4, lib, library_path,
     q2_dequant, q2_pack, q4_dequant, q4_pack, set_path, version, workspace_size,
+    workspace_size_min,
     KIND_GEMV_Q2, KIND_GEMV_Q4, KIND_PREP, KIND_TC_Q2, KIND_TC_Q2_LORA, KIND_TC_Q4,
     launch_count, profile_enable, profile_read, ETOOLARGE, NOALLOC_SCRATCH_BYTES,
     gemm_q2_noalloc,

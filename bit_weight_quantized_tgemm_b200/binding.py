@@ -36,6 +36,7 @@ _SIGS = {
     "q2_dequant": (_i, [_P, _P, _P, _i, _i, _P]),
     "q4_dequant": (_i, [_P, _P, _P, _i, _i, _P]),
     "tgemm_workspace_size": (_sz, [_i, _i, _i, _i, _i]),
+    "tgemm_workspace_size_min": (_sz, [_i, _i, _i, _i, _i]),
     "tgemm_q2": (_i, [_P, _P, _P, _P, _i, _i, _i, _i, _P, _sz, _P]),
     "tgemm_q2_lora": (_i, [_P, _P, _P, _P, _P, _i, _P, _i, _i, _i, _i, _P, _sz, _P]),
     "tgemm_q4": (_i, [_P, _P, _P, _P, _i, _i, _i, _i, _P, _sz, _P]),
@@ -164,6 +165,11 @@ def q4_dequant(wq: torch.Tensor, sz: torch.Tensor) -> torch.Tensor:
 
 def workspace_size(op: int, M: int, N: int, K: int, r: int = 0) -> int:
     return int(lib().tgemm_workspace_size(op, M, N, K, r))
+
+
+def workspace_size_min(op: int, M: int, N: int, K: int, r: int = 0) -> int:
+    """Smallest accepted workspace (whole tiles per CTA); see tgemm_workspace_size_min."""
+    return int(lib().tgemm_workspace_size_min(op, M, N, K, r))
 
 
 _ws_cache = {}

@@ -1,5 +1,12 @@
 // gemm_tc.cuh -- large-M path: persistent tcgen05 (5th-generation tensor core) kernel.
 //
+// Schedule: a tile's work is `ksteps` units (its 128-k stages, then the branch's stages).
+// The units of all tiles, tile-major, are cut into equal contiguous ranges, one per CTA.
+// When the range length is a multiple of ksteps every CTA owns whole tiles; otherwise
+// (chosen by the host when tiles divide badly over the SMs, e.g. 40 or 152 tiles on 148
+// SMs) a tile can be shared by consecutive CTAs ("stream-K"): each writes its f32 partial
+// sum to a slot in the workspace and the last to arrive adds the slots in k order.
+//
 // Tile: 128 weight rows (MMA M, TMEM lanes) x 256 tokens (MMA N, accumulator columns),
 // 128 k per stage (an M=128 MMA costs the same time for any N up to 256, so N is 256;
 // a stage of eight K=16 MMAs keeps the single issuing thread's per-stage wait and commit
@@ -86,6 +93,9 @@ struct TcParams {
   int tiles_m, num_tiles;
   int kt_main;     // ceil(K / 128)
   int kt_lora;     // extra stages for the low-rank branch (0 without it)
+  int ksteps;      // kt_main + kt_lora: units of work per tile
+  int upc;         // units per CTA: CTA c owns units [c * upc, min(U, (c + 1) * upc))
+  int units;       // U = num_tiles * ksteps
   int lora_mmas;   // K=16 MMAs in those stages: 2 * round_up(r, 16) / 16
   int R;           // round_up(r, 16): width of u_hi (and of u_lo) in the concatenation
   int r;
@@ -94,7 +104,25 @@ struct TcParams {
   const uint16_t* scales;  // Q2: d [N][K/128]; 4-bit: sz [N][K/64][2]
   const uint16_t* lb;      // low-rank B [N][r] (bf16)
   void* y;
+  float* part;             // split tiles: 2 slots of 128 x 256 f32 per CTA
+  int* cnt;                // split tiles: 8 arrival counters per tile, zero at launch
 };
+
+// One tile's share of a CTA's unit range: tile `tile`, stages [ka, kb).
+struct TcSeg {
+  int tile, ka, kb;
+};
+__device__ __forceinline__ TcSeg tc_seg_at(const TcParams& p, int u, int u1) {
+  const int t = u / p.ksteps;
+  const int end = min(u1, (t + 1) * p.ksteps);
+  return TcSeg{t, u - t * p.ksteps, end - t * p.ksteps};
+}
+// Slot of the partial sum that CTA c writes for its segment of tile t: a segment that
+// starts mid-tile (or at the tile's start) is the CTA's first, any other its last.
+__device__ __forceinline__ int tc_slot(const TcParams& p, int c, int t) {
+  return c * p.upc >= t * p.ksteps ? 2 * c : 2 * c + 1;
+}
+constexpr int kTcSlotFloats = kTcRows * kTcTok;
 
 __device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity) {
   const uint64_t t0 = globaltimer_ns();
@@ -177,25 +205,25 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  const int ksteps = p.kt_main + (LORA ? p.kt_lora : 0);
+  const int ksteps = p.ksteps;
+  const int u0 = static_cast<int>(blockIdx.x) * p.upc;  // this CTA's units [u0, u1)
+  const int u1 = min(p.units, u0 + p.upc);
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       uint32_t it = 0;
-      bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
+      for (int u = u0; u < u1; ++u, ++it) {
+        const int tile = u / ksteps, ks = u - tile * ksteps;
         const int tm = tile % p.tiles_m;
-        for (int ks = 0; ks < ksteps; ++ks, ++it) {
-          const uint32_t s = it % kTcStages, ph = (it / kTcStages) & 1u;
-          if (!mbar_wait(empty_bar(s), ph ^ 1u, abort_flag)) { ok = false; break; }
-          const uint32_t xdst = sbase + F::kXOff + s * kTcXBytes;
-          mbar_arrive_expect_tx(full_bar(s), kTcXBytes);
-          const CUtensorMap* map = ks < p.kt_main ? &tm_x : &tm_u;
-          const int k0 = (ks < p.kt_main ? ks : ks - p.kt_main) * kTcBK;
-          tma_load_2d(xdst, map, full_bar(s), k0, tm * kTcTok);
-          tma_load_2d(xdst + kTcXBoxBytes, map, full_bar(s), k0 + kTcBox, tm * kTcTok);
-        }
+        const uint32_t s = it % kTcStages, ph = (it / kTcStages) & 1u;
+        if (!mbar_wait(empty_bar(s), ph ^ 1u, abort_flag)) break;
+        const uint32_t xdst = sbase + F::kXOff + s * kTcXBytes;
+        mbar_arrive_expect_tx(full_bar(s), kTcXBytes);
+        const CUtensorMap* map = ks < p.kt_main ? &tm_x : &tm_u;
+        const int k0 = (ks < p.kt_main ? ks : ks - p.kt_main) * kTcBK;
+        tma_load_2d(xdst, map, full_bar(s), k0, tm * kTcTok);
+        tma_load_2d(xdst + kTcXBoxBytes, map, full_bar(s), k0 + kTcBox, tm * kTcTok);
       }
       // every load issued must land before the CTA may exit
       const uint32_t n_issued = it;
@@ -207,13 +235,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     if (lane == 0) {
       constexpr uint32_t kIdescMain = make_idesc_f16(0u, kTcRows, kTcTok);  // f16 x f16
       constexpr uint32_t kIdescLora = make_idesc_f16(1u, kTcRows, kTcTok);  // bf16 x bf16
-      uint32_t it = 0, tcount = 0;
+      uint32_t it = 0, scount = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x, ++tcount) {
-        if (!mbar_wait(accempty_bar, (tcount & 1u) ^ 1u, abort_flag)) { ok = false; break; }
+      for (int u = u0; ok && u < u1; ++scount) {
+        const TcSeg sg = tc_seg_at(p, u, u1);
+        u += sg.kb - sg.ka;
+        if (!mbar_wait(accempty_bar, (scount & 1u) ^ 1u, abort_flag)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base;
-        for (int ks = 0; ks < ksteps; ++ks, ++it) {
+        for (int ks = sg.ka; ks < sg.kb; ++ks, ++it) {
           const uint32_t s = it % kTcStages, ph = (it / kTcStages) & 1u;
           if (!mbar_wait(full_bar(s), ph, abort_flag)) { ok = false; break; }
           tc_fence_after();
@@ -228,11 +258,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
             for (int kk = 0; kk < kTcBK / 16; ++kk)
               mma_f16_ts(d_tmem, a_tmem + 8u * kk, bdesc(kk), kIdescMain,
-                         (ks > 0 || kk > 0) ? 1u : 0u);
+                         (ks > sg.ka || kk > 0) ? 1u : 0u);
           } else {
             const int done = (ks - p.kt_main) * (kTcBK / 16);
             for (int kk = 0; kk < kTcBK / 16 && done + kk < p.lora_mmas; ++kk)
-              mma_f16_ts(d_tmem, a_tmem + 8u * kk, bdesc(kk), kIdescLora, 1u);
+              mma_f16_ts(d_tmem, a_tmem + 8u * kk, bdesc(kk), kIdescLora,
+                         (ks > sg.ka || kk > 0) ? 1u : 0u);
           }
           mma_commit(empty_bar(s));
         }
@@ -256,23 +287,20 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                             32u * half;
     uint32_t wit = 0;
     bool ok = true;
-    // This CTA's work is one stream of (tile, stage) items, item i being stage i % ksteps
-    // of its (i / ksteps)-th tile; prefetching runs across tile boundaries, so a new
-    // tile's first stages are already loaded when the previous tile ends.
-    const int my_tiles = p.num_tiles > static_cast<int>(blockIdx.x)
-                             ? (p.num_tiles - 1 - static_cast<int>(blockIdx.x)) / static_cast<int>(gridDim.x) + 1
-                             : 0;
-    const int n_items = my_tiles * ksteps;
+    // This CTA's work is one stream of (tile, stage) items, item i being unit u0 + i;
+    // prefetching runs across tile boundaries, so a new tile's first stages are already
+    // loaded when the previous tile ends.
+    const int n_items = u1 > u0 ? u1 - u0 : 0;
     struct Item {
       int ks;
       int row;
       bool valid;
     };
     auto decode = [&](int i) -> Item {
-      const int ti = i / ksteps;
-      const int tile = static_cast<int>(blockIdx.x) + ti * static_cast<int>(gridDim.x);
+      const int u = u0 + i;
+      const int tile = u / ksteps;
       const int row = (tile / p.tiles_m) * kTcRows + rt;
-      return Item{i - ti * ksteps, row, i < n_items && row < p.N};
+      return Item{u - tile * ksteps, row, i < n_items && row < p.N};
     };
     struct Codes {
       uint4 a, b;    // Q2 uses a (64 codes); 4-bit uses a and b (64 codes)
@@ -386,41 +414,95 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;                // TMEM lane quarter this warp may access
     const int eh = (warp - 10) >> 2;       // which half of the accumulator's columns
+    const int piece = warp - 10;           // this warp's 32 x 128 piece of the tile
     constexpr int kChunks = kTcTok / 32 / 2;
-    uint32_t tcount = 0;
-    for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++tcount) {
-      const int tm = tile % p.tiles_m, tn = tile / p.tiles_m;
-      if (!mbar_wait_warp(accfull_bar, tcount & 1u, abort_flag)) break;
+    constexpr int kPieceFloats = kTcSlotFloats / kTcEpiWarps;
+    uint32_t scount = 0;
+    for (int u = u0; u < u1; ++scount) {
+      const TcSeg sg = tc_seg_at(p, u, u1);
+      u += sg.kb - sg.ka;
+      const int tm = sg.tile % p.tiles_m, tn = sg.tile / p.tiles_m;
+      if (!mbar_wait_warp(accfull_bar, scount & 1u, abort_flag)) break;
       tc_fence_after();
       const int n = tn * kTcRows + q * 32 + lane;  // this thread's weight row
       const bool nv = n < p.N;
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + eh * (kTcTok / 2);
       const int mbase = tm * kTcTok + eh * (kTcTok / 2);
+      // y[m0 + e][n] for e < 32 (lanes write consecutive n: coalesced)
+      auto put = [&](int m0, const uint32_t (&v)[32]) {
+        if (!nv || m0 >= p.M) return;
+        if (p.out_f32) {
+          float* dst = reinterpret_cast<float*>(p.y) + static_cast<int64_t>(m0) * p.N + n;
+#pragma unroll
+          for (int e = 0; e < 32; ++e)
+            if (m0 + e < p.M) dst[static_cast<int64_t>(e) * p.N] = __uint_as_float(v[e]);
+        } else {
+          __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.y) + static_cast<int64_t>(m0) * p.N + n;
+#pragma unroll
+          for (int e = 0; e < 32; ++e)
+            if (m0 + e < p.M) dst[static_cast<int64_t>(e) * p.N] = __float2bfloat16_rn(__uint_as_float(v[e]));
+        }
+      };
+      if (sg.ka == 0 && sg.kb == ksteps) {
+        // the whole tile: accumulator -> y
+#pragma unroll 1
+        for (int cc = 0; cc < kChunks; ++cc) {
+          uint32_t v[32];
+          tmem_ld_32x32b_x32(tbase + cc * 32, v);
+          tmem_wait_ld();
+          if (cc == kChunks - 1) {
+            // the accumulator is read out: let the next segment's MMAs start
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(accempty_bar);
+          }
+          put(mbase + cc * 32, v);
+        }
+        continue;
+      }
+      // Part of a tile shared with other CTAs: write this piece's f32 partial sum to the
+      // CTA's slot; the warp that completes the piece's arrival count adds all slots of
+      // the tile in k order (deterministic) and stores y.  Nothing waits on another CTA.
+      float* mine = p.part + static_cast<int64_t>(tc_slot(p, blockIdx.x, sg.tile)) * kTcSlotFloats +
+                    piece * kPieceFloats;
 #pragma unroll 1
       for (int cc = 0; cc < kChunks; ++cc) {
         uint32_t v[32];
         tmem_ld_32x32b_x32(tbase + cc * 32, v);
         tmem_wait_ld();
         if (cc == kChunks - 1) {
-          // the accumulator is read out: let the next tile's MMAs start
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(accempty_bar);
         }
-        const int m0 = mbase + cc * 32;
-        if (nv && m0 < p.M) {
-          if (p.out_f32) {
-            float* dst = reinterpret_cast<float*>(p.y) + static_cast<int64_t>(m0) * p.N + n;
 #pragma unroll
-            for (int e = 0; e < 32; ++e)
-              if (m0 + e < p.M) dst[static_cast<int64_t>(e) * p.N] = __uint_as_float(v[e]);
-          } else {
-            __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.y) + static_cast<int64_t>(m0) * p.N + n;
+        for (int e = 0; e < 32; ++e) __stcg(mine + (cc * 32 + e) * 32 + lane, __uint_as_float(v[e]));
+      }
+      __threadfence();
+      __syncwarp();
+      int before = 0;
+      if (lane == 0) before = atomicAdd(p.cnt + sg.tile * kTcEpiWarps + piece, 1);
+      before = __shfl_sync(0xFFFFFFFFu, before, 0);
+      const int c_lo = sg.tile * ksteps / p.upc;
+      const int c_hi = ((sg.tile + 1) * ksteps - 1) / p.upc;
+      if (before != c_hi - c_lo) continue;  // another CTA's warp finishes this piece
+      __threadfence();
+#pragma unroll 1
+      for (int cc = 0; cc < kChunks; ++cc) {
+        float acc[32];
 #pragma unroll
-            for (int e = 0; e < 32; ++e)
-              if (m0 + e < p.M) dst[static_cast<int64_t>(e) * p.N] = __float2bfloat16_rn(__uint_as_float(v[e]));
-          }
+        for (int e = 0; e < 32; ++e) acc[e] = 0.f;
+#pragma unroll 1
+        for (int c = c_lo; c <= c_hi; ++c) {
+          const float* src = p.part + static_cast<int64_t>(tc_slot(p, c, sg.tile)) * kTcSlotFloats +
+                             piece * kPieceFloats + cc * 32 * 32 + lane;
+#pragma unroll
+          for (int e = 0; e < 32; ++e) acc[e] += __ldcg(src + e * 32);
         }
+        uint32_t v[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(acc[e]);
+        put(mbase + cc * 32, v);
       }
     }
   }
@@ -438,12 +520,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
 // bf16 [M][K] -> f16 [M][K] with the pair permutation the dequantizers produce
 // (FMT 0: within each 16-group, position 2i <- i, 2i+1 <- i+8; FMT 1: within each
-// 8-group, 2i <- i, 2i+1 <- i+4).  One thread per 16 elements.
+// 8-group, 2i <- i, 2i+1 <- i+4).  One thread per 16 elements.  It also zeroes the
+// matmul's `ncnt` split-tile arrival counters, which the matmul kernel that follows on
+// the stream expects at zero.
 template <int FMT>
 __global__ void __launch_bounds__(256) prep_x16_kernel(const uint16_t* __restrict__ x,
                                                        uint16_t* __restrict__ x16,
-                                                       int64_t ngroups) {
+                                                       int64_t ngroups, int* __restrict__ cnt,
+                                                       int ncnt) {
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < ncnt; i += stride)
+    cnt[i] = 0;
   for (int64_t gidx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; gidx < ngroups;
        gidx += stride) {
     const uint4* src = reinterpret_cast<const uint4*>(x) + 2 * gidx;

@@ -191,15 +191,50 @@ LoraDims lora_dims(int r, int K) {
   return d;
 }
 
+// Tensor-core schedule: units (tile, 128-k stage) cut into one contiguous range per CTA.
+// Whole tiles per CTA when the tiles fill the SMs evenly enough; otherwise ranges of
+// ceil(U / SMs) units that may split tiles between CTAs (see gemm_tc.cuh).
+constexpr int kDefaultSms = 148;    // sizes workspaces when no device is visible (B200)
+constexpr int kSplitPenalty = 2;    // units a split tile is charged (partial sums + fixup)
+
+struct TcSchedule {
+  int ksteps = 0, tiles_m = 0, num_tiles = 0, units = 0, upc = 0, grid = 0;
+  bool split = false;
+};
+
+TcSchedule tc_schedule(int M, int N, int K, int kt_lora, int sms) {
+  TcSchedule s;
+  s.ksteps = (K + kTcBK - 1) / kTcBK + kt_lora;
+  s.tiles_m = (M + kTcTok - 1) / kTcTok;
+  s.num_tiles = s.tiles_m * ((N + kTcRows - 1) / kTcRows);
+  s.units = s.num_tiles * s.ksteps;
+  const int waves = (s.num_tiles + sms - 1) / sms;
+  const int upc_whole = waves * s.ksteps;
+  const int upc_split = (s.units + sms - 1) / sms;
+  s.split = upc_split + kSplitPenalty < upc_whole;
+  s.upc = s.split ? upc_split : upc_whole;
+  s.grid = (s.units + s.upc - 1) / s.upc;
+  return s;
+}
+
+int sms_for_sizing() {
+  DeviceInfo di;
+  if (current_device_info(&di) == TGEMM_OK && di.sms > 0) return di.sms;
+  return kDefaultSms;
+}
+
 struct Workspace {
   size_t x16 = 0, x16_bytes = 0;    // f16 activations (tensor-core path)
   size_t ucat = 0, ucat_bytes = 0;  // [u_hi | u_lo] (tensor-core path)
   size_t u32 = 0, u32_bytes = 0;    // f32 u (small-M path)
   size_t part = 0, part_bytes = 0;  // f32 partial sums of u
+  size_t slots = 0, slots_bytes = 0;  // split tiles: f32 partial sums, 2 per CTA
+  size_t cnt = 0, cnt_bytes = 0;      // split tiles: arrival counters
   size_t total = 0;
+  size_t total_whole = 0;           // the same without the split-tile part
 };
 
-Workspace workspace_layout(int op, int M, int K, int r, int path) {
+Workspace workspace_layout(int op, int M, int N, int K, int r, int path, int sms) {
   Workspace w;
   size_t off = 0;
   const bool lora = op == TGEMM_OP_Q2_LORA;
@@ -222,6 +257,18 @@ Workspace workspace_layout(int op, int M, int K, int r, int path) {
     w.part = off;
     w.part_bytes = static_cast<size_t>(ld.slices) * M * ld.rpad * 4;
     off = round_up(off + w.part_bytes, 256);
+  }
+  w.total_whole = off;
+  if (path == TGEMM_PATH_TENSOR) {
+    const TcSchedule sc = tc_schedule(M, N, K, lora ? lora_dims(r, K).L : 0, sms);
+    if (sc.split) {
+      w.slots = off;
+      w.slots_bytes = static_cast<size_t>(2) * sc.grid * kTcSlotFloats * 4;
+      off = round_up(off + w.slots_bytes, 256);
+      w.cnt = off;
+      w.cnt_bytes = static_cast<size_t>(sc.num_tiles) * kTcEpiWarps * 4;
+      off = round_up(off + w.cnt_bytes, 256);
+    }
   }
   w.total = off;
   return w;
@@ -271,13 +318,17 @@ int run_gemm(int fmt, const uint16_t* x, const uint8_t* wq, const uint16_t* scal
   if (!aligned(scales, fmt == 0 ? 2 : 4)) return TGEMM_EALIGN;
   if (lora && (!aligned(la, 4) || !aligned(lb, 2))) return TGEMM_EALIGN;
   const int path = choose_path(M);
-  const Workspace wl = workspace_layout(op, M, K, r, path);
-  if (wl.total > 0) {
-    if (!workspace || ws_bytes < wl.total) return TGEMM_EWORKSPACE;
+  // the required size does not depend on the device (only the optional split-tile part does)
+  const size_t required = workspace_layout(op, M, N, K, r, path, kDefaultSms).total_whole;
+  if (required > 0) {
+    if (!workspace || ws_bytes < required) return TGEMM_EWORKSPACE;
     if (!aligned(workspace, 256)) return TGEMM_EALIGN;
   }
   DeviceInfo di;
   if (int st = current_device_info(&di)) return st;
+  const Workspace wl = workspace_layout(op, M, N, K, r, path, di.sms);
+  // split tiles only when the workspace has room for their partial sums
+  const bool split_ok = wl.slots_bytes > 0 && ws_bytes >= wl.total;
   const cudaStream_t st = as_stream(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   const int out_f32 = out_dtype == TGEMM_OUT_F32 ? 1 : 0;
@@ -313,14 +364,23 @@ int run_gemm(int fmt, const uint16_t* x, const uint8_t* wq, const uint16_t* scal
   }
 
   // ---- tensor-core path
+  TcSchedule sc = tc_schedule(M, N, K, lora ? ld.L : 0, di.sms);
+  if (sc.split && !split_ok) {
+    // whole tiles per CTA (the workspace holds no partial-sum slots)
+    sc.split = false;
+    sc.upc = (sc.num_tiles + di.sms - 1) / di.sms * sc.ksteps;
+    sc.grid = (sc.units + sc.upc - 1) / sc.upc;
+  }
+  int* cnt = sc.split ? reinterpret_cast<int*>(ws + wl.cnt) : nullptr;
+  const int ncnt = sc.split ? sc.num_tiles * kTcEpiWarps : 0;
   uint16_t* x16 = reinterpret_cast<uint16_t*>(ws + wl.x16);
   const int64_t ngroups = static_cast<int64_t>(M) * K / 16;
   const int pgrid = grid_for(ngroups, 256, di.sms);
   if (int e = launch(TGEMM_KIND_PREP, st, [&] {
         if (fmt == 0)
-          prep_x16_kernel<0><<<pgrid, 256, 0, st>>>(x, x16, ngroups);
+          prep_x16_kernel<0><<<pgrid, 256, 0, st>>>(x, x16, ngroups, cnt, ncnt);
         else
-          prep_x16_kernel<1><<<pgrid, 256, 0, st>>>(x, x16, ngroups);
+          prep_x16_kernel<1><<<pgrid, 256, 0, st>>>(x, x16, ngroups, cnt, ncnt);
       }))
     return e;
   uint16_t* ucat = nullptr;
@@ -343,11 +403,13 @@ int run_gemm(int fmt, const uint16_t* x, const uint8_t* wq, const uint16_t* scal
   p.M = M;
   p.N = N;
   p.K = K;
-  p.tiles_m = (M + kTcTok - 1) / kTcTok;
-  const int tiles_n = (N + kTcRows - 1) / kTcRows;
-  p.num_tiles = p.tiles_m * tiles_n;
+  p.tiles_m = sc.tiles_m;
+  p.num_tiles = sc.num_tiles;
   p.kt_main = (K + kTcBK - 1) / kTcBK;
   p.kt_lora = lora ? ld.L : 0;
+  p.ksteps = sc.ksteps;
+  p.upc = sc.upc;
+  p.units = sc.units;
   p.lora_mmas = lora ? 2 * ld.R / 16 : 0;
   p.R = ld.R;
   p.r = r;
@@ -356,7 +418,9 @@ int run_gemm(int fmt, const uint16_t* x, const uint8_t* wq, const uint16_t* scal
   p.scales = scales;
   p.lb = lb;
   p.y = y;
-  const int grid = p.num_tiles < di.sms ? p.num_tiles : di.sms;
+  p.part = sc.split ? reinterpret_cast<float*>(ws + wl.slots) : nullptr;
+  p.cnt = cnt;
+  const int grid = sc.grid;
   if (fmt == 0 && !lora) {
     if (int e = tc_prepare<0, false>()) return e;
     return launch(TGEMM_KIND_TC_Q2, st, [&] {
@@ -469,11 +533,17 @@ int q4_dequant(const uint8_t* wq, const uint16_t* sz, float* w, int N, int K, vo
 }
 
 size_t tgemm_workspace_size(int op, int M, int N, int K, int r) {
-  (void)N;
-  if (M < 1 || K < 1) return 0;
+  if (M < 1 || N < 1 || K < 1) return 0;
   if (op != TGEMM_OP_Q2 && op != TGEMM_OP_Q2_LORA && op != TGEMM_OP_Q4) return 0;
   if (op == TGEMM_OP_Q2_LORA && (r < 1 || r > 256)) return 0;
-  return workspace_layout(op, M, K, r, choose_path(M)).total;
+  return workspace_layout(op, M, N, K, r, choose_path(M), sms_for_sizing()).total;
+}
+
+size_t tgemm_workspace_size_min(int op, int M, int N, int K, int r) {
+  if (M < 1 || N < 1 || K < 1) return 0;
+  if (op != TGEMM_OP_Q2 && op != TGEMM_OP_Q2_LORA && op != TGEMM_OP_Q4) return 0;
+  if (op == TGEMM_OP_Q2_LORA && (r < 1 || r > 256)) return 0;
+  return workspace_layout(op, M, N, K, r, choose_path(M), kDefaultSms).total_whole;
 }
 
 int tgemm_q2(const uint16_t* x, const uint8_t* wq, const uint16_t* d, void* y, int M, int N,
@@ -493,7 +563,8 @@ int tgemm_q2_noalloc(const uint16_t* x, const uint8_t* wq, const uint16_t* d, vo
                      int N, int K, int out_dtype, void* stream) {
   if (!x || !wq || !d || !y) return TGEMM_EINVAL;
   if (M < 1 || N < 1 || K < 128 || K % 128) return TGEMM_EINVAL;
-  const size_t need = workspace_layout(TGEMM_OP_Q2, M, K, 0, choose_path(M)).total;
+  const size_t need =
+      workspace_layout(TGEMM_OP_Q2, M, N, K, 0, choose_path(M), sms_for_sizing()).total_whole;
   if (need > TGEMM_NOALLOC_SCRATCH_BYTES) return TGEMM_ETOOLARGE;
   void* scratch = nullptr;
   if (need > 0) {

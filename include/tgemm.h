@@ -61,7 +61,7 @@ extern "C" {
 #define TGEMM_EALIGN     -2 /* a pointer is not aligned as documented for its argument */
 #define TGEMM_ECUDA      -3 /* a CUDA runtime call or kernel launch failed */
 #define TGEMM_EARCH      -4 /* the current device is not compute capability 10.0 */
-#define TGEMM_EWORKSPACE -5 /* workspace missing or smaller than tgemm_workspace_size() */
+#define TGEMM_EWORKSPACE -5 /* workspace missing or smaller than tgemm_workspace_size_min() */
 #define TGEMM_ETOOLARGE  -6 /* tgemm_q2_noalloc: the problem needs more scratch than its
                                built-in buffer (TGEMM_NOALLOC_SCRATCH_BYTES) holds */
 
@@ -125,18 +125,30 @@ int q4_dequant(const uint8_t* wq, const uint16_t* sz, float* w, int N, int K, vo
 
 /*
  * tgemm_workspace_size -- bytes of workspace the matmul `op` (TGEMM_OP_*) needs for
- * these sizes under the current path setting (0 when none).  r is ignored unless op is
+ * these sizes under the current path setting to run its fastest schedule (0 when it
+ * needs none).  On the tensor-core path that schedule may split tiles between CTAs
+ * when the tiles fill the SMs unevenly, and then the size includes f32 partial sums
+ * (2 x 128 KB per CTA) and arrival counters; it depends on the current device's SM
+ * count (148 is assumed when no device is visible).  r is ignored unless op is
  * TGEMM_OP_Q2_LORA.  Returns 0 for invalid arguments as well; the matmul call then
  * reports the argument error.
  */
 size_t tgemm_workspace_size(int op, int M, int N, int K, int r);
 
 /*
+ * tgemm_workspace_size_min -- the smallest workspace the matmul accepts (0 when it
+ * needs none).  With less than tgemm_workspace_size() bytes the call keeps whole tiles
+ * per CTA; the results agree to f32 rounding of the partial sums.  Same arguments and
+ * error behaviour as tgemm_workspace_size.
+ */
+size_t tgemm_workspace_size_min(int op, int M, int N, int K, int r);
+
+/*
  * tgemm_q2 -- y = x . W^T for Q2_0 weights.
  *   x [M][K] bf16 (16-byte aligned), wq [N][K/4] (16-byte aligned), d [N][K/128] f16
  *   (2-byte aligned), y [M][N] (16-byte aligned), out_dtype TGEMM_OUT_*.
- *   workspace: device memory of at least tgemm_workspace_size(TGEMM_OP_Q2, M, N, K, 0)
- *   bytes (256-byte aligned; may be NULL when that size is 0).  The call overwrites it;
+ *   workspace: device memory of tgemm_workspace_size(TGEMM_OP_Q2, M, N, K, 0) bytes, or
+ *   at least tgemm_workspace_size_min() (256-byte aligned; may be NULL when that is 0).  The call overwrites it;
  *   calls sharing a workspace must not overlap on the GPU.
  *   Requires M, N >= 1, K % 128 == 0.
  */

@@ -60,9 +60,33 @@ def test_workspace_sizes():
         # small-M path: f32 u + the partial sums
         assert tg.workspace_size(tg.OP_Q2_LORA, 4, 9216, 3072, 64) == 4 * 64 * 4 + 6 * 4 * 64 * 4
         assert tg.workspace_size(tg.OP_Q2_LORA, 1536, 9216, 3072, 0) == 0  # invalid r
+        # whole tiles fill 148 SMs evenly here: minimum == full size
+        assert tg.workspace_size_min(tg.OP_Q2, 1536, 9216, 3072) == 1536 * 3072 * 2
+        assert tg.workspace_size_min(tg.OP_Q2_LORA, 1536, 9216, 3072, 64) == lora
         assert tg.workspace_size(9, 1, 1, 128) == 0
     finally:
         tg.set_path(prev)
+
+
+def test_split_tile_workspace():
+    """40 tiles of 76 stages on 148 SMs: 145 CTAs of 21 units, tiles split between them.
+    The full size adds two 128 KB f32 slots per CTA and 8 counters per tile."""
+    if tg.lib().tgemm_workspace_size(tg.OP_Q2, 1536, 9216, 3072, 0) == 0:
+        pytest.skip("path forced elsewhere")
+    x16 = 512 * 9728 * 2
+    assert tg.workspace_size_min(tg.OP_Q4, 512, 2560, 9728) == x16
+    if _visible_sms() not in (None, 148):
+        pytest.skip("sizes below assume 148 SMs")
+    slots = 2 * 145 * 128 * 256 * 4
+    assert tg.workspace_size(tg.OP_Q4, 512, 2560, 9728) == x16 + slots + 40 * 8 * 4
+
+
+def _visible_sms():
+    import torch
+
+    if not torch.cuda.is_available():
+        return None
+    return torch.cuda.get_device_properties(0).multi_processor_count
 
 
 P = ctypes.c_void_p
