@@ -102,6 +102,25 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
       : "memory");
 }
 
+// Four 8x8 b16 matrices from shared memory (lane l supplies the row address of matrix
+// l / 8, row l % 8); register i holds matrix i's fragment (row lane / 4, columns
+// 2 (lane % 4) and 2 (lane % 4) + 1).
+__device__ __forceinline__ void ldmatrix_x4(uint32_t saddr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(saddr));
+}
+
+// D += A B for one m16n8k16 tile, bf16 operands, f32 accumulators (legacy warp MMA).
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                               uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
+      "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
 // Make this thread's generic-proxy shared-memory writes visible to the async proxy
 // (tensor core reads of operands written with st.shared).
 __device__ __forceinline__ void fence_proxy_async_smem() {

@@ -558,6 +558,136 @@ __global__ void __launch_bounds__(256) prep_x16_kernel(const uint16_t* __restric
   }
 }
 
+// Activation prep and the branch's first product in one pass over x (tensor-core path
+// with the low-rank branch).  CTA (token block of kPlTok, K slice of kLoraKc):
+//   - writes the f16, pair-permuted copy of its x tile (as prep_x16_kernel);
+//   - keeps the bf16 tile in shared memory and multiplies it with the matching slice
+//     of A, 64 columns of u at a time (ldmatrix + mma.sync, f32 accumulation);
+//   - stores the slice's partial sums in part[slice][m][col] (f32, `rpad` columns).
+// lora_finalize_kernel then adds the slices in order.  Also zeroes `ncnt` counters.
+constexpr int kLoraKc = 512;      // K slice of the branch's partial sums
+constexpr int kPlTok = 64;
+constexpr int kPlPitch = kLoraKc + 8;  // bf16 elements per shared row (16-byte rows, no ldmatrix conflicts)
+constexpr int kPlSmemBytes = 2 * kPlTok * kPlPitch * 2;
+
+template <int FMT>
+__global__ void __launch_bounds__(256) prep_lora_kernel(const uint16_t* __restrict__ x,
+                                                        uint16_t* __restrict__ x16,
+                                                        const uint16_t* __restrict__ a, int M,
+                                                        int K, int r, int rpad,
+                                                        float* __restrict__ part,
+                                                        int* __restrict__ cnt, int ncnt,
+                                                        int a_vec) {
+  static_assert((kPlPitch * 2) % 16 == 0, "pitch");
+  extern __shared__ __align__(16) uint16_t pl_smem[];
+  uint16_t* xs = pl_smem;                     // [kPlTok][kPlPitch] bf16 x tile
+  uint16_t* as = pl_smem + kPlTok * kPlPitch;  // [64][kPlPitch] bf16 rows of A
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  {
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * gridDim.y * blockDim.x;
+    for (int64_t i = (static_cast<int64_t>(blockIdx.y) * gridDim.x + blockIdx.x) * blockDim.x + tid;
+         i < ncnt; i += stride)
+      cnt[i] = 0;
+  }
+  const int m0 = blockIdx.x * kPlTok;
+  const int k0 = blockIdx.y * kLoraKc;
+  // x tile: 64 rows x 32 groups of 16 (thread -> group, a warp covers one row)
+  for (int gi = tid; gi < kPlTok * 32; gi += 256) {
+    const int row = gi >> 5, g = gi & 31;
+    const int m = m0 + row, k = k0 + 16 * g;
+    uint4 v0 = make_uint4(0, 0, 0, 0), v1 = v0;
+    const bool in = m < M && k < K;
+    if (in) {
+      const uint4* src = reinterpret_cast<const uint4*>(x + static_cast<int64_t>(m) * K + k);
+      v0 = __ldg(src);
+      v1 = __ldg(src + 1);
+    }
+    uint4* sdst = reinterpret_cast<uint4*>(xs + row * kPlPitch + 16 * g);
+    sdst[0] = v0;
+    sdst[1] = v1;
+    if (in) {
+      const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+      float f[16];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        f[2 * i] = __uint_as_float(w[i] << 16);
+        f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+      }
+      uint32_t o[8];
+      if (FMT == 0) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) o[i] = pack_f16x2(f[i], f[i + 8]);
+      } else {
+#pragma unroll
+        for (int e8 = 0; e8 < 2; ++e8)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) o[4 * e8 + i] = pack_f16x2(f[8 * e8 + i], f[8 * e8 + i + 4]);
+      }
+      uint4* gdst = reinterpret_cast<uint4*>(x16 + static_cast<int64_t>(m) * K + k);
+      gdst[0] = make_uint4(o[0], o[1], o[2], o[3]);
+      gdst[1] = make_uint4(o[4], o[5], o[6], o[7]);
+    }
+  }
+  const int mt = warp & 3;   // 16-token row block of the warp
+  const int nh = warp >> 2;  // 32-column half of the 64-column chunk
+  const int ksteps = min(kLoraKc, K - k0) / 16;
+  for (int c0 = 0; c0 < rpad; c0 += 64) {
+    __syncthreads();  // x tile written (first pass) / previous A chunk consumed
+    for (int gi = tid; gi < 64 * 32; gi += 256) {
+      const int row = gi >> 5, g = gi & 31;
+      const int col = c0 + row, k = k0 + 16 * g;
+      uint4 v0 = make_uint4(0, 0, 0, 0), v1 = v0;
+      if (col < r && k < K) {
+        if (a_vec) {
+          const uint4* src = reinterpret_cast<const uint4*>(a + static_cast<int64_t>(col) * K + k);
+          v0 = __ldg(src);
+          v1 = __ldg(src + 1);
+        } else {  // A only 4-byte aligned
+          const uint32_t* src = reinterpret_cast<const uint32_t*>(a + static_cast<int64_t>(col) * K + k);
+          v0 = make_uint4(__ldg(src), __ldg(src + 1), __ldg(src + 2), __ldg(src + 3));
+          v1 = make_uint4(__ldg(src + 4), __ldg(src + 5), __ldg(src + 6), __ldg(src + 7));
+        }
+      }
+      uint4* sdst = reinterpret_cast<uint4*>(as + row * kPlPitch + 16 * g);
+      sdst[0] = v0;
+      sdst[1] = v1;
+    }
+    __syncthreads();
+    float acc[4][4];
+#pragma unroll
+    for (int t = 0; t < 4; ++t)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[t][e] = 0.f;
+    // ldmatrix row addresses: A (x) matrices (m 0-7 | 8-15) x (k 0-7 | 8-15);
+    // B (rows of A) matrices (n 0-7, k 0-7), (n 0-7, k 8-15), (n 8-15, k 0-7), (n 8-15, k 8-15)
+    const int mi = lane >> 3, rr = lane & 7;
+    const uint32_t xa = smem_u32(xs + (mt * 16 + (mi & 1) * 8 + rr) * kPlPitch + (mi >> 1) * 8);
+    const uint32_t ba = smem_u32(as + (nh * 32 + (mi >> 1) * 8 + rr) * kPlPitch + (mi & 1) * 8);
+    for (int ks = 0; ks < ksteps; ++ks) {
+      uint32_t af[4], b01[4], b23[4];
+      ldmatrix_x4(xa + ks * 32, af);
+      ldmatrix_x4(ba + ks * 32, b01);
+      ldmatrix_x4(ba + 16 * kPlPitch * 2 + ks * 32, b23);
+      mma_bf16_16816(acc[0], af, b01[0], b01[1]);
+      mma_bf16_16816(acc[1], af, b01[2], b01[3]);
+      mma_bf16_16816(acc[2], af, b23[0], b23[1]);
+      mma_bf16_16816(acc[3], af, b23[2], b23[3]);
+    }
+    // fragment (t, e): token mt*16 + lane/4 (+8 for e >= 2), column nh*32 + 8t + 2(lane%4) + (e&1)
+    const int g4 = lane >> 2, c4 = lane & 3;
+#pragma unroll
+    for (int t = 0; t < 4; ++t)
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int m = m0 + mt * 16 + g4 + 8 * h;
+        if (m >= M) continue;
+        const int col = c0 + nh * 32 + 8 * t + 2 * c4;
+        float2* dst = reinterpret_cast<float2*>(part + (static_cast<int64_t>(blockIdx.y) * M + m) * rpad + col);
+        *dst = make_float2(acc[t][2 * h], acc[t][2 * h + 1]);
+      }
+  }
+}
+
 // u = x A^T for the low-rank branch, in two deterministic phases (no atomics).
 // Phase 1 (lora_down_partial_kernel): CTA (token block of 16, K slice of kLoraKc, column
 // chunk of 64) accumulates its slice on mma.sync (bf16 in, f32 accumulate); its 8 warps
@@ -566,8 +696,6 @@ __global__ void __launch_bounds__(256) prep_x16_kernel(const uint16_t* __restric
 // Phase 2 (lora_finalize_kernel): sums the slices in a fixed order and writes u in f32
 // [M][r] (small-M path) and/or the concatenation ucat [M][wcat] =
 // [bf16(u) pad R | bf16(u - bf16(u)) pad R | 0] (tensor-core path).
-constexpr int kLoraKc = 512;
-
 __global__ void __launch_bounds__(256) lora_down_partial_kernel(
     const uint16_t* __restrict__ x, const uint16_t* __restrict__ a, int M, int K, int r,
     int rpad, float* __restrict__ part) {

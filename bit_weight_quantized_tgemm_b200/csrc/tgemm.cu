@@ -291,6 +291,16 @@ int launch_lora_down(const uint16_t* x, const uint16_t* la, int M, int K, int r,
   });
 }
 
+int prep_lora_prepare() {
+  static std::once_flag once;
+  static cudaError_t err = cudaSuccess;
+  std::call_once(once, [] {
+    err = cudaFuncSetAttribute(prep_lora_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               kPlSmemBytes);
+  });
+  return err == cudaSuccess ? TGEMM_OK : TGEMM_ECUDA;
+}
+
 template <int FMT, bool LORA>
 int gemv_prepare() {
   static std::once_flag once;
@@ -374,19 +384,34 @@ int run_gemm(int fmt, const uint16_t* x, const uint8_t* wq, const uint16_t* scal
   int* cnt = sc.split ? reinterpret_cast<int*>(ws + wl.cnt) : nullptr;
   const int ncnt = sc.split ? sc.num_tiles * kTcEpiWarps : 0;
   uint16_t* x16 = reinterpret_cast<uint16_t*>(ws + wl.x16);
-  const int64_t ngroups = static_cast<int64_t>(M) * K / 16;
-  const int pgrid = grid_for(ngroups, 256, di.sms);
-  if (int e = launch(TGEMM_KIND_PREP, st, [&] {
-        if (fmt == 0)
-          prep_x16_kernel<0><<<pgrid, 256, 0, st>>>(x, x16, ngroups, cnt, ncnt);
-        else
-          prep_x16_kernel<1><<<pgrid, 256, 0, st>>>(x, x16, ngroups, cnt, ncnt);
-      }))
-    return e;
   uint16_t* ucat = nullptr;
   if (lora) {
+    // one pass over x: the f16 copy and the slices of u = x A^T; then u -> [u_hi | u_lo]
     ucat = reinterpret_cast<uint16_t*>(ws + wl.ucat);
-    if (int e = launch_lora_down(x, la, M, K, r, ld, part, nullptr, ucat, st, di.sms)) return e;
+    if (int e = prep_lora_prepare()) return e;
+    const dim3 grid((M + kPlTok - 1) / kPlTok, ld.slices);
+    const int a_vec = aligned(la, 16) ? 1 : 0;
+    if (int e = launch(TGEMM_KIND_PREP, st, [&] {
+          prep_lora_kernel<0><<<grid, 256, kPlSmemBytes, st>>>(x, x16, la, M, K, r, ld.rpad, part,
+                                                               cnt, ncnt, a_vec);
+        }))
+      return e;
+    const int fgrid = grid_for(static_cast<int64_t>(M) * ld.wcat, 256, di.sms);
+    if (int e = launch(TGEMM_KIND_PREP, st, [&] {
+          lora_finalize_kernel<<<fgrid, 256, 0, st>>>(part, ld.slices, M, r, ld.rpad, ld.R, ld.wcat,
+                                                      nullptr, ucat);
+        }))
+      return e;
+  } else {
+    const int64_t ngroups = static_cast<int64_t>(M) * K / 16;
+    const int pgrid = grid_for(ngroups, 256, di.sms);
+    if (int e = launch(TGEMM_KIND_PREP, st, [&] {
+          if (fmt == 0)
+            prep_x16_kernel<0><<<pgrid, 256, 0, st>>>(x, x16, ngroups, cnt, ncnt);
+          else
+            prep_x16_kernel<1><<<pgrid, 256, 0, st>>>(x, x16, ngroups, cnt, ncnt);
+        }))
+      return e;
   }
   CUtensorMap tm_x, tm_u;
   if (int e = make_map_2d(&tm_x, x16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, K, M, kTcBox, kTcTok,

@@ -92,6 +92,28 @@ def test_q2_lora_shapes(oracle, path, pname, M, N, K, r):
 
 
 @pytest.mark.parametrize("pname", list(PATHS))
+def test_lora_a_only_4_byte_aligned(oracle, path, pname):
+    """A at a 4-byte (not 16-byte) boundary, which the ABI allows: the branch's loads of A
+    take the narrow path.  Token and K extents span several prep tiles and a ragged edge."""
+    path(PATHS[pname])
+    M, N, K, r = 150 if pname == "tensor" else 9, 256, 1152, 24
+    prob = synth.q2_problem((22, M, N, K, r), M, N, K, r=r, ab_sigma=0.05)
+    wq, d, twq, td = _q2_device(prob, oracle)
+    a_dev = dev(prob.a, torch.bfloat16)
+    a_buf = torch.empty(r * K + 2, dtype=torch.bfloat16, device="cuda")
+    a = a_buf[2:].view(r, K)
+    a.copy_(a_dev)
+    assert a.data_ptr() % 16 == 4
+    y, buf = nan_filled((M, N), torch.float32)
+    tg.gemm_q2_lora(dev(prob.x, torch.bfloat16), twq, td, a, dev(prob.b, torch.bfloat16),
+                    out_dtype=tg.OUT_F32, y=y)
+    torch.cuda.synchronize()
+    assert canary_intact(buf, M * N)
+    gate_output(y, oracle.q2_lora_gemm(prob.x, wq, d, prob.a, prob.b, N), oracle,
+                f"lora a+4B {pname}")
+
+
+@pytest.mark.parametrize("pname", list(PATHS))
 def test_lora_branch_alone(oracle, path, pname):
     """W == 0 (all codes 1), A, B ~ N(0,1): the output is the branch alone."""
     path(PATHS[pname])
