@@ -283,9 +283,18 @@ def version() -> int:
     return int(lib().tgemm_version())
 
 
-def profile_enable(on: bool) -> bool:
-    """Record CUDA events around every launch (see tgemm_profile_enable)."""
-    return bool(lib().tgemm_profile_enable(1 if on else 0))
+PROFILE_ALL = (1 << 6) - 1
+
+
+def profile_enable(kinds) -> int:
+    """Record CUDA events around launches of the kernel kinds in the bit mask ``kinds``
+    (``True`` = every kind, ``False`` = none; see tgemm_profile_enable).  Returns the
+    previous mask."""
+    if kinds is True:
+        kinds = PROFILE_ALL
+    elif kinds is False or kinds is None:
+        kinds = 0
+    return int(lib().tgemm_profile_enable(int(kinds)))
 
 
 def profile_read(kind: int, reset: bool = True):

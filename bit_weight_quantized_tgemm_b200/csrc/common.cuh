@@ -121,6 +121,17 @@ __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+// Programmatic dependent launch.  Every kernel of the library is launched so that the
+// next kernel on the stream may be scheduled before it ends; each kernel first lets its
+// own dependent be scheduled, then waits until the kernels it depends on have finished
+// and their memory is visible, and only after that touches global memory.  A dependent
+// grid is scheduled only once every CTA of this one has passed the trigger (so all of
+// them are resident): waiting CTAs never hold resources this grid still needs.
+__device__ __forceinline__ void pdl_trigger_and_wait() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 // Make this thread's generic-proxy shared-memory writes visible to the async proxy
 // (tensor core reads of operands written with st.shared).
 __device__ __forceinline__ void fence_proxy_async_smem() {

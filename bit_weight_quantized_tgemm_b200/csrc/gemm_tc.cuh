@@ -204,6 +204,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  pdl_trigger_and_wait();  // everything above touched only shared and tensor memory
   const uint32_t tmem_base = *tmem_slot;
   const int ksteps = p.ksteps;
   const int u0 = static_cast<int>(blockIdx.x) * p.upc;  // this CTA's units [u0, u1)
@@ -518,9 +519,33 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
 // ---- activation preparation ---------------------------------------------------------
 
+// One 16-element group: bf16 -> f16 with the pair permutation of format FMT.
+template <int FMT>
+__device__ __forceinline__ void x16_group(const uint4& v0, const uint4& v1, uint4* dst) {
+  const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+  float f[16];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    f[2 * i] = __uint_as_float(w[i] << 16);
+    f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+  }
+  uint32_t o[8];
+  if (FMT == 0) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) o[i] = pack_f16x2(f[i], f[i + 8]);
+  } else {
+#pragma unroll
+    for (int e8 = 0; e8 < 2; ++e8)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) o[4 * e8 + i] = pack_f16x2(f[8 * e8 + i], f[8 * e8 + i + 4]);
+  }
+  dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
+  dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
+}
+
 // bf16 [M][K] -> f16 [M][K] with the pair permutation the dequantizers produce
 // (FMT 0: within each 16-group, position 2i <- i, 2i+1 <- i+8; FMT 1: within each
-// 8-group, 2i <- i, 2i+1 <- i+4).  One thread per 16 elements.  It also zeroes the
+// 8-group, 2i <- i, 2i+1 <- i+4).  Up to four 16-element groups per thread per round.  It also zeroes the
 // matmul's `ncnt` split-tile arrival counters, which the matmul kernel that follows on
 // the stream expects at zero.
 template <int FMT>
@@ -528,33 +553,28 @@ __global__ void __launch_bounds__(256) prep_x16_kernel(const uint16_t* __restric
                                                        uint16_t* __restrict__ x16,
                                                        int64_t ngroups, int* __restrict__ cnt,
                                                        int ncnt) {
-  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < ncnt; i += stride)
-    cnt[i] = 0;
-  for (int64_t gidx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; gidx < ngroups;
-       gidx += stride) {
-    const uint4* src = reinterpret_cast<const uint4*>(x) + 2 * gidx;
-    const uint4 a = __ldg(src), b = __ldg(src + 1);
-    const uint32_t v[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-    float f[16];
+  pdl_trigger_and_wait();
+  const int64_t nthreads = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  const int64_t first = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  for (int64_t i = first; i < ncnt; i += nthreads) cnt[i] = 0;
+  const uint4* src = reinterpret_cast<const uint4*>(x);
+  uint4* dst = reinterpret_cast<uint4*>(x16);
+  // up to four groups per thread per round, all loads issued before any conversion
+  for (int64_t base = first; base < ngroups; base += 4 * nthreads) {
+    uint4 v[4][2];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      f[2 * i] = __uint_as_float(v[i] << 16);
-      f[2 * i + 1] = __uint_as_float(v[i] & 0xFFFF0000u);
+    for (int j = 0; j < 4; ++j) {
+      const int64_t g = base + j * nthreads;
+      if (g < ngroups) {
+        v[j][0] = __ldg(src + 2 * g);
+        v[j][1] = __ldg(src + 2 * g + 1);
+      }
     }
-    uint32_t o[8];
-    if (FMT == 0) {
 #pragma unroll
-      for (int i = 0; i < 8; ++i) o[i] = pack_f16x2(f[i], f[i + 8]);
-    } else {
-#pragma unroll
-      for (int e8 = 0; e8 < 2; ++e8)
-#pragma unroll
-        for (int i = 0; i < 4; ++i) o[4 * e8 + i] = pack_f16x2(f[8 * e8 + i], f[8 * e8 + i + 4]);
+    for (int j = 0; j < 4; ++j) {
+      const int64_t g = base + j * nthreads;
+      if (g < ngroups) x16_group<FMT>(v[j][0], v[j][1], dst + 2 * g);
     }
-    uint4* dst = reinterpret_cast<uint4*>(x16) + 2 * gidx;
-    dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
-    dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
   }
 }
 
@@ -578,6 +598,7 @@ __global__ void __launch_bounds__(256) prep_lora_kernel(const uint16_t* __restri
                                                         float* __restrict__ part,
                                                         int* __restrict__ cnt, int ncnt,
                                                         int a_vec) {
+  pdl_trigger_and_wait();
   static_assert((kPlPitch * 2) % 16 == 0, "pitch");
   extern __shared__ __align__(16) uint16_t pl_smem[];
   uint16_t* xs = pl_smem;                     // [kPlTok][kPlPitch] bf16 x tile
@@ -591,41 +612,34 @@ __global__ void __launch_bounds__(256) prep_lora_kernel(const uint16_t* __restri
   }
   const int m0 = blockIdx.x * kPlTok;
   const int k0 = blockIdx.y * kLoraKc;
-  // x tile: 64 rows x 32 groups of 16 (thread -> group, a warp covers one row)
-  for (int gi = tid; gi < kPlTok * 32; gi += 256) {
-    const int row = gi >> 5, g = gi & 31;
-    const int m = m0 + row, k = k0 + 16 * g;
-    uint4 v0 = make_uint4(0, 0, 0, 0), v1 = v0;
-    const bool in = m < M && k < K;
-    if (in) {
-      const uint4* src = reinterpret_cast<const uint4*>(x + static_cast<int64_t>(m) * K + k);
-      v0 = __ldg(src);
-      v1 = __ldg(src + 1);
+  // x tile: 64 rows x 32 groups of 16 (thread -> group, a warp covers one row); each
+  // thread's 8 groups are loaded 4 at a time before any is stored
+#pragma unroll 1
+  for (int half = 0; half < 2; ++half) {
+    uint4 v[4][2];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int gi = tid + 256 * (4 * half + j);
+      const int row = gi >> 5, g = gi & 31;
+      const int m = m0 + row, k = k0 + 16 * g;
+      v[j][0] = make_uint4(0, 0, 0, 0);
+      v[j][1] = v[j][0];
+      if (m < M && k < K) {
+        const uint4* src = reinterpret_cast<const uint4*>(x + static_cast<int64_t>(m) * K + k);
+        v[j][0] = __ldg(src);
+        v[j][1] = __ldg(src + 1);
+      }
     }
-    uint4* sdst = reinterpret_cast<uint4*>(xs + row * kPlPitch + 16 * g);
-    sdst[0] = v0;
-    sdst[1] = v1;
-    if (in) {
-      const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-      float f[16];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        f[2 * i] = __uint_as_float(w[i] << 16);
-        f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
-      }
-      uint32_t o[8];
-      if (FMT == 0) {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) o[i] = pack_f16x2(f[i], f[i + 8]);
-      } else {
-#pragma unroll
-        for (int e8 = 0; e8 < 2; ++e8)
-#pragma unroll
-          for (int i = 0; i < 4; ++i) o[4 * e8 + i] = pack_f16x2(f[8 * e8 + i], f[8 * e8 + i + 4]);
-      }
-      uint4* gdst = reinterpret_cast<uint4*>(x16 + static_cast<int64_t>(m) * K + k);
-      gdst[0] = make_uint4(o[0], o[1], o[2], o[3]);
-      gdst[1] = make_uint4(o[4], o[5], o[6], o[7]);
+    for (int j = 0; j < 4; ++j) {
+      const int gi = tid + 256 * (4 * half + j);
+      const int row = gi >> 5, g = gi & 31;
+      const int m = m0 + row, k = k0 + 16 * g;
+      uint4* sdst = reinterpret_cast<uint4*>(xs + row * kPlPitch + 16 * g);
+      sdst[0] = v[j][0];
+      sdst[1] = v[j][1];
+      if (m < M && k < K)
+        x16_group<FMT>(v[j][0], v[j][1], reinterpret_cast<uint4*>(x16 + static_cast<int64_t>(m) * K + k));
     }
   }
   const int mt = warp & 3;   // 16-token row block of the warp
@@ -633,24 +647,36 @@ __global__ void __launch_bounds__(256) prep_lora_kernel(const uint16_t* __restri
   const int ksteps = min(kLoraKc, K - k0) / 16;
   for (int c0 = 0; c0 < rpad; c0 += 64) {
     __syncthreads();  // x tile written (first pass) / previous A chunk consumed
-    for (int gi = tid; gi < 64 * 32; gi += 256) {
-      const int row = gi >> 5, g = gi & 31;
-      const int col = c0 + row, k = k0 + 16 * g;
-      uint4 v0 = make_uint4(0, 0, 0, 0), v1 = v0;
-      if (col < r && k < K) {
-        if (a_vec) {
-          const uint4* src = reinterpret_cast<const uint4*>(a + static_cast<int64_t>(col) * K + k);
-          v0 = __ldg(src);
-          v1 = __ldg(src + 1);
-        } else {  // A only 4-byte aligned
-          const uint32_t* src = reinterpret_cast<const uint32_t*>(a + static_cast<int64_t>(col) * K + k);
-          v0 = make_uint4(__ldg(src), __ldg(src + 1), __ldg(src + 2), __ldg(src + 3));
-          v1 = make_uint4(__ldg(src + 4), __ldg(src + 5), __ldg(src + 6), __ldg(src + 7));
+#pragma unroll 1
+    for (int half = 0; half < 2; ++half) {
+      uint4 v[4][2];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int gi = tid + 256 * (4 * half + j);
+        const int row = gi >> 5, g = gi & 31;
+        const int col = c0 + row, k = k0 + 16 * g;
+        v[j][0] = make_uint4(0, 0, 0, 0);
+        v[j][1] = v[j][0];
+        if (col < r && k < K) {
+          if (a_vec) {
+            const uint4* src = reinterpret_cast<const uint4*>(a + static_cast<int64_t>(col) * K + k);
+            v[j][0] = __ldg(src);
+            v[j][1] = __ldg(src + 1);
+          } else {  // A only 4-byte aligned
+            const uint32_t* src = reinterpret_cast<const uint32_t*>(a + static_cast<int64_t>(col) * K + k);
+            v[j][0] = make_uint4(__ldg(src), __ldg(src + 1), __ldg(src + 2), __ldg(src + 3));
+            v[j][1] = make_uint4(__ldg(src + 4), __ldg(src + 5), __ldg(src + 6), __ldg(src + 7));
+          }
         }
       }
-      uint4* sdst = reinterpret_cast<uint4*>(as + row * kPlPitch + 16 * g);
-      sdst[0] = v0;
-      sdst[1] = v1;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int gi = tid + 256 * (4 * half + j);
+        const int row = gi >> 5, g = gi & 31;
+        uint4* sdst = reinterpret_cast<uint4*>(as + row * kPlPitch + 16 * g);
+        sdst[0] = v[j][0];
+        sdst[1] = v[j][1];
+      }
     }
     __syncthreads();
     float acc[4][4];
@@ -699,6 +725,7 @@ __global__ void __launch_bounds__(256) prep_lora_kernel(const uint16_t* __restri
 __global__ void __launch_bounds__(256) lora_down_partial_kernel(
     const uint16_t* __restrict__ x, const uint16_t* __restrict__ a, int M, int K, int r,
     int rpad, float* __restrict__ part) {
+  pdl_trigger_and_wait();
   __shared__ float red[8][16][65];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, c = lane & 3;
@@ -762,6 +789,7 @@ __global__ void __launch_bounds__(256) lora_finalize_kernel(const float* __restr
                                                             int R, int wcat,
                                                             float* __restrict__ u32,
                                                             uint16_t* __restrict__ ucat) {
+  pdl_trigger_and_wait();
   const int64_t total = static_cast<int64_t>(M) * wcat;
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;

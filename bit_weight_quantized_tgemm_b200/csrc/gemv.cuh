@@ -115,6 +115,7 @@ __global__ void __launch_bounds__(256) gemv_kernel(
     fence_mbar_init();
   }
   __syncthreads();
+  pdl_trigger_and_wait();
   uint32_t phase = 0;
 
   for (int m0 = 0; m0 < M; m0 += 16) {

@@ -39,6 +39,7 @@ __global__ void __launch_bounds__(256) q2_pack_kernel(const uint8_t* __restrict_
                                                       uint8_t* __restrict__ wq,
                                                       uint16_t* __restrict__ d, int64_t n_units,
                                                       int64_t n_scales, uint32_t* status) {
+  pdl_trigger_and_wait();
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
   const int64_t tid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   const int64_t iters = (n_units > n_scales ? n_units : n_scales);
@@ -78,6 +79,7 @@ __global__ void __launch_bounds__(256) q4_pack_kernel(const uint8_t* __restrict_
                                                       uint8_t* __restrict__ wq,
                                                       uint16_t* __restrict__ sz, int64_t n_units,
                                                       int64_t n_groups, uint32_t* status) {
+  pdl_trigger_and_wait();
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
   const int64_t tid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   const int64_t iters = (n_units > n_groups ? n_units : n_groups);
@@ -124,6 +126,7 @@ __global__ void __launch_bounds__(256) q2_dequant_kernel(const uint8_t* __restri
                                                          const uint16_t* __restrict__ d,
                                                          float* __restrict__ w, int64_t n_words,
                                                          int K) {
+  pdl_trigger_and_wait();
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
   const int64_t words_per_row = K / 16;
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n_words;
@@ -149,6 +152,7 @@ __global__ void __launch_bounds__(256) q4_dequant_kernel(const uint8_t* __restri
                                                          const uint16_t* __restrict__ sz,
                                                          float* __restrict__ w, int64_t n_words,
                                                          int K) {
+  pdl_trigger_and_wait();
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
   const int64_t words_per_row = K / 8;
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n_words;

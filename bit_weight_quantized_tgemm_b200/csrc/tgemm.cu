@@ -87,16 +87,36 @@ cudaEvent_t take_event() {
   return e;
 }
 
-// Run `launch_fn` (one kernel launch on `st`), count it, and time it when profiling.
+// Launch `kernel` on `st` with programmatic stream serialization: it may be scheduled
+// while the previous kernel on the stream is finishing (every kernel of the library
+// waits for its predecessors with griddepcontrol.wait before touching global memory).
+template <typename... KArgs, typename... Args>
+cudaError_t pdl_launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t st, Args... args) {
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
+// Run `launch_fn` (one kernel launch on `st`, returning its cudaError_t), count it, and
+// time it when profiling.
 template <typename Fn>
 int launch(int kind, cudaStream_t st, Fn&& launch_fn) {
   cudaEvent_t b = nullptr, e = nullptr;
-  if (g_profile.load(std::memory_order_relaxed)) {
+  if (g_profile.load(std::memory_order_relaxed) & (1 << kind)) {
     b = take_event();
     e = take_event();
     if (b && e) cudaEventRecord(b, st);
   }
-  launch_fn();
+  const cudaError_t le = launch_fn();
   g_launches.fetch_add(1, std::memory_order_relaxed);
   const int status = launch_status();
   if (b && e) {
@@ -104,7 +124,7 @@ int launch(int kind, cudaStream_t st, Fn&& launch_fn) {
     std::lock_guard<std::mutex> lock(g_prof_mu);
     g_records.push_back({kind, b, e});
   }
-  return status;
+  return le == cudaSuccess ? status : TGEMM_ECUDA;
 }
 
 int grid_for(int64_t work_items, int per_block, int sms) {
@@ -280,13 +300,13 @@ int launch_lora_down(const uint16_t* x, const uint16_t* la, int M, int K, int r,
                      cudaStream_t st, int sms) {
   const dim3 grid((M + 15) / 16, ld.slices, ld.rpad / 64);
   if (int e = launch(TGEMM_KIND_PREP, st, [&] {
-        lora_down_partial_kernel<<<grid, 256, 0, st>>>(x, la, M, K, r, ld.rpad, part);
+        return pdl_launch(lora_down_partial_kernel, grid, 256, 0, st, x, la, M, K, r, ld.rpad, part);
       }))
     return e;
   const int64_t items = ucat ? static_cast<int64_t>(M) * ld.wcat : static_cast<int64_t>(M) * r;
   const int fgrid = grid_for(items, 256, sms);
   return launch(TGEMM_KIND_PREP, st, [&] {
-    lora_finalize_kernel<<<fgrid, 256, 0, st>>>(part, ld.slices, M, r, ld.rpad, ld.R, ld.wcat,
+    return pdl_launch(lora_finalize_kernel, fgrid, 256, 0, st, part, ld.slices, M, r, ld.rpad, ld.R, ld.wcat,
                                                 u32, ucat);
   });
 }
@@ -358,18 +378,18 @@ int run_gemm(int fmt, const uint16_t* x, const uint8_t* wq, const uint16_t* scal
     if (fmt == 0 && lora) {
       if (int e = gemv_prepare<0, true>()) return e;
       return launch(TGEMM_KIND_GEMV_Q2, st, [&] {
-        gemv_kernel<0, true><<<grid, 256, smem, st>>>(x, wq, scales, y, M, N, K, out_f32, u32, lb, r, mrows, kp);
+        return pdl_launch(gemv_kernel<0, true>, grid, 256, smem, st, x, wq, scales, y, M, N, K, out_f32, u32, lb, r, mrows, kp);
       });
     }
     if (fmt == 0) {
       if (int e = gemv_prepare<0, false>()) return e;
       return launch(TGEMM_KIND_GEMV_Q2, st, [&] {
-        gemv_kernel<0, false><<<grid, 256, smem, st>>>(x, wq, scales, y, M, N, K, out_f32, nullptr, nullptr, 0, mrows, kp);
+        return pdl_launch(gemv_kernel<0, false>, grid, 256, smem, st, x, wq, scales, y, M, N, K, out_f32, nullptr, nullptr, 0, mrows, kp);
       });
     }
     if (int e = gemv_prepare<1, false>()) return e;
     return launch(TGEMM_KIND_GEMV_Q4, st, [&] {
-      gemv_kernel<1, false><<<grid, 256, smem, st>>>(x, wq, scales, y, M, N, K, out_f32, nullptr, nullptr, 0, mrows, kp);
+      return pdl_launch(gemv_kernel<1, false>, grid, 256, smem, st, x, wq, scales, y, M, N, K, out_f32, nullptr, nullptr, 0, mrows, kp);
     });
   }
 
@@ -392,13 +412,13 @@ int run_gemm(int fmt, const uint16_t* x, const uint8_t* wq, const uint16_t* scal
     const dim3 grid((M + kPlTok - 1) / kPlTok, ld.slices);
     const int a_vec = aligned(la, 16) ? 1 : 0;
     if (int e = launch(TGEMM_KIND_PREP, st, [&] {
-          prep_lora_kernel<0><<<grid, 256, kPlSmemBytes, st>>>(x, x16, la, M, K, r, ld.rpad, part,
+          return pdl_launch(prep_lora_kernel<0>, grid, 256, kPlSmemBytes, st, x, x16, la, M, K, r, ld.rpad, part,
                                                                cnt, ncnt, a_vec);
         }))
       return e;
     const int fgrid = grid_for(static_cast<int64_t>(M) * ld.wcat, 256, di.sms);
     if (int e = launch(TGEMM_KIND_PREP, st, [&] {
-          lora_finalize_kernel<<<fgrid, 256, 0, st>>>(part, ld.slices, M, r, ld.rpad, ld.R, ld.wcat,
+          return pdl_launch(lora_finalize_kernel, fgrid, 256, 0, st, part, ld.slices, M, r, ld.rpad, ld.R, ld.wcat,
                                                       nullptr, ucat);
         }))
       return e;
@@ -407,9 +427,9 @@ int run_gemm(int fmt, const uint16_t* x, const uint8_t* wq, const uint16_t* scal
     const int pgrid = grid_for(ngroups, 256, di.sms);
     if (int e = launch(TGEMM_KIND_PREP, st, [&] {
           if (fmt == 0)
-            prep_x16_kernel<0><<<pgrid, 256, 0, st>>>(x, x16, ngroups, cnt, ncnt);
+            return pdl_launch(prep_x16_kernel<0>, pgrid, 256, 0, st, x, x16, ngroups, cnt, ncnt);
           else
-            prep_x16_kernel<1><<<pgrid, 256, 0, st>>>(x, x16, ngroups, cnt, ncnt);
+            return pdl_launch(prep_x16_kernel<1>, pgrid, 256, 0, st, x, x16, ngroups, cnt, ncnt);
         }))
       return e;
   }
@@ -449,18 +469,18 @@ int run_gemm(int fmt, const uint16_t* x, const uint8_t* wq, const uint16_t* scal
   if (fmt == 0 && !lora) {
     if (int e = tc_prepare<0, false>()) return e;
     return launch(TGEMM_KIND_TC_Q2, st, [&] {
-      tc_gemm_kernel<0, false><<<grid, kTcThreads, TcFmt<0>::kSmemBytes, st>>>(tm_x, tm_u, p);
+      return pdl_launch(tc_gemm_kernel<0, false>, grid, kTcThreads, TcFmt<0>::kSmemBytes, st, tm_x, tm_u, p);
     });
   }
   if (fmt == 0) {
     if (int e = tc_prepare<0, true>()) return e;
     return launch(TGEMM_KIND_TC_Q2_LORA, st, [&] {
-      tc_gemm_kernel<0, true><<<grid, kTcThreads, TcFmt<0>::kSmemBytes, st>>>(tm_x, tm_u, p);
+      return pdl_launch(tc_gemm_kernel<0, true>, grid, kTcThreads, TcFmt<0>::kSmemBytes, st, tm_x, tm_u, p);
     });
   }
   if (int e = tc_prepare<1, false>()) return e;
   return launch(TGEMM_KIND_TC_Q4, st, [&] {
-    tc_gemm_kernel<1, false><<<grid, kTcThreads, TcFmt<1>::kSmemBytes, st>>>(tm_x, tm_u, p);
+    return pdl_launch(tc_gemm_kernel<1, false>, grid, kTcThreads, TcFmt<1>::kSmemBytes, st, tm_x, tm_u, p);
   });
 }
 
@@ -510,7 +530,7 @@ int q2_pack(const uint8_t* codes, const float* scale, uint8_t* wq, uint16_t* d, 
   const int64_t scales = static_cast<int64_t>(N) * K / 128;
   const cudaStream_t st = as_stream(stream);
   return launch(TGEMM_KIND_PREP, st, [&] {
-    q2_pack_kernel<<<grid_for(units, 256, di.sms), 256, 0, st>>>(codes, scale, wq, d, units, scales, status);
+    return pdl_launch(q2_pack_kernel, grid_for(units, 256, di.sms), 256, 0, st, codes, scale, wq, d, units, scales, status);
   });
 }
 
@@ -527,7 +547,7 @@ int q4_pack(const uint8_t* codes, const float* s, const float* z, uint8_t* wq, u
   const int64_t groups = static_cast<int64_t>(N) * K / 64;
   const cudaStream_t st = as_stream(stream);
   return launch(TGEMM_KIND_PREP, st, [&] {
-    q4_pack_kernel<<<grid_for(units, 256, di.sms), 256, 0, st>>>(codes, s, z, wq, sz, units, groups, status);
+    return pdl_launch(q4_pack_kernel, grid_for(units, 256, di.sms), 256, 0, st, codes, s, z, wq, sz, units, groups, status);
   });
 }
 
@@ -540,7 +560,7 @@ int q2_dequant(const uint8_t* wq, const uint16_t* d, float* w, int N, int K, voi
   const int64_t words = static_cast<int64_t>(N) * K / 16;
   const cudaStream_t st = as_stream(stream);
   return launch(TGEMM_KIND_PREP, st, [&] {
-    q2_dequant_kernel<<<grid_for(words, 256, di.sms), 256, 0, st>>>(wq, d, w, words, K);
+    return pdl_launch(q2_dequant_kernel, grid_for(words, 256, di.sms), 256, 0, st, wq, d, w, words, K);
   });
 }
 
@@ -553,7 +573,7 @@ int q4_dequant(const uint8_t* wq, const uint16_t* sz, float* w, int N, int K, vo
   const int64_t words = static_cast<int64_t>(N) * K / 8;
   const cudaStream_t st = as_stream(stream);
   return launch(TGEMM_KIND_PREP, st, [&] {
-    q4_dequant_kernel<<<grid_for(words, 256, di.sms), 256, 0, st>>>(wq, sz, w, words, K);
+    return pdl_launch(q4_dequant_kernel, grid_for(words, 256, di.sms), 256, 0, st, wq, sz, w, words, K);
   });
 }
 
@@ -639,7 +659,7 @@ int tgemm_device_error(uint32_t* bits, int clear) {
 
 int tgemm_version(void) { return 100; }
 
-int tgemm_profile_enable(int on) { return g_profile.exchange(on ? 1 : 0); }
+int tgemm_profile_enable(int kinds) { return g_profile.exchange(kinds & TGEMM_PROFILE_ALL); }
 
 int tgemm_profile_read(int kind, double* total_ms, int64_t* launches, int reset) {
   if (kind < 0 || kind >= TGEMM_NUM_KINDS || !total_ms || !launches) return TGEMM_EINVAL;

@@ -229,11 +229,14 @@ int tgemm_version(void);
 #define TGEMM_NUM_KINDS        6
 
 /*
- * tgemm_profile_enable -- when `on` is nonzero, every subsequent launch records a pair of
- * CUDA events around itself on the call's stream (host cost: two event records per
- * launch; do not enable while capturing a CUDA graph).  Returns the previous setting.
+ * tgemm_profile_enable -- `kinds` is a bit mask of (1 << TGEMM_KIND_*): every subsequent
+ * launch of a kernel kind whose bit is set records a pair of CUDA events around itself
+ * on the call's stream (host cost: two event records per such launch; do not enable
+ * while capturing a CUDA graph).  TGEMM_PROFILE_ALL enables every kind, 0 disables.
+ * Returns the previous mask.
  */
-int tgemm_profile_enable(int on);
+#define TGEMM_PROFILE_ALL ((1 << TGEMM_NUM_KINDS) - 1)
+int tgemm_profile_enable(int kinds);
 
 /*
  * tgemm_profile_read -- wait for the recorded events of `kind` (TGEMM_KIND_*), store the
