@@ -132,6 +132,15 @@ __device__ __forceinline__ void pdl_trigger_and_wait() {
   asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
+__device__ __forceinline__ uint4 ld_shared_v4(uint32_t saddr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(saddr)
+               : "memory");
+  return v;
+}
+
 // Make this thread's generic-proxy shared-memory writes visible to the async proxy
 // (tensor core reads of operands written with st.shared).
 __device__ __forceinline__ void fence_proxy_async_smem() {

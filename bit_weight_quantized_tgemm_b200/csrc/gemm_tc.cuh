@@ -69,7 +69,8 @@ constexpr int kTcBox = 64;     // k per TMA box (one 128-byte swizzle row of f16
 // TMEM, filled by the TMA producer and the dequant warps and released together.
 constexpr int kTcStages = TGEMM_TC_STAGES;
 constexpr int kTcEpiWarps = 8;
-constexpr int kTcThreads = (2 + 8 + kTcEpiWarps) * 32;
+constexpr int kTcWProdWarp = 2 + 8 + kTcEpiWarps;  // the packed-weight TMA producer
+constexpr int kTcThreads = (kTcWProdWarp + 1) * 32;
 constexpr int kTcXBytes = kTcTok * kTcBK * 2;   // 64 KB: two 32 KB boxes
 constexpr int kTcXBoxBytes = kTcTok * kTcBox * 2;
 constexpr int kTcTmemCols = 512;
@@ -81,9 +82,15 @@ static_assert(kTcACol0 + kTcStages * kTcACols <= kTcTmemCols, "TMEM budget");
 template <int FMT>
 struct TcFmt {
   static constexpr int kWqRowBytes = FMT == 0 ? 32 : 64;  // packed bytes per row per stage
+  // Packed weights reach the dequant warps through their own ring of shared-memory
+  // stages (one TMA box of 128 rows per stage), filled this many stages ahead: deep
+  // enough to hide a DRAM miss, small enough to fit beside the activation stages.
+  static constexpr int kWStages = FMT == 0 ? 8 : 4;
+  static constexpr int kWBytes = kTcRows * kWqRowBytes;
   static constexpr int kXOff = 0;
-  static constexpr int kBarOff = kXOff + kTcStages * kTcXBytes;
-  static constexpr int kNumBars = 2 * kTcStages + 2 + 1;
+  static constexpr int kWOff = kXOff + kTcStages * kTcXBytes;
+  static constexpr int kBarOff = kWOff + kWStages * kWBytes;
+  static constexpr int kNumBars = 2 * kTcStages + 3 + 2 * kWStages;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kSmemBytes = kMiscOff + 16 + 1024;  // + alignment slack
 };
@@ -164,7 +171,8 @@ __device__ __forceinline__ void q4_word_to_f16(uint32_t w, uint32_t s2, uint32_t
 template <int FMT, bool LORA>
 __global__ void __launch_bounds__(kTcThreads, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x,
-                   const __grid_constant__ CUtensorMap tm_u, const TcParams p) {
+                   const __grid_constant__ CUtensorMap tm_u,
+                   const __grid_constant__ CUtensorMap tm_w, const TcParams p) {
   using F = TcFmt<FMT>;
   static_assert(F::kSmemBytes <= 232448, "shared memory budget");
   extern __shared__ uint8_t smem_raw[];
@@ -177,6 +185,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const uint32_t accfull_bar = bar0 + 8u * (2 * kTcStages);
   const uint32_t accempty_bar = bar0 + 8u * (2 * kTcStages + 1);
   const uint32_t drain_bar = bar0 + 8u * (2 * kTcStages + 2);
+  auto wfull_bar = [&](int w) { return bar0 + 8u * (2 * kTcStages + 3 + w); };
+  auto wempty_bar = [&](int w) { return bar0 + 8u * (2 * kTcStages + 3 + F::kWStages + w); };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + F::kMiscOff);
   volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + F::kMiscOff + 4);
 
@@ -190,6 +200,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     mbar_init(accfull_bar, 1);             // MMA commit
     mbar_init(accempty_bar, kTcEpiWarps);  // epilogue warps
     mbar_init(drain_bar, 1);
+    for (int w = 0; w < F::kWStages; ++w) {
+      mbar_init(wfull_bar(w), 1);   // weight producer's expect_tx
+      mbar_init(wempty_bar(w), 8);  // 8 dequant warps have read their codes
+    }
     *abort_flag = 0u;
     fence_mbar_init();
   }
@@ -197,6 +211,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     tma_prefetch_desc(&tm_x);
     if (LORA) tma_prefetch_desc(&tm_u);
   }
+  if (warp == kTcWProdWarp && lane == 0) tma_prefetch_desc(&tm_w);
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_slot), kTcTmemCols);
     tmem_relinquish();
@@ -281,16 +296,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int rt = 32 * q + lane;         // weight row within the tile
     const int half = (warp - 2) >> 2;     // which 64 codes of the stage's 128
     const int nscale = FMT == 0 ? p.K / 128 : p.K / 64;
-    const int64_t wq_row = FMT == 0 ? p.K / 4 : p.K / 2;
     constexpr int kHalfBytes = F::kWqRowBytes / 2;  // 16 (Q2) or 32 (4-bit) bytes per stage
-    constexpr int kPf = FMT == 0 ? 3 : 2;           // items per prefetch register set
     const uint32_t a_lane = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + kTcACol0 +
                             32u * half;
-    uint32_t wit = 0;
+    // this thread's codes inside a weight stage (row rt, half `half`)
+    const uint32_t w_mine = sbase + F::kWOff + rt * F::kWqRowBytes + half * kHalfBytes;
+    uint32_t wit = 0;  // A stages written
+    uint32_t wcnt = 0;  // weight stages consumed
     bool ok = true;
-    // This CTA's work is one stream of (tile, stage) items, item i being unit u0 + i;
-    // prefetching runs across tile boundaries, so a new tile's first stages are already
-    // loaded when the previous tile ends.
+    // This CTA's work is one stream of (tile, stage) items, item i being unit u0 + i.
     const int n_items = u1 > u0 ? u1 - u0 : 0;
     struct Item {
       int ks;
@@ -303,59 +317,57 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const int row = (tile / p.tiles_m) * kTcRows + rt;
       return Item{u - tile * ksteps, row, i < n_items && row < p.N};
     };
-    struct Codes {
-      uint4 a, b;    // Q2 uses a (64 codes); 4-bit uses a and b (64 codes)
-      uint32_t sc;   // Q2 block scale d, or the 4-bit group's (s, z)
-    };
-    // Codes and scale of one item, issued ahead of their use into two register sets used
-    // in turn, so no register that a load is still filling is ever touched early.
-    auto fetch = [&](int i, Codes& c) {
-      c.a = make_uint4(0, 0, 0, 0);
-      c.b = c.a;
-      c.sc = 0u;
+    // The scale of item i: Q2 block scale d, or the 4-bit group's (s, z) pair (0 where the
+    // item has none: a branch stage, a row past N, or a 4-bit half-stage past K).
+    auto scale_of = [&](int i) -> uint32_t {
       const Item it = decode(i);
-      if (!it.valid || it.ks >= p.kt_main) return;
-      const int k_first = it.ks * kTcBK + 64 * half;  // first k of this thread's 64
-      if (k_first >= p.K) return;                     // a 4-bit row ending mid-stage
-      const uint8_t* src = p.wq + static_cast<int64_t>(it.row) * wq_row +
-                           static_cast<int64_t>(it.ks) * F::kWqRowBytes + half * kHalfBytes;
+      if (!it.valid || it.ks >= p.kt_main) return 0u;
+      const int k_first = it.ks * kTcBK + 64 * half;
+      if (k_first >= p.K) return 0u;
       const uint16_t* srow = p.scales + static_cast<int64_t>(it.row) * nscale * (FMT == 0 ? 1 : 2);
-      c.a = __ldg(reinterpret_cast<const uint4*>(src));
-      if (FMT == 0) {
-        c.sc = static_cast<uint32_t>(srow[it.ks]);
-      } else {
-        c.b = __ldg(reinterpret_cast<const uint4*>(src) + 1);
-        c.sc = reinterpret_cast<const uint32_t*>(srow)[k_first / 64];
-      }
+      return FMT == 0 ? static_cast<uint32_t>(__ldg(srow + it.ks))
+                      : __ldg(reinterpret_cast<const uint32_t*>(srow) + k_first / 64);
     };
-    // Dequantize item i into its A stage of TMEM.
-    auto process = [&](int i, const Codes& c) {
-      if (!ok || i >= n_items) return;
+    uint32_t sc_next = scale_of(0);  // loaded one item ahead
+    for (int i = 0; ok && i < n_items; ++i) {
       const Item it = decode(i);
-      const int ks = it.ks;
+      const uint32_t sc = sc_next;
+      sc_next = scale_of(i + 1);
       uint32_t o[32];
-      if (!LORA || ks < p.kt_main) {
+      if (!LORA || it.ks < p.kt_main) {
+        // codes from the weight ring (rows past N and k past K arrive zero-filled)
+        const uint32_t w = wcnt % F::kWStages, wph = (wcnt / F::kWStages) & 1u;
+        if (!mbar_wait_warp(wfull_bar(w), wph, abort_flag)) {
+          ok = false;
+          break;
+        }
+        uint4 ca, cb = make_uint4(0, 0, 0, 0);
+        ca = ld_shared_v4(w_mine + w * F::kWBytes);
+        if (FMT != 0) cb = ld_shared_v4(w_mine + w * F::kWBytes + 16);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(wempty_bar(w));
+        ++wcnt;
         if (FMT == 0) {
-          const uint32_t d2 = c.sc | (c.sc << 16);
-          q2_word_to_f16(c.a.x, d2, o);
-          q2_word_to_f16(c.a.y, d2, o + 8);
-          q2_word_to_f16(c.a.z, d2, o + 16);
-          q2_word_to_f16(c.a.w, d2, o + 24);
+          const uint32_t d2 = sc | (sc << 16);
+          q2_word_to_f16(ca.x, d2, o);
+          q2_word_to_f16(ca.y, d2, o + 8);
+          q2_word_to_f16(ca.z, d2, o + 16);
+          q2_word_to_f16(ca.w, d2, o + 24);
         } else {
-          const uint32_t s2 = (c.sc & 0xFFFFu) | (c.sc << 16);
-          const uint32_t z2 = (c.sc >> 16) | (c.sc & 0xFFFF0000u);
-          q4_word_to_f16(c.a.x, s2, z2, o);
-          q4_word_to_f16(c.a.y, s2, z2, o + 4);
-          q4_word_to_f16(c.a.z, s2, z2, o + 8);
-          q4_word_to_f16(c.a.w, s2, z2, o + 12);
-          q4_word_to_f16(c.b.x, s2, z2, o + 16);
-          q4_word_to_f16(c.b.y, s2, z2, o + 20);
-          q4_word_to_f16(c.b.z, s2, z2, o + 24);
-          q4_word_to_f16(c.b.w, s2, z2, o + 28);
+          const uint32_t s2 = (sc & 0xFFFFu) | (sc << 16);
+          const uint32_t z2 = (sc >> 16) | (sc & 0xFFFF0000u);
+          q4_word_to_f16(ca.x, s2, z2, o);
+          q4_word_to_f16(ca.y, s2, z2, o + 4);
+          q4_word_to_f16(ca.z, s2, z2, o + 8);
+          q4_word_to_f16(ca.w, s2, z2, o + 12);
+          q4_word_to_f16(cb.x, s2, z2, o + 16);
+          q4_word_to_f16(cb.y, s2, z2, o + 20);
+          q4_word_to_f16(cb.z, s2, z2, o + 24);
+          q4_word_to_f16(cb.w, s2, z2, o + 28);
         }
       } else {
         // low-rank stage: weight-side columns [j0, j0 + 64) of [B | B], zero beyond 2R
-        const int j0 = (ks - p.kt_main) * kTcBK + 64 * half;
+        const int j0 = (it.ks - p.kt_main) * kTcBK + 64 * half;
         const bool vec = (p.r & 7) == 0 && (reinterpret_cast<uintptr_t>(p.lb) & 15) == 0;
 #pragma unroll
         for (int cq = 0; cq < 8; ++cq) {
@@ -388,7 +400,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const uint32_t ws = wit % kTcStages, wph = (wit / kTcStages) & 1u;
       if (!mbar_wait_warp(empty_bar(ws), wph ^ 1u, abort_flag)) {
         ok = false;
-        return;
+        break;
       }
       tc_fence_after();
       tmem_st_32x32b_x32(a_lane + ws * kTcACols, o);
@@ -397,21 +409,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(full_bar(ws));
       ++wit;
-    };
-    Codes ca[kPf], cb[kPf];
-#pragma unroll
-    for (int j = 0; j < kPf; ++j) fetch(j, ca[j]);
-    for (int g = 0; ok && g < n_items; g += 2 * kPf) {
-#pragma unroll
-      for (int j = 0; j < kPf; ++j) fetch(g + kPf + j, cb[j]);
-#pragma unroll
-      for (int j = 0; j < kPf; ++j) process(g + j, ca[j]);
-#pragma unroll
-      for (int j = 0; j < kPf; ++j) fetch(g + 2 * kPf + j, ca[j]);
-#pragma unroll
-      for (int j = 0; j < kPf; ++j) process(g + kPf + j, cb[j]);
     }
-  } else {
+  } else if (warp < kTcWProdWarp) {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;                // TMEM lane quarter this warp may access
     const int eh = (warp - 10) >> 2;       // which half of the accumulator's columns
@@ -505,6 +504,26 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(acc[e]);
         put(mbase + cc * 32, v);
       }
+    }
+  } else {
+    // ------------------------------------------------------------ packed-weight producer
+    // One TMA box per main stage: the tile's 128 rows x the stage's packed bytes, into
+    // the weight ring, as far ahead of the dequant warps as the ring allows.
+    if (lane == 0) {
+      uint32_t wit = 0;
+      for (int u = u0; u < u1; ++u) {
+        const int tile = u / ksteps, ks = u - tile * ksteps;
+        if (ks >= p.kt_main) continue;  // branch stages carry no codes
+        const uint32_t w = wit % F::kWStages, ph = (wit / F::kWStages) & 1u;
+        if (!mbar_wait(wempty_bar(w), ph ^ 1u, abort_flag)) break;
+        mbar_arrive_expect_tx(wfull_bar(w), F::kWBytes);
+        tma_load_2d(sbase + F::kWOff + w * F::kWBytes, &tm_w, wfull_bar(w),
+                    ks * F::kWqRowBytes, (tile / p.tiles_m) * kTcRows);
+        ++wit;
+      }
+      // every load issued must land before the CTA may exit
+      for (uint32_t j = (wit > F::kWStages ? wit - F::kWStages : 0); j < wit; ++j)
+        mbar_wait_drain(wfull_bar(j % F::kWStages), (j / F::kWStages) & 1u);
     }
   }
 

@@ -444,6 +444,13 @@ int run_gemm(int fmt, const uint16_t* x, const uint8_t* wq, const uint16_t* scal
   } else {
     tm_u = tm_x;  // unused
   }
+  // packed weights as a [N][row bytes] u8 tensor, boxes of one stage x 128 rows
+  CUtensorMap tm_w;
+  const uint64_t wq_row_bytes = fmt == 0 ? static_cast<uint64_t>(K) / 4 : static_cast<uint64_t>(K) / 2;
+  if (int e = make_map_2d(&tm_w, wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, wq_row_bytes, N,
+                          fmt == 0 ? TcFmt<0>::kWqRowBytes : TcFmt<1>::kWqRowBytes, kTcRows,
+                          CU_TENSOR_MAP_SWIZZLE_NONE))
+    return e;
   TcParams p;
   p.M = M;
   p.N = N;
@@ -469,18 +476,18 @@ int run_gemm(int fmt, const uint16_t* x, const uint8_t* wq, const uint16_t* scal
   if (fmt == 0 && !lora) {
     if (int e = tc_prepare<0, false>()) return e;
     return launch(TGEMM_KIND_TC_Q2, st, [&] {
-      return pdl_launch(tc_gemm_kernel<0, false>, grid, kTcThreads, TcFmt<0>::kSmemBytes, st, tm_x, tm_u, p);
+      return pdl_launch(tc_gemm_kernel<0, false>, grid, kTcThreads, TcFmt<0>::kSmemBytes, st, tm_x, tm_u, tm_w, p);
     });
   }
   if (fmt == 0) {
     if (int e = tc_prepare<0, true>()) return e;
     return launch(TGEMM_KIND_TC_Q2_LORA, st, [&] {
-      return pdl_launch(tc_gemm_kernel<0, true>, grid, kTcThreads, TcFmt<0>::kSmemBytes, st, tm_x, tm_u, p);
+      return pdl_launch(tc_gemm_kernel<0, true>, grid, kTcThreads, TcFmt<0>::kSmemBytes, st, tm_x, tm_u, tm_w, p);
     });
   }
   if (int e = tc_prepare<1, false>()) return e;
   return launch(TGEMM_KIND_TC_Q4, st, [&] {
-    return pdl_launch(tc_gemm_kernel<1, false>, grid, kTcThreads, TcFmt<1>::kSmemBytes, st, tm_x, tm_u, p);
+    return pdl_launch(tc_gemm_kernel<1, false>, grid, kTcThreads, TcFmt<1>::kSmemBytes, st, tm_x, tm_u, tm_w, p);
   });
 }
 
