@@ -69,7 +69,17 @@ constexpr int kTcBox = 64;     // k per TMA box (one 128-byte swizzle row of f16
 // TMEM, filled by the TMA producer and the dequant warps and released together.
 constexpr int kTcStages = TGEMM_TC_STAGES;
 constexpr int kTcEpiWarps = 8;
-constexpr int kTcWProdWarp = 2 + 8 + kTcEpiWarps;  // the packed-weight TMA producer
+#ifndef TGEMM_TC_DEQ_WARPS
+#define TGEMM_TC_DEQ_WARPS 8
+#endif
+// Dequant warps: kTcDeqParts per TMEM lane quarter, each unpacking kTcDeqCodes codes of
+// its row per stage.
+constexpr int kTcDeqWarps = TGEMM_TC_DEQ_WARPS;
+constexpr int kTcDeqParts = kTcDeqWarps / 4;
+constexpr int kTcDeqCodes = 128 / kTcDeqParts;
+static_assert(kTcDeqWarps == 8 || kTcDeqWarps == 16, "2 or 4 dequant warps per lane quarter");
+constexpr int kTcEpiWarp0 = 2 + kTcDeqWarps;                // first epilogue warp
+constexpr int kTcWProdWarp = kTcEpiWarp0 + kTcEpiWarps;     // the packed-weight TMA producer
 constexpr int kTcThreads = (kTcWProdWarp + 1) * 32;
 constexpr int kTcXBytes = kTcTok * kTcBK * 2;   // 64 KB: two 32 KB boxes
 constexpr int kTcXBoxBytes = kTcTok * kTcBox * 2;
@@ -194,7 +204,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kTcStages; ++s) {
-      mbar_init(full_bar(s), 1 + 8);   // producer's expect_tx + 8 dequant warps
+      mbar_init(full_bar(s), 1 + kTcDeqWarps);  // producer's expect_tx + dequant warps
       mbar_init(empty_bar(s), 1);      // MMA commit
     }
     mbar_init(accfull_bar, 1);             // MMA commit
@@ -202,7 +212,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     mbar_init(drain_bar, 1);
     for (int w = 0; w < F::kWStages; ++w) {
       mbar_init(wfull_bar(w), 1);   // weight producer's expect_tx
-      mbar_init(wempty_bar(w), 8);  // 8 dequant warps have read their codes
+      mbar_init(wempty_bar(w), kTcDeqWarps);  // every dequant warp has read its codes
     }
     *abort_flag = 0u;
     fence_mbar_init();
@@ -290,92 +300,96 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       mma_commit(drain_bar);
       mbar_wait_drain(drain_bar, 0u);
     }
-  } else if (warp < 10) {
+  } else if (warp < kTcEpiWarp0) {
     // ------------------------------------------------------------ dequantizers
-    const int q = warp & 3;               // TMEM lane quarter this warp may access
-    const int rt = 32 * q + lane;         // weight row within the tile
-    const int half = (warp - 2) >> 2;     // which 64 codes of the stage's 128
+    constexpr int kC = kTcDeqCodes;                       // codes per thread per stage
+    constexpr int kWords = FMT == 0 ? kC / 16 : kC / 8;   // 32-bit words of packed codes
+    const int q = warp & 3;                // TMEM lane quarter this warp may access
+    const int rt = 32 * q + lane;          // weight row within the tile
+    const int part = (warp - 2) >> 2;      // which kC codes of the stage's 128
     const int nscale = FMT == 0 ? p.K / 128 : p.K / 64;
-    constexpr int kHalfBytes = F::kWqRowBytes / 2;  // 16 (Q2) or 32 (4-bit) bytes per stage
     const uint32_t a_lane = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + kTcACol0 +
-                            32u * half;
-    // this thread's codes inside a weight stage (row rt, half `half`)
-    const uint32_t w_mine = sbase + F::kWOff + rt * F::kWqRowBytes + half * kHalfBytes;
-    uint32_t wit = 0;  // A stages written
+                            static_cast<uint32_t>(part * (kC / 2));
+    // this thread's codes inside a weight stage (row rt, part `part`)
+    const uint32_t w_mine =
+        sbase + F::kWOff + rt * F::kWqRowBytes + part * (F::kWqRowBytes / kTcDeqParts);
+    uint32_t wit = 0;   // A stages written
     uint32_t wcnt = 0;  // weight stages consumed
     bool ok = true;
-    // This CTA's work is one stream of (tile, stage) items, item i being unit u0 + i.
+    // This CTA's work is one stream of (tile, stage) items, item i being unit u0 + i; the
+    // position is advanced item by item (no divisions on the way).
     const int n_items = u1 > u0 ? u1 - u0 : 0;
-    struct Item {
-      int ks;
-      int row;
-      bool valid;
-    };
-    auto decode = [&](int i) -> Item {
-      const int u = u0 + i;
-      const int tile = u / ksteps;
-      const int row = (tile / p.tiles_m) * kTcRows + rt;
-      return Item{u - tile * ksteps, row, i < n_items && row < p.N};
-    };
-    // The scale of item i: Q2 block scale d, or the 4-bit group's (s, z) pair (0 where the
-    // item has none: a branch stage, a row past N, or a 4-bit half-stage past K).
-    auto scale_of = [&](int i) -> uint32_t {
-      const Item it = decode(i);
-      if (!it.valid || it.ks >= p.kt_main) return 0u;
-      const int k_first = it.ks * kTcBK + 64 * half;
+    int tile = u0 / ksteps, ks = u0 - tile * ksteps;
+    int row = (tile / p.tiles_m) * kTcRows + rt;
+    // The scale of the item at (ks, row): Q2 block scale d, or the 4-bit group's (s, z)
+    // pair (0 where the item has none: a branch stage, a row past N, codes past K).
+    auto scale_at = [&](int ks_, int row_, bool in) -> uint32_t {
+      if (!in || row_ >= p.N || ks_ >= p.kt_main) return 0u;
+      const int k_first = ks_ * kTcBK + part * kC;
       if (k_first >= p.K) return 0u;
-      const uint16_t* srow = p.scales + static_cast<int64_t>(it.row) * nscale * (FMT == 0 ? 1 : 2);
-      return FMT == 0 ? static_cast<uint32_t>(__ldg(srow + it.ks))
+      const uint16_t* srow = p.scales + static_cast<int64_t>(row_) * nscale * (FMT == 0 ? 1 : 2);
+      return FMT == 0 ? static_cast<uint32_t>(__ldg(srow + ks_))
                       : __ldg(reinterpret_cast<const uint32_t*>(srow) + k_first / 64);
     };
-    uint32_t sc_next = scale_of(0);  // loaded one item ahead
+    uint32_t sc_next = scale_at(ks, row, n_items > 0);  // loaded one item ahead
     for (int i = 0; ok && i < n_items; ++i) {
-      const Item it = decode(i);
       const uint32_t sc = sc_next;
-      sc_next = scale_of(i + 1);
-      uint32_t o[32];
-      if (!LORA || it.ks < p.kt_main) {
+      const bool valid = row < p.N;
+      int nks = ks + 1, ntile = tile, nrow = row;
+      if (nks == ksteps) {
+        nks = 0;
+        ++ntile;
+        nrow = (ntile / p.tiles_m) * kTcRows + rt;
+      }
+      sc_next = scale_at(nks, nrow, i + 1 < n_items);
+      uint32_t o[kC / 2];
+      if (!LORA || ks < p.kt_main) {
         // codes from the weight ring (rows past N and k past K arrive zero-filled)
         const uint32_t w = wcnt % F::kWStages, wph = (wcnt / F::kWStages) & 1u;
         if (!mbar_wait_warp(wfull_bar(w), wph, abort_flag)) {
           ok = false;
           break;
         }
-        uint4 ca, cb = make_uint4(0, 0, 0, 0);
-        ca = ld_shared_v4(w_mine + w * F::kWBytes);
-        if (FMT != 0) cb = ld_shared_v4(w_mine + w * F::kWBytes + 16);
+        uint32_t cw[kWords];
+        const uint32_t src = w_mine + w * F::kWBytes;
+        if (kWords == 2) {
+          const uint2 v = ld_shared_v2(src);
+          cw[0] = v.x;
+          cw[1] = v.y;
+        } else {
+#pragma unroll
+          for (int j = 0; j < kWords; j += 4) {
+            const uint4 v = ld_shared_v4(src + 4 * j);
+            cw[j] = v.x;
+            cw[j + 1] = v.y;
+            cw[j + 2] = v.z;
+            cw[j + 3] = v.w;
+          }
+        }
         __syncwarp();
         if (lane == 0) mbar_arrive(wempty_bar(w));
         ++wcnt;
         if (FMT == 0) {
           const uint32_t d2 = sc | (sc << 16);
-          q2_word_to_f16(ca.x, d2, o);
-          q2_word_to_f16(ca.y, d2, o + 8);
-          q2_word_to_f16(ca.z, d2, o + 16);
-          q2_word_to_f16(ca.w, d2, o + 24);
+#pragma unroll
+          for (int j = 0; j < kWords; ++j) q2_word_to_f16(cw[j], d2, o + 8 * j);
         } else {
           const uint32_t s2 = (sc & 0xFFFFu) | (sc << 16);
           const uint32_t z2 = (sc >> 16) | (sc & 0xFFFF0000u);
-          q4_word_to_f16(ca.x, s2, z2, o);
-          q4_word_to_f16(ca.y, s2, z2, o + 4);
-          q4_word_to_f16(ca.z, s2, z2, o + 8);
-          q4_word_to_f16(ca.w, s2, z2, o + 12);
-          q4_word_to_f16(cb.x, s2, z2, o + 16);
-          q4_word_to_f16(cb.y, s2, z2, o + 20);
-          q4_word_to_f16(cb.z, s2, z2, o + 24);
-          q4_word_to_f16(cb.w, s2, z2, o + 28);
+#pragma unroll
+          for (int j = 0; j < kWords; ++j) q4_word_to_f16(cw[j], s2, z2, o + 4 * j);
         }
       } else {
-        // low-rank stage: weight-side columns [j0, j0 + 64) of [B | B], zero beyond 2R
-        const int j0 = (it.ks - p.kt_main) * kTcBK + 64 * half;
+        // low-rank stage: weight-side values [j0, j0 + kC) of [B | B], zero beyond 2R
+        const int j0 = (ks - p.kt_main) * kTcBK + part * kC;
         const bool vec = (p.r & 7) == 0 && (reinterpret_cast<uintptr_t>(p.lb) & 15) == 0;
 #pragma unroll
-        for (int cq = 0; cq < 8; ++cq) {
+        for (int cq = 0; cq < kC / 8; ++cq) {
           const int jc = j0 + 8 * cq;
           const int ic = jc < p.R ? jc : jc - p.R;
           if (vec && jc < 2 * p.R && ic + 8 <= p.r) {
             uint4 v = make_uint4(0, 0, 0, 0);
-            if (it.valid) v = *reinterpret_cast<const uint4*>(p.lb + static_cast<int64_t>(it.row) * p.r + ic);
+            if (valid) v = *reinterpret_cast<const uint4*>(p.lb + static_cast<int64_t>(row) * p.r + ic);
             o[4 * cq] = v.x;
             o[4 * cq + 1] = v.y;
             o[4 * cq + 2] = v.z;
@@ -390,20 +404,26 @@ __global__ void __launch_bounds__(kTcThreads, 1)
               const int j = jc + 2 * e + h;
               const int ii = j < p.R ? j : j - p.R;
               uint32_t v = 0;
-              if (it.valid && j < 2 * p.R && ii < p.r) v = p.lb[static_cast<int64_t>(it.row) * p.r + ii];
+              if (valid && j < 2 * p.R && ii < p.r) v = p.lb[static_cast<int64_t>(row) * p.r + ii];
               v2 |= v << (16 * h);
             }
             o[4 * cq + e] = v2;
           }
         }
       }
+      tile = ntile;
+      ks = nks;
+      row = nrow;
       const uint32_t ws = wit % kTcStages, wph = (wit / kTcStages) & 1u;
       if (!mbar_wait_warp(empty_bar(ws), wph ^ 1u, abort_flag)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      tmem_st_32x32b_x32(a_lane + ws * kTcACols, o);
+      if (kC == 64)
+        tmem_st_32x32b_x32(a_lane + ws * kTcACols, *reinterpret_cast<uint32_t(*)[32]>(o));
+      else
+        tmem_st_32x32b_x16(a_lane + ws * kTcACols, *reinterpret_cast<uint32_t(*)[16]>(o));
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
@@ -413,8 +433,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   } else if (warp < kTcWProdWarp) {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;                // TMEM lane quarter this warp may access
-    const int eh = (warp - 10) >> 2;       // which half of the accumulator's columns
-    const int piece = warp - 10;           // this warp's 32 x 128 piece of the tile
+    const int eh = (warp - kTcEpiWarp0) >> 2;  // which half of the accumulator's columns
+    const int piece = warp - kTcEpiWarp0;      // this warp's 32 x 128 piece of the tile
     constexpr int kChunks = kTcTok / 32 / 2;
     constexpr int kPieceFloats = kTcSlotFloats / kTcEpiWarps;
     uint32_t scount = 0;
