@@ -127,9 +127,20 @@ __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a
 // and their memory is visible, and only after that touches global memory.  A dependent
 // grid is scheduled only once every CTA of this one has passed the trigger (so all of
 // them are resident): waiting CTAs never hold resources this grid still needs.
-__device__ __forceinline__ void pdl_trigger_and_wait() {
+__device__ __forceinline__ void pdl_trigger() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger_and_wait() {
+  pdl_trigger();
+  pdl_wait();
+}
+
+// Bring the line holding p into L2.  Allowed before pdl_wait(): it delivers nothing to
+// the SM, and L2 is where any concurrent writer's stores land, so later loads (issued
+// after the wait) still see the final data.
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(reinterpret_cast<uint64_t>(p)));
 }
 
 __device__ __forceinline__ uint2 ld_shared_v2(uint32_t saddr) {

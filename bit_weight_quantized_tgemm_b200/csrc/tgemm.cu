@@ -327,7 +327,7 @@ int gemv_prepare() {
   static cudaError_t err = cudaSuccess;
   std::call_once(once, [] {
     err = cudaFuncSetAttribute(gemv_kernel<FMT, LORA>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               gemv_smem_bytes(16, kGvKP));
+                               kGvXBudget);
   });
   return err == cudaSuccess ? TGEMM_OK : TGEMM_ECUDA;
 }
@@ -373,7 +373,7 @@ int run_gemm(int fmt, const uint16_t* x, const uint8_t* wq, const uint16_t* scal
     }
     const int grid = (N + kGvRows - 1) / kGvRows;
     const int mrows = M < 16 ? M : 16;
-    const int kp = K < kGvKP ? K : kGvKP;
+    const int kp = gemv_pass_k(mrows, K);
     const size_t smem = gemv_smem_bytes(mrows, kp);
     if (fmt == 0 && lora) {
       if (int e = gemv_prepare<0, true>()) return e;
