@@ -159,22 +159,38 @@ __device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity,
   return __all_sync(0xFFFFFFFFu, mbar_wait(bar, parity, abort_flag));
 }
 
+// Unpacking without per-pair shifts.  A field of b bits at mantissa bit position p of an
+// f16 whose other mantissa bits are zero and whose exponent makes the field's lowest bit
+// worth 1 reads as 2^(10-p) + q: so one lop3 (mask the field, or in the exponent) turns a
+// code in place into an exact f16 integer offset by a known constant, as long as the field
+// lies inside the 10-bit mantissa.  Both halves of a 32-bit word are done at once (f16x2).
+//   2-bit fields at bits 0, 2, 4, 6, 8:  exponents of 1024, 256, 64, 16, 4
+//   4-bit fields at bits 0, 4:           exponents of 1024, 64
+// Fields at bits 10 and up are moved down by one shift first.
 // Q2: 16 codes -> 8 f16x2 pairs (codes i, i+8) of (q - 1) * d.
 __device__ __forceinline__ void q2_word_to_f16(uint32_t w, uint32_t d2, uint32_t* o) {
+  // per field position j: the magic (2^(10-2j) as f16x2) and 2^(10-2j) + 1
+  constexpr uint32_t kMagic[5] = {0x64006400u, 0x5C005C00u, 0x54005400u, 0x4C004C00u, 0x44004400u};
+  constexpr uint32_t kBase1[5] = {0x64016401u, 0x5C045C04u, 0x54105410u, 0x4C404C40u, 0x45004500u};
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    const uint32_t t = lop3_and_or(w >> (2 * i), 0x00030003u, 0x64006400u);  // 1024 + q
-    o[i] = hmul2_u32(hsub2_u32(t, 0x64016401u), d2);                           // (q-1)*d
+    const int j = i < 5 ? i : i - 5;
+    const uint32_t src = i < 5 ? w : (w >> 10);
+    const uint32_t t = lop3_and_or(src, 0x00030003u << (2 * j), kMagic[j]);  // base + q
+    o[i] = hmul2_u32(hsub2_u32(t, kBase1[j]), d2);                              // (q-1)*d
   }
 }
 
 // 4-bit: 8 codes -> 4 f16x2 pairs (codes i, i+4) of (q - z) * s.
 __device__ __forceinline__ void q4_word_to_f16(uint32_t w, uint32_t s2, uint32_t z2,
                                                uint32_t* o) {
+  constexpr uint32_t kMagic[2] = {0x64006400u, 0x54005400u};  // 1024, 64
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    const uint32_t t = lop3_and_or(w >> (4 * i), 0x000F000Fu, 0x64006400u);  // 1024 + q
-    o[i] = hmul2_u32(hsub2_u32(hsub2_u32(t, 0x64006400u), z2), s2);           // (q-z)*s
+    const int j = i & 1;
+    const uint32_t src = i < 2 ? w : (w >> 8);
+    const uint32_t t = lop3_and_or(src, 0x000F000Fu << (4 * j), kMagic[j]);  // base + q
+    o[i] = hmul2_u32(hsub2_u32(hsub2_u32(t, kMagic[j]), z2), s2);             // (q-z)*s
   }
 }
 
