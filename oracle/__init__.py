@@ -52,6 +52,8 @@ _SIGS = {
     "oracle_q4_gemm": (None, [_P, _P, _P, _I, _I, _I, _P]),
     "oracle_q2_gemm_at": (None, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P, _I, _P]),
     "oracle_q4_gemm_at": (None, [_P, _P, _P, _I, _I, _I, _P, _P, _I, _P]),
+    "oracle_q2_dual_gemm": (None, [_P, _P, _P, _I, _P, _P, _P, _I, _I, _I, _P]),
+    "oracle_q2_dual_gemm_at": (None, [_P, _P, _P, _I, _P, _P, _P, _I, _I, _I, _P, _P, _I, _P]),
     "oracle_num_threads": (ctypes.c_int, []),
 }
 
@@ -208,6 +210,37 @@ class Oracle:
         out = np.empty(mi.shape, dtype=np.float64)
         self.lib.oracle_q2_gemm_at(px, pw, pd, pa, pb, r, M, N, K, pmi, pni, mi.size,
                                    out.ctypes.data_as(_P))
+        return out
+
+    def q2_dual_gemm(self, x1_bf16, wq1, d1, x2_bf16, wq2, d2, N: int) -> np.ndarray:
+        """y = x1 W1^T + x2 W2^T (a projection split along its input axis), f64."""
+        x1, px1 = self._c(x1_bf16, np.uint16)
+        wq1, pw1 = self._c(wq1, np.uint8)
+        d1, pd1 = self._c(d1, np.uint16)
+        x2, px2 = self._c(x2_bf16, np.uint16)
+        wq2, pw2 = self._c(wq2, np.uint8)
+        d2, pd2 = self._c(d2, np.uint16)
+        M, K1 = x1.shape
+        K2 = x2.shape[1]
+        y = np.empty((M, N), dtype=np.float64)
+        self.lib.oracle_q2_dual_gemm(px1, pw1, pd1, K1, px2, pw2, pd2, K2, M, N,
+                                     y.ctypes.data_as(_P))
+        return y
+
+    def q2_dual_gemm_at(self, x1_bf16, wq1, d1, x2_bf16, wq2, d2, N: int, mi, ni):
+        x1, px1 = self._c(x1_bf16, np.uint16)
+        wq1, pw1 = self._c(wq1, np.uint8)
+        d1, pd1 = self._c(d1, np.uint16)
+        x2, px2 = self._c(x2_bf16, np.uint16)
+        wq2, pw2 = self._c(wq2, np.uint8)
+        d2, pd2 = self._c(d2, np.uint16)
+        mi, pmi = self._c(mi, np.int64)
+        ni, pni = self._c(ni, np.int64)
+        M, K1 = x1.shape
+        K2 = x2.shape[1]
+        out = np.empty(mi.shape, dtype=np.float64)
+        self.lib.oracle_q2_dual_gemm_at(px1, pw1, pd1, K1, px2, pw2, pd2, K2, M, N, pmi, pni,
+                                        mi.size, out.ctypes.data_as(_P))
         return out
 
     def q4_gemm_at(self, x_bf16, wq, sz, N: int, mi, ni):

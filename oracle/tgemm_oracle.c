@@ -342,6 +342,21 @@ void oracle_q4_gemm(const uint16_t* x, const uint8_t* wq, const uint16_t* sz, in
   free(w);
 }
 
+/* y = x1 W1^T + x2 W2^T [P2-GD]: the two products of a projection split along its input
+ * axis, each computed on its own, then summed. */
+void oracle_q2_dual_gemm(const uint16_t* x1, const uint8_t* wq1, const uint16_t* d1, int64_t K1,
+                         const uint16_t* x2, const uint8_t* wq2, const uint16_t* d2, int64_t K2,
+                         int64_t M, int64_t N, double* y) {
+  double* y2 = (double*)malloc((size_t)(M * N) * sizeof(double));
+  if (!y2) return;
+  oracle_q2_gemm(x1, wq1, d1, M, N, K1, y);
+  oracle_q2_gemm(x2, wq2, d2, M, N, K2, y2);
+#ifndef ORACLE_PLANT_DUAL_SECOND_DROPPED
+  for (int64_t i = 0; i < M * N; ++i) y[i] += y2[i];
+#endif
+  free(y2);
+}
+
 /* ------------------------------------------------------------------------------------
  * Sampled outputs: each requested y[m][n] computed on its own from the packed row n
  * (row slicing [P2-GD]: row n is the byte run wq[n*K/4 ...], scales d[n*K/128 ...]).
@@ -379,6 +394,20 @@ void oracle_q2_gemm_at(const uint16_t* x, const uint8_t* wq, const uint16_t* d,
     free(w);
   }
   (void)N;
+}
+
+void oracle_q2_dual_gemm_at(const uint16_t* x1, const uint8_t* wq1, const uint16_t* d1,
+                            int64_t K1, const uint16_t* x2, const uint8_t* wq2,
+                            const uint16_t* d2, int64_t K2, int64_t M, int64_t N,
+                            const int64_t* mi, const int64_t* ni, int64_t count, double* out) {
+  double* o2 = (double*)malloc((size_t)count * sizeof(double));
+  if (!o2) return;
+  oracle_q2_gemm_at(x1, wq1, d1, NULL, NULL, 0, M, N, K1, mi, ni, count, out);
+  oracle_q2_gemm_at(x2, wq2, d2, NULL, NULL, 0, M, N, K2, mi, ni, count, o2);
+#ifndef ORACLE_PLANT_DUAL_SECOND_DROPPED
+  for (int64_t s = 0; s < count; ++s) out[s] += o2[s];
+#endif
+  free(o2);
 }
 
 void oracle_q4_gemm_at(const uint16_t* x, const uint8_t* wq, const uint16_t* sz, int64_t M,

@@ -14,7 +14,10 @@
  *            byte along the input axis, w = (q - 1) * d; the only rounding is the
  *            scale's f32 -> f16 conversion, which must round-trip exactly.
  *   [P2-GD]  same page, "The GPU driver, and the bug that looked like broken math" --
- *            quantized rows are independent byte runs (row slicing).
+ *            quantized rows are independent byte runs (row slicing); a projection
+ *            whose input is two activations concatenated per token is split along its
+ *            input axis into two matmuls that are summed ("Slice weights, not
+ *            activations").
  *   [P2-WL]  same page, "What's left" -- the 4-bit format dequantizes as
  *            (q - zero) * scale.
  *   [P3-FB]  "You Can Now Just Ask for an Image -- and Your Browser Draws It",
@@ -80,6 +83,17 @@ void oracle_q2_lora_gemm(const uint16_t* x, const uint8_t* wq, const uint16_t* d
                          int64_t N, int64_t K, double* y);
 void oracle_q4_gemm(const uint16_t* x, const uint8_t* wq, const uint16_t* sz, int64_t M,
                     int64_t N, int64_t K, double* y);
+
+/* A projection split along its input axis [P2-GD]: y = x1 W1^T + x2 W2^T, with
+ * x1 [M][K1], W1 packed [N][K1/4] + [N][K1/128], x2 [M][K2], W2 packed likewise.  Two
+ * independent f64 products, added element by element. */
+void oracle_q2_dual_gemm(const uint16_t* x1, const uint8_t* wq1, const uint16_t* d1, int64_t K1,
+                         const uint16_t* x2, const uint8_t* wq2, const uint16_t* d2, int64_t K2,
+                         int64_t M, int64_t N, double* y);
+void oracle_q2_dual_gemm_at(const uint16_t* x1, const uint8_t* wq1, const uint16_t* d1,
+                            int64_t K1, const uint16_t* x2, const uint8_t* wq2,
+                            const uint16_t* d2, int64_t K2, int64_t M, int64_t N,
+                            const int64_t* mi, const int64_t* ni, int64_t count, double* out);
 
 /* Sampled outputs, one at a time: out[i] = y[mi[i]][ni[i]].  a/b may be NULL (no branch). */
 void oracle_q2_gemm_at(const uint16_t* x, const uint8_t* wq, const uint16_t* d,

@@ -407,4 +407,44 @@ def pin_sampled_matches_full(o):
                        atol=1e-12)
 
 
+def pin_q2_dual_is_the_split_concatenation(o):
+    """A projection split along its input axis ("Slice weights, not activations"):
+    x1 W1^T + x2 W2^T must equal the single product [x1 | x2] [W1 | W2]^T."""
+    rng = np.random.default_rng(23)
+    for M, N, K1, K2 in [(3, 5, 128, 384), (6, 4, 256, 256), (1, 9, 384, 128)]:
+        x1, x2 = _rand_x(rng, M, K1), _rand_x(rng, M, K2)
+        c1 = rng.integers(0, 3, size=(N, K1), dtype=np.uint8)
+        c2 = rng.integers(0, 3, size=(N, K2), dtype=np.uint8)
+        s1 = np.abs(rng.standard_normal((N, K1 // 128))).astype(np.float16).astype(np.float32)
+        s2 = np.abs(rng.standard_normal((N, K2 // 128))).astype(np.float16).astype(np.float32)
+        wq1, d1, _ = o.q2_pack(c1, s1)
+        wq2, d2, _ = o.q2_pack(c2, s2)
+        wq, d, _ = o.q2_pack(np.concatenate([c1, c2], axis=1), np.concatenate([s1, s2], axis=1))
+        whole = o.q2_gemm(np.concatenate([x1, x2], axis=1), wq, d, N)
+        dual = o.q2_dual_gemm(x1, wq1, d1, x2, wq2, d2, N)
+        assert np.allclose(dual, whole, rtol=1e-12, atol=1e-12), (M, N, K1, K2)
+        assert not np.allclose(dual, o.q2_gemm(x1, wq1, d1, N), rtol=1e-6, atol=1e-6)
+
+
+def pin_q2_dual_closed_forms(o):
+    """Second matrix all codes 1 (zero weights) or second activation zero: only the first
+    product remains, exactly; and the sampled form matches the whole-matrix form."""
+    rng = np.random.default_rng(29)
+    M, N, K1, K2 = 4, 6, 256, 128
+    x1, x2 = _rand_x(rng, M, K1), _rand_x(rng, M, K2)
+    c1 = rng.integers(0, 3, size=(N, K1), dtype=np.uint8)
+    s1 = np.full((N, K1 // 128), 0.5, np.float32)
+    wq1, d1, _ = o.q2_pack(c1, s1)
+    first = o.q2_gemm(x1, wq1, d1, N)
+    wz, dz, _ = o.q2_pack(np.ones((N, K2), np.uint8), np.ones((N, K2 // 128), np.float32))
+    assert np.array_equal(o.q2_dual_gemm(x1, wq1, d1, x2, wz, dz, N), first)
+    c2 = rng.integers(0, 3, size=(N, K2), dtype=np.uint8)
+    wq2, d2, _ = o.q2_pack(c2, np.full((N, K2 // 128), 0.25, np.float32))
+    assert np.array_equal(o.q2_dual_gemm(x1, wq1, d1, np.zeros_like(x2), wq2, d2, N), first)
+    full = o.q2_dual_gemm(x1, wq1, d1, x2, wq2, d2, N)
+    mi, ni = rng.integers(0, M, 15), rng.integers(0, N, 15)
+    assert np.allclose(o.q2_dual_gemm_at(x1, wq1, d1, x2, wq2, d2, N, mi, ni), full[mi, ni],
+                       rtol=1e-12, atol=1e-12)
+
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

@@ -19,6 +19,7 @@ PLANTS = [
     "ORACLE_PLANT_F16_TRUNCATE",      # f32 -> f16 truncates instead of rounding
     "ORACLE_PLANT_GEMM_TRANSPOSED",   # transposed weight operand
     "ORACLE_PLANT_LORA_DROPPED",      # side branch missing
+    "ORACLE_PLANT_DUAL_SECOND_DROPPED",  # split projection: second product missing
 ]
 
 
