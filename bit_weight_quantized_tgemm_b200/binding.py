@@ -37,9 +37,12 @@ _SIGS = {
     "q4_dequant": (_i, [_P, _P, _P, _i, _i, _P]),
     "tgemm_workspace_size": (_sz, [_i, _i, _i, _i, _i]),
     "tgemm_workspace_size_min": (_sz, [_i, _i, _i, _i, _i]),
+    "tgemm_q2_dual_workspace_size": (_sz, [_i, _i, _i, _i]),
+    "tgemm_q2_dual_workspace_size_min": (_sz, [_i, _i, _i, _i]),
     "tgemm_q2": (_i, [_P, _P, _P, _P, _i, _i, _i, _i, _P, _sz, _P]),
     "tgemm_q2_lora": (_i, [_P, _P, _P, _P, _P, _i, _P, _i, _i, _i, _i, _P, _sz, _P]),
     "tgemm_q4": (_i, [_P, _P, _P, _P, _i, _i, _i, _i, _P, _sz, _P]),
+    "tgemm_q2_dual": (_i, [_P, _P, _P, _i, _P, _P, _P, _i, _P, _i, _i, _i, _P, _sz, _P]),
     "tgemm_q2_noalloc": (_i, [_P, _P, _P, _P, _i, _i, _i, _i, _P]),
     "tgemm_strerror": (ctypes.c_char_p, [_i]),
     "tgemm_set_path": (_i, [_i]),
@@ -246,6 +249,35 @@ def gemm_q2_lora(x, wq, d, a, b, *, out_dtype: int = OUT_BF16, y=None, workspace
     ws, nbytes = _workspace(OP_Q2_LORA, M, N, K, r, x.device, workspace)
     _check(lib().tgemm_q2_lora(_ptr(x), _ptr(wq), _ptr(d), _ptr(a), _ptr(b), r, _ptr(y), M, N,
                                K, out_dtype, _ptr(ws), nbytes, _stream()), "tgemm_q2_lora")
+    return y
+
+
+def dual_workspace_size(M: int, N: int, K1: int, K2: int, minimum: bool = False) -> int:
+    """Workspace bytes for gemm_q2_dual (fastest schedule, or the accepted minimum)."""
+    fn = lib().tgemm_q2_dual_workspace_size_min if minimum else lib().tgemm_q2_dual_workspace_size
+    return int(fn(M, N, K1, K2))
+
+
+def gemm_q2_dual(x1, wq1, d1, x2, wq2, d2, *, out_dtype: int = OUT_BF16, y=None, workspace=None):
+    """y = x1 . W1^T + x2 . W2^T: a projection split along its input axis, one kernel."""
+    for t, dt, nm in ((x1, torch.bfloat16, "x1"), (wq1, torch.uint8, "wq1"), (d1, torch.float16, "d1"),
+                      (x2, torch.bfloat16, "x2"), (wq2, torch.uint8, "wq2"), (d2, torch.float16, "d2")):
+        _need(t, dt, nm)
+    M, K1 = x1.shape
+    K2 = x2.shape[1]
+    N = wq1.shape[0]
+    if x2.shape[0] != M or wq2.shape[0] != N:
+        raise ValueError("x1/x2 must have the same tokens and W1/W2 the same rows")
+    y = _out(y, M, N, out_dtype, x1.device)
+    need = dual_workspace_size(M, N, K1, K2)
+    if workspace is None and need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=x1.device)
+    if workspace is not None:
+        _need(workspace, torch.uint8, "workspace")
+    nbytes = workspace.numel() if workspace is not None else 0
+    _check(lib().tgemm_q2_dual(_ptr(x1), _ptr(wq1), _ptr(d1), K1, _ptr(x2), _ptr(wq2), _ptr(d2),
+                               K2, _ptr(y), M, N, out_dtype, _ptr(workspace), nbytes, _stream()),
+           "tgemm_q2_dual")
     return y
 
 

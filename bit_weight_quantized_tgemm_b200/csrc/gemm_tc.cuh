@@ -108,7 +108,9 @@ struct TcFmt {
 struct TcParams {
   int M, N, K;
   int tiles_m, num_tiles;
-  int kt_main;     // ceil(K / 128)
+  int kt_main;     // main stages: ceil(K / 128), or kt1 + ceil(K2 / 128) for two inputs
+  int kt1;         // stages of the first input; stages [kt1, kt_main) read the second
+  int K2;          // the second input's width (0: one input)
   int kt_lora;     // extra stages for the low-rank branch (0 without it)
   int ksteps;      // kt_main + kt_lora: units of work per tile
   int upc;         // units per CTA: CTA c owns units [c * upc, min(U, (c + 1) * upc))
@@ -119,6 +121,7 @@ struct TcParams {
   int out_f32;
   const uint8_t* wq;       // packed codes [N][K/4] (Q2) or [N][K/2] (4-bit)
   const uint16_t* scales;  // Q2: d [N][K/128]; 4-bit: sz [N][K/64][2]
+  const uint16_t* scales2; // the second input's scales (two inputs only)
   const uint16_t* lb;      // low-rank B [N][r] (bf16)
   void* y;
   float* part;             // split tiles: 2 slots of 128 x 256 f32 per CTA
@@ -198,7 +201,9 @@ template <int FMT, bool LORA>
 __global__ void __launch_bounds__(kTcThreads, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x,
                    const __grid_constant__ CUtensorMap tm_u,
-                   const __grid_constant__ CUtensorMap tm_w, const TcParams p) {
+                   const __grid_constant__ CUtensorMap tm_w,
+                   const __grid_constant__ CUtensorMap tm_x2,
+                   const __grid_constant__ CUtensorMap tm_w2, const TcParams p) {
   using F = TcFmt<FMT>;
   static_assert(F::kSmemBytes <= 232448, "shared memory budget");
   extern __shared__ uint8_t smem_raw[];
@@ -236,8 +241,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tm_x);
     if (LORA) tma_prefetch_desc(&tm_u);
+    if (p.kt1 < p.kt_main) tma_prefetch_desc(&tm_x2);
   }
-  if (warp == kTcWProdWarp && lane == 0) tma_prefetch_desc(&tm_w);
+  if (warp == kTcWProdWarp && lane == 0) {
+    tma_prefetch_desc(&tm_w);
+    if (p.kt1 < p.kt_main) tma_prefetch_desc(&tm_w2);
+  }
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_slot), kTcTmemCols);
     tmem_relinquish();
@@ -262,8 +271,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         if (!mbar_wait(empty_bar(s), ph ^ 1u, abort_flag)) break;
         const uint32_t xdst = sbase + F::kXOff + s * kTcXBytes;
         mbar_arrive_expect_tx(full_bar(s), kTcXBytes);
-        const CUtensorMap* map = ks < p.kt_main ? &tm_x : &tm_u;
-        const int k0 = (ks < p.kt_main ? ks : ks - p.kt_main) * kTcBK;
+        // stage ks: first input, second input, or the branch's u
+        const CUtensorMap* map = ks < p.kt1 ? &tm_x : (ks < p.kt_main ? &tm_x2 : &tm_u);
+        const int k0 = (ks < p.kt1 ? ks : (ks < p.kt_main ? ks - p.kt1 : ks - p.kt_main)) * kTcBK;
         tma_load_2d(xdst, map, full_bar(s), k0, tm * kTcTok);
         tma_load_2d(xdst + kTcXBoxBytes, map, full_bar(s), k0 + kTcBox, tm * kTcTok);
       }
@@ -324,6 +334,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int rt = 32 * q + lane;          // weight row within the tile
     const int part = (warp - 2) >> 2;      // which kC codes of the stage's 128
     const int nscale = FMT == 0 ? p.K / 128 : p.K / 64;
+    const int nscale2 = FMT == 0 ? p.K2 / 128 : p.K2 / 64;
     const uint32_t a_lane = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + kTcACol0 +
                             static_cast<uint32_t>(part * (kC / 2));
     // this thread's codes inside a weight stage (row rt, part `part`)
@@ -341,9 +352,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     // pair (0 where the item has none: a branch stage, a row past N, codes past K).
     auto scale_at = [&](int ks_, int row_, bool in) -> uint32_t {
       if (!in || row_ >= p.N || ks_ >= p.kt_main) return 0u;
+      const bool second = ks_ >= p.kt1;  // the second input's stages
+      if (second) ks_ -= p.kt1;
       const int k_first = ks_ * kTcBK + part * kC;
-      if (k_first >= p.K) return 0u;
-      const uint16_t* srow = p.scales + static_cast<int64_t>(row_) * nscale * (FMT == 0 ? 1 : 2);
+      if (k_first >= (second ? p.K2 : p.K)) return 0u;
+      const uint16_t* srow = (second ? p.scales2 : p.scales) +
+                             static_cast<int64_t>(row_) * (second ? nscale2 : nscale) * (FMT == 0 ? 1 : 2);
       return FMT == 0 ? static_cast<uint32_t>(__ldg(srow + ks_))
                       : __ldg(reinterpret_cast<const uint32_t*>(srow) + k_first / 64);
     };
@@ -553,8 +567,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const uint32_t w = wit % F::kWStages, ph = (wit / F::kWStages) & 1u;
         if (!mbar_wait(wempty_bar(w), ph ^ 1u, abort_flag)) break;
         mbar_arrive_expect_tx(wfull_bar(w), F::kWBytes);
-        tma_load_2d(sbase + F::kWOff + w * F::kWBytes, &tm_w, wfull_bar(w),
-                    ks * F::kWqRowBytes, (tile / p.tiles_m) * kTcRows);
+        const bool second = ks >= p.kt1;
+        tma_load_2d(sbase + F::kWOff + w * F::kWBytes, second ? &tm_w2 : &tm_w, wfull_bar(w),
+                    (second ? ks - p.kt1 : ks) * F::kWqRowBytes, (tile / p.tiles_m) * kTcRows);
         ++wit;
       }
       // every load issued must land before the CTA may exit

@@ -103,11 +103,14 @@ __device__ __forceinline__ void x_fragment_order(const uint32_t (&v)[8], uint32_
   }
 }
 
-template <int FMT, bool LORA>
+// DUAL: a second input (x2, wq2, scales2, K2) whose product adds into the same sums.
+template <int FMT, bool LORA, bool DUAL>
 __global__ void __launch_bounds__(256) gemv_kernel(
     const uint16_t* __restrict__ x, const uint8_t* __restrict__ wq,
     const uint16_t* __restrict__ scales, void* __restrict__ y, int M, int N, int K, int out_f32,
-    const float* __restrict__ u, const uint16_t* __restrict__ lb, int r, int mrows, int kp) {
+    const float* __restrict__ u, const uint16_t* __restrict__ lb, int r, int mrows, int kp,
+    const uint16_t* __restrict__ x2, const uint8_t* __restrict__ wq2,
+    const uint16_t* __restrict__ scales2, int K2) {
   extern __shared__ __align__(16) uint8_t gv_smem[];
   // the warps' partial sums, over the staged activations once all passes are done
   auto red = reinterpret_cast<float(*)[16][kGvRows + 1]>(gv_smem);
@@ -134,11 +137,8 @@ __global__ void __launch_bounds__(256) gemv_kernel(
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, c = lane & 3;
   const int n0 = blockIdx.x * kGvRows;
-  const int nunits = (K + kGvUnit - 1) / kGvUnit;
   constexpr int kUnitBytes = FMT == 0 ? 32 : 64;  // packed bytes of one row per unit
   constexpr int kQW = FMT == 0 ? 2 : 4;           // 32-bit words a lane loads per row-unit
-  const int64_t row_bytes = FMT == 0 ? K / 4 : K / 2;
-  const int nscale = FMT == 0 ? K / 128 : K / 64;  // scale entries per row
 
   // ldmatrix.x4 row address of this lane: matrices (tokens 0-7 | 8-15) x (k 0-7 | 8-15)
   const int mi = lane >> 3, arow = (mi & 1) * 8 + (lane & 7);
@@ -155,147 +155,158 @@ __global__ void __launch_bounds__(256) gemv_kernel(
 #pragma unroll
       for (int e = 0; e < 4; ++e) acc[j][e] = 0.f;
 
-    for (int k0 = 0; k0 < K; k0 += kp) {
-      const int kpass = min(kp, K - k0);
-      const int u_base = k0 / kGvUnit;
-      const int u_end = min(nunits, (k0 + kpass + kGvUnit - 1) / kGvUnit);
-      // ---- every packed-weight load of this pass (lane (g, c): quarter c of row g)
-      uint32_t wreg[kGvMaxU][2][kQW];
+    // one input, or two (a projection split along its input axis: their products add
+    // into the same partial sums)
+    for (int part = 0; part < (DUAL ? 2 : 1); ++part) {
+      const uint16_t* xq = part ? x2 : x;
+      const uint8_t* wqq = part ? wq2 : wq;
+      const uint16_t* sq = part ? scales2 : scales;
+      const int Kq = part ? K2 : K;
+      const int nunitsq = (Kq + kGvUnit - 1) / kGvUnit;
+      const int64_t row_bytesq = FMT == 0 ? Kq / 4 : Kq / 2;
+      const int nscaleq = FMT == 0 ? Kq / 128 : Kq / 64;
+      for (int k0 = 0; k0 < Kq; k0 += kp) {
+        const int kpass = min(kp, Kq - k0);
+        const int u_base = k0 / kGvUnit;
+        const int u_end = min(nunitsq, (k0 + kpass + kGvUnit - 1) / kGvUnit);
+        // ---- every packed-weight load of this pass (lane (g, c): quarter c of row g)
+        uint32_t wreg[kGvMaxU][2][kQW];
 #pragma unroll
-      for (int i = 0; i < kGvMaxU; ++i) {
-        const int unit = u_base + i * kGvWarps + warp;
-#pragma unroll
-        for (int j = 0; j < 2; ++j) {
-          const int row = n0 + 8 * j + g;
-          const bool ok = unit < u_end && row < N;
-          const uint8_t* base = wq + static_cast<int64_t>(row) * row_bytes +
-                                static_cast<int64_t>(unit) * kUnitBytes;
-          if (FMT == 0) {
-            uint2 v = make_uint2(0x55555555u, 0x55555555u);  // code 1 everywhere = weight 0
-            if (ok) v = __ldg(reinterpret_cast<const uint2*>(base + 8 * c));
-            wreg[i][j][0] = v.x;
-            wreg[i][j][1] = v.y;
-          } else {
-            // a unit's second 32 bytes exist only where K reaches its second group
-            uint4 v = make_uint4(0u, 0u, 0u, 0u);
-            if (ok && (c < 2 || static_cast<int64_t>(unit) * kGvUnit + 64 < K))
-              v = __ldg(reinterpret_cast<const uint4*>(base + 16 * c));
-            wreg[i][j][0] = v.x;
-            wreg[i][j][1] = v.y;
-            wreg[i][j][2] = v.z;
-            wreg[i][j][3] = v.w;
-          }
-        }
-      }
-      // ---- this pass's scales for the CTA's rows
-      {
-        const int s_base = FMT == 0 ? u_base : 2 * u_base;
-        const int s_cnt = FMT == 0 ? (u_end - u_base) : min(nscale - s_base, 2 * (u_end - u_base));
-        for (int it = tid; it < kGvRows * s_cnt; it += blockDim.x) {
-          const int rl = it / s_cnt, si = it - rl * s_cnt;
-          const int n = n0 + rl;
-          uint32_t v = 0;
-          if (n < N) {
-            const int64_t idx = static_cast<int64_t>(n) * nscale + s_base + si;
-            v = FMT == 0 ? static_cast<uint32_t>(scales[idx])
-                         : reinterpret_cast<const uint32_t*>(scales)[idx];
-          }
-          scl[rl][si] = v;
-        }
-      }
-      // ---- the pass's activations, in fragment order
-      {
-        const int ng = kpass / 16;  // 16-element groups per token row
-        for (int gi = tid; gi < mt * ng; gi += blockDim.x) {
-          const int row = gi / ng, grp = gi - row * ng;
-          const uint4* src = reinterpret_cast<const uint4*>(
-              x + static_cast<int64_t>(m0 + row) * K + k0 + 16 * grp);
-          const uint4 a = __ldg(src), b = __ldg(src + 1);
-          const uint32_t v[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-          uint32_t o[8];
-          x_fragment_order<FMT>(v, o);
-          const uint32_t dst = xs + row * rs + 32 * grp;
-          st_shared_v4(dst, o[0], o[1], o[2], o[3]);
-          st_shared_v4(dst + 16, o[4], o[5], o[6], o[7]);
-        }
-      }
-      __syncthreads();
-      // ---- the warp's units: A fragments by ldmatrix, B fragments from the codes
-#pragma unroll
-      for (int i = 0; i < kGvMaxU; ++i) {
-        const int unit = u_base + i * kGvWarps + warp;
-        if (unit >= u_end) break;
-        const int ku = (unit - u_base) * kGvUnit;  // unit offset within the pass
-        if (FMT == 0) {
-          float part[2][4];
-#pragma unroll
-          for (int j = 0; j < 2; ++j)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) part[j][e] = 0.f;
-#pragma unroll
-          for (int s = 0; s < 8; ++s) {  // k16 step s: word s of the row-unit
-            uint32_t af[4];
-            ldmatrix_x4(a_row + 2 * (ku + 16 * s), af);
-            const int src = (lane & ~3) | (s >> 1);  // the quad lane that loaded word s
-#pragma unroll
-            for (int j = 0; j < 2; ++j) {
-              const uint32_t w = __shfl_sync(0xFFFFFFFFu, wreg[i][j][s & 1], src);
-              mma_bf16_16816(part[j], af, q2_pair_bf16(w, 2 * c), q2_pair_bf16(w, 2 * c + 8));
-            }
-          }
-          // part[j][e]: token g (+8 for e >= 2), weight row 8j + 2c + (e & 1)
+        for (int i = 0; i < kGvMaxU; ++i) {
+          const int unit = u_base + i * kGvWarps + warp;
 #pragma unroll
           for (int j = 0; j < 2; ++j) {
-            const int rl = 8 * j + 2 * c, ui = unit - u_base;
-            const float d0 = __half2float(__ushort_as_half(static_cast<uint16_t>(scl[rl][ui])));
-            const float d1 = __half2float(__ushort_as_half(static_cast<uint16_t>(scl[rl + 1][ui])));
-            acc[j][0] = fmaf(d0, part[j][0], acc[j][0]);
-            acc[j][1] = fmaf(d1, part[j][1], acc[j][1]);
-            acc[j][2] = fmaf(d0, part[j][2], acc[j][2]);
-            acc[j][3] = fmaf(d1, part[j][3], acc[j][3]);
+            const int row = n0 + 8 * j + g;
+            const bool ok = unit < u_end && row < N;
+            const uint8_t* base = wqq + static_cast<int64_t>(row) * row_bytesq +
+                                  static_cast<int64_t>(unit) * kUnitBytes;
+            if (FMT == 0) {
+              uint2 v = make_uint2(0x55555555u, 0x55555555u);  // code 1 everywhere = weight 0
+              if (ok) v = __ldg(reinterpret_cast<const uint2*>(base + 8 * c));
+              wreg[i][j][0] = v.x;
+              wreg[i][j][1] = v.y;
+            } else {
+              // a unit's second 32 bytes exist only where K reaches its second group
+              uint4 v = make_uint4(0u, 0u, 0u, 0u);
+              if (ok && (c < 2 || static_cast<int64_t>(unit) * kGvUnit + 64 < Kq))
+                v = __ldg(reinterpret_cast<const uint4*>(base + 16 * c));
+              wreg[i][j][0] = v.x;
+              wreg[i][j][1] = v.y;
+              wreg[i][j][2] = v.z;
+              wreg[i][j][3] = v.w;
+            }
           }
-        } else {
+        }
+        // ---- this pass's sq for the CTA's rows
+        {
+          const int s_base = FMT == 0 ? u_base : 2 * u_base;
+          const int s_cnt = FMT == 0 ? (u_end - u_base) : min(nscaleq - s_base, 2 * (u_end - u_base));
+          for (int it = tid; it < kGvRows * s_cnt; it += blockDim.x) {
+            const int rl = it / s_cnt, si = it - rl * s_cnt;
+            const int n = n0 + rl;
+            uint32_t v = 0;
+            if (n < N) {
+              const int64_t idx = static_cast<int64_t>(n) * nscaleq + s_base + si;
+              v = FMT == 0 ? static_cast<uint32_t>(sq[idx])
+                           : reinterpret_cast<const uint32_t*>(sq)[idx];
+            }
+            scl[rl][si] = v;
+          }
+        }
+        // ---- the pass's activations, in fragment order
+        {
+          const int ng = kpass / 16;  // 16-element groups per token row
+          for (int gi = tid; gi < mt * ng; gi += blockDim.x) {
+            const int row = gi / ng, grp = gi - row * ng;
+            const uint4* src = reinterpret_cast<const uint4*>(
+                xq + static_cast<int64_t>(m0 + row) * Kq + k0 + 16 * grp);
+            const uint4 a = __ldg(src), b = __ldg(src + 1);
+            const uint32_t v[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+            uint32_t o[8];
+            x_fragment_order<FMT>(v, o);
+            const uint32_t dst = xs + row * rs + 32 * grp;
+            st_shared_v4(dst, o[0], o[1], o[2], o[3]);
+            st_shared_v4(dst + 16, o[4], o[5], o[6], o[7]);
+          }
+        }
+        __syncthreads();
+        // ---- the warp's units: A fragments by ldmatrix, B fragments from the codes
 #pragma unroll
-          for (int h2 = 0; h2 < 2; ++h2) {
-            const int grp = 2 * unit + h2;
-            if (grp * 64 >= K) break;
-            float part[2][4], ssum[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int i = 0; i < kGvMaxU; ++i) {
+          const int unit = u_base + i * kGvWarps + warp;
+          if (unit >= u_end) break;
+          const int ku = (unit - u_base) * kGvUnit;  // unit offset within the pass
+          if (FMT == 0) {
+            float part[2][4];
 #pragma unroll
             for (int j = 0; j < 2; ++j)
 #pragma unroll
               for (int e = 0; e < 4; ++e) part[j][e] = 0.f;
 #pragma unroll
-            for (int sq = 0; sq < 4; ++sq) {  // k16 step s: words 2s, 2s+1 of the row-unit
-              const int s = 4 * h2 + sq;
+            for (int s = 0; s < 8; ++s) {  // k16 step s: word s of the row-unit
               uint32_t af[4];
               ldmatrix_x4(a_row + 2 * (ku + 16 * s), af);
-              mma_bf16_16816(ssum, af, 0x3F803F80u, 0x3F803F80u);  // x against ones
-              const int src = (lane & ~3) | (s >> 1);
+              const int src = (lane & ~3) | (s >> 1);  // the quad lane that loaded word s
 #pragma unroll
               for (int j = 0; j < 2; ++j) {
-                const uint32_t w0 = __shfl_sync(0xFFFFFFFFu, wreg[i][j][2 * (s & 1)], src);
-                const uint32_t w1 = __shfl_sync(0xFFFFFFFFu, wreg[i][j][2 * (s & 1) + 1], src);
-                mma_bf16_16816(part[j], af, q4_pair_bf16(w0, 4 * c), q4_pair_bf16(w1, 4 * c));
+                const uint32_t w = __shfl_sync(0xFFFFFFFFu, wreg[i][j][s & 1], src);
+                mma_bf16_16816(part[j], af, q2_pair_bf16(w, 2 * c), q2_pair_bf16(w, 2 * c + 8));
               }
             }
-            // ssum[0] = S for token g, ssum[2] = S for token g + 8
+            // part[j][e]: token g (+8 for e >= 2), weight row 8j + 2c + (e & 1)
 #pragma unroll
             for (int j = 0; j < 2; ++j) {
-              const int rl = 8 * j + 2 * c, gi = grp - 2 * u_base;
-              const uint32_t v0 = scl[rl][gi], v1 = scl[rl + 1][gi];
-              const float s0 = __half2float(__ushort_as_half(static_cast<uint16_t>(v0 & 0xFFFFu)));
-              const float z0 = __half2float(__ushort_as_half(static_cast<uint16_t>(v0 >> 16)));
-              const float s1 = __half2float(__ushort_as_half(static_cast<uint16_t>(v1 & 0xFFFFu)));
-              const float z1 = __half2float(__ushort_as_half(static_cast<uint16_t>(v1 >> 16)));
-              acc[j][0] = fmaf(s0, fmaf(-z0, ssum[0], part[j][0]), acc[j][0]);
-              acc[j][1] = fmaf(s1, fmaf(-z1, ssum[0], part[j][1]), acc[j][1]);
-              acc[j][2] = fmaf(s0, fmaf(-z0, ssum[2], part[j][2]), acc[j][2]);
-              acc[j][3] = fmaf(s1, fmaf(-z1, ssum[2], part[j][3]), acc[j][3]);
+              const int rl = 8 * j + 2 * c, ui = unit - u_base;
+              const float d0 = __half2float(__ushort_as_half(static_cast<uint16_t>(scl[rl][ui])));
+              const float d1 = __half2float(__ushort_as_half(static_cast<uint16_t>(scl[rl + 1][ui])));
+              acc[j][0] = fmaf(d0, part[j][0], acc[j][0]);
+              acc[j][1] = fmaf(d1, part[j][1], acc[j][1]);
+              acc[j][2] = fmaf(d0, part[j][2], acc[j][2]);
+              acc[j][3] = fmaf(d1, part[j][3], acc[j][3]);
+            }
+          } else {
+#pragma unroll
+            for (int h2 = 0; h2 < 2; ++h2) {
+              const int grp = 2 * unit + h2;
+              if (grp * 64 >= Kq) break;
+              float part[2][4], ssum[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+              for (int j = 0; j < 2; ++j)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) part[j][e] = 0.f;
+#pragma unroll
+              for (int sq = 0; sq < 4; ++sq) {  // k16 step s: words 2s, 2s+1 of the row-unit
+                const int s = 4 * h2 + sq;
+                uint32_t af[4];
+                ldmatrix_x4(a_row + 2 * (ku + 16 * s), af);
+                mma_bf16_16816(ssum, af, 0x3F803F80u, 0x3F803F80u);  // xq against ones
+                const int src = (lane & ~3) | (s >> 1);
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                  const uint32_t w0 = __shfl_sync(0xFFFFFFFFu, wreg[i][j][2 * (s & 1)], src);
+                  const uint32_t w1 = __shfl_sync(0xFFFFFFFFu, wreg[i][j][2 * (s & 1) + 1], src);
+                  mma_bf16_16816(part[j], af, q4_pair_bf16(w0, 4 * c), q4_pair_bf16(w1, 4 * c));
+                }
+              }
+              // ssum[0] = S for token g, ssum[2] = S for token g + 8
+#pragma unroll
+              for (int j = 0; j < 2; ++j) {
+                const int rl = 8 * j + 2 * c, gi = grp - 2 * u_base;
+                const uint32_t v0 = scl[rl][gi], v1 = scl[rl + 1][gi];
+                const float s0 = __half2float(__ushort_as_half(static_cast<uint16_t>(v0 & 0xFFFFu)));
+                const float z0 = __half2float(__ushort_as_half(static_cast<uint16_t>(v0 >> 16)));
+                const float s1 = __half2float(__ushort_as_half(static_cast<uint16_t>(v1 & 0xFFFFu)));
+                const float z1 = __half2float(__ushort_as_half(static_cast<uint16_t>(v1 >> 16)));
+                acc[j][0] = fmaf(s0, fmaf(-z0, ssum[0], part[j][0]), acc[j][0]);
+                acc[j][1] = fmaf(s1, fmaf(-z1, ssum[0], part[j][1]), acc[j][1]);
+                acc[j][2] = fmaf(s0, fmaf(-z0, ssum[2], part[j][2]), acc[j][2]);
+                acc[j][3] = fmaf(s1, fmaf(-z1, ssum[2], part[j][3]), acc[j][3]);
+              }
             }
           }
         }
+        __syncthreads();  // everyone is done with this pass's activations and sq
       }
-      __syncthreads();  // everyone is done with this pass's activations and scales
     }
 
     // ---- reduce the warps' partial sums and write y ---------------------------------

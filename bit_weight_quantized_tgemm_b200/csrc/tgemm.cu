@@ -254,13 +254,14 @@ struct Workspace {
   size_t total_whole = 0;           // the same without the split-tile part
 };
 
-Workspace workspace_layout(int op, int M, int N, int K, int r, int path, int sms) {
+// K2 > 0: a second input of width K2 (a projection split along its input axis).
+Workspace workspace_layout(int op, int M, int N, int K, int r, int path, int sms, int K2 = 0) {
   Workspace w;
   size_t off = 0;
   const bool lora = op == TGEMM_OP_Q2_LORA;
   if (path == TGEMM_PATH_TENSOR) {
     w.x16 = off;
-    w.x16_bytes = static_cast<size_t>(M) * K * 2;
+    w.x16_bytes = static_cast<size_t>(M) * (K + K2) * 2;
     off = round_up(off + w.x16_bytes, 256);
     if (lora) {
       w.ucat = off;
@@ -280,7 +281,7 @@ Workspace workspace_layout(int op, int M, int N, int K, int r, int path, int sms
   }
   w.total_whole = off;
   if (path == TGEMM_PATH_TENSOR) {
-    const TcSchedule sc = tc_schedule(M, N, K, lora ? lora_dims(r, K).L : 0, sms);
+    const TcSchedule sc = tc_schedule(M, N, K + K2, lora ? lora_dims(r, K).L : 0, sms);
     if (sc.split) {
       w.slots = off;
       w.slots_bytes = static_cast<size_t>(2) * sc.grid * kTcSlotFloats * 4;
@@ -321,12 +322,12 @@ int prep_lora_prepare() {
   return err == cudaSuccess ? TGEMM_OK : TGEMM_ECUDA;
 }
 
-template <int FMT, bool LORA>
+template <int FMT, bool LORA, bool DUAL = false>
 int gemv_prepare() {
   static std::once_flag once;
   static cudaError_t err = cudaSuccess;
   std::call_once(once, [] {
-    err = cudaFuncSetAttribute(gemv_kernel<FMT, LORA>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    err = cudaFuncSetAttribute(gemv_kernel<FMT, LORA, DUAL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                kGvXBudget);
   });
   return err == cudaSuccess ? TGEMM_OK : TGEMM_ECUDA;
@@ -334,10 +335,21 @@ int gemv_prepare() {
 
 // ---- the matmul driver ---------------------------------------------------------------
 
+// The optional second input of a projection split along its input axis (Q2 only).
+struct SecondInput {
+  const uint16_t* x = nullptr;
+  const uint8_t* wq = nullptr;
+  const uint16_t* d = nullptr;
+  int K = 0;
+};
+
 int run_gemm(int fmt, const uint16_t* x, const uint8_t* wq, const uint16_t* scales,
              const uint16_t* la, const uint16_t* lb, int r, void* y, int M, int N, int K,
-             int out_dtype, void* workspace, size_t ws_bytes, void* stream) {
+             int out_dtype, void* workspace, size_t ws_bytes, void* stream,
+             const SecondInput& in2 = SecondInput()) {
   const bool lora = la != nullptr;
+  const bool dual = in2.K > 0;
+  const int K2 = in2.K;
   const int op = fmt == 1 ? TGEMM_OP_Q4 : (lora ? TGEMM_OP_Q2_LORA : TGEMM_OP_Q2);
   const int kblock = fmt == 0 ? 128 : 64;
   if (!x || !wq || !scales || !y) return TGEMM_EINVAL;
@@ -347,16 +359,20 @@ int run_gemm(int fmt, const uint16_t* x, const uint8_t* wq, const uint16_t* scal
   if (!aligned(x, 16) || !aligned(wq, 16) || !aligned(y, 16)) return TGEMM_EALIGN;
   if (!aligned(scales, fmt == 0 ? 2 : 4)) return TGEMM_EALIGN;
   if (lora && (!aligned(la, 4) || !aligned(lb, 2))) return TGEMM_EALIGN;
+  if (dual) {
+    if (fmt != 0 || lora || !in2.x || !in2.wq || !in2.d || K2 < 128 || K2 % 128) return TGEMM_EINVAL;
+    if (!aligned(in2.x, 16) || !aligned(in2.wq, 16) || !aligned(in2.d, 2)) return TGEMM_EALIGN;
+  }
   const int path = choose_path(M);
   // the required size does not depend on the device (only the optional split-tile part does)
-  const size_t required = workspace_layout(op, M, N, K, r, path, kDefaultSms).total_whole;
+  const size_t required = workspace_layout(op, M, N, K, r, path, kDefaultSms, K2).total_whole;
   if (required > 0) {
     if (!workspace || ws_bytes < required) return TGEMM_EWORKSPACE;
     if (!aligned(workspace, 256)) return TGEMM_EALIGN;
   }
   DeviceInfo di;
   if (int st = current_device_info(&di)) return st;
-  const Workspace wl = workspace_layout(op, M, N, K, r, path, di.sms);
+  const Workspace wl = workspace_layout(op, M, N, K, r, path, di.sms, K2);
   // split tiles only when the workspace has room for their partial sums
   const bool split_ok = wl.slots_bytes > 0 && ws_bytes >= wl.total;
   const cudaStream_t st = as_stream(stream);
@@ -373,28 +389,39 @@ int run_gemm(int fmt, const uint16_t* x, const uint8_t* wq, const uint16_t* scal
     }
     const int grid = (N + kGvRows - 1) / kGvRows;
     const int mrows = M < 16 ? M : 16;
-    const int kp = gemv_pass_k(mrows, K);
+    const int kp = gemv_pass_k(mrows, K > K2 ? K : K2);
     const size_t smem = gemv_smem_bytes(mrows, kp);
     if (fmt == 0 && lora) {
       if (int e = gemv_prepare<0, true>()) return e;
       return launch(TGEMM_KIND_GEMV_Q2, st, [&] {
-        return pdl_launch(gemv_kernel<0, true>, grid, 256, smem, st, x, wq, scales, y, M, N, K, out_f32, u32, lb, r, mrows, kp);
+        return pdl_launch(gemv_kernel<0, true, false>, grid, 256, smem, st, x, wq, scales, y, M, N, K, out_f32, u32, lb, r, mrows, kp,
+                          nullptr, nullptr, nullptr, 0);
+      });
+    }
+    if (fmt == 0 && dual) {
+      if (int e = gemv_prepare<0, false, true>()) return e;
+      return launch(TGEMM_KIND_GEMV_Q2, st, [&] {
+        return pdl_launch(gemv_kernel<0, false, true>, grid, 256, smem, st, x, wq, scales, y, M, N, K, out_f32, nullptr, nullptr, 0, mrows, kp,
+                          in2.x, in2.wq, in2.d, K2);
       });
     }
     if (fmt == 0) {
       if (int e = gemv_prepare<0, false>()) return e;
       return launch(TGEMM_KIND_GEMV_Q2, st, [&] {
-        return pdl_launch(gemv_kernel<0, false>, grid, 256, smem, st, x, wq, scales, y, M, N, K, out_f32, nullptr, nullptr, 0, mrows, kp);
+        return pdl_launch(gemv_kernel<0, false, false>, grid, 256, smem, st, x, wq, scales, y, M, N, K, out_f32, nullptr, nullptr, 0, mrows, kp,
+                          static_cast<const uint16_t*>(nullptr), static_cast<const uint8_t*>(nullptr),
+                          static_cast<const uint16_t*>(nullptr), 0);
       });
     }
     if (int e = gemv_prepare<1, false>()) return e;
     return launch(TGEMM_KIND_GEMV_Q4, st, [&] {
-      return pdl_launch(gemv_kernel<1, false>, grid, 256, smem, st, x, wq, scales, y, M, N, K, out_f32, nullptr, nullptr, 0, mrows, kp);
+      return pdl_launch(gemv_kernel<1, false, false>, grid, 256, smem, st, x, wq, scales, y, M, N, K, out_f32, nullptr, nullptr, 0, mrows, kp,
+                        nullptr, nullptr, nullptr, 0);
     });
   }
 
   // ---- tensor-core path
-  TcSchedule sc = tc_schedule(M, N, K, lora ? ld.L : 0, di.sms);
+  TcSchedule sc = tc_schedule(M, N, K + K2, lora ? ld.L : 0, di.sms);
   if (sc.split && !split_ok) {
     // whole tiles per CTA (the workspace holds no partial-sum slots)
     sc.split = false;
@@ -433,6 +460,17 @@ int run_gemm(int fmt, const uint16_t* x, const uint8_t* wq, const uint16_t* scal
         }))
       return e;
   }
+  // the second input's f16 copy follows the first's in the workspace
+  uint16_t* x16b = x16 + static_cast<int64_t>(M) * K;
+  if (dual) {
+    const int64_t ngroups2 = static_cast<int64_t>(M) * K2 / 16;
+    const int pgrid2 = grid_for(ngroups2, 256, di.sms);
+    if (int e = launch(TGEMM_KIND_PREP, st, [&] {
+          return pdl_launch(prep_x16_kernel<0>, pgrid2, 256, 0, st, in2.x, x16b, ngroups2,
+                            static_cast<int*>(nullptr), 0);
+        }))
+      return e;
+  }
   CUtensorMap tm_x, tm_u;
   if (int e = make_map_2d(&tm_x, x16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, K, M, kTcBox, kTcTok,
                           CU_TENSOR_MAP_SWIZZLE_128B))
@@ -451,13 +489,26 @@ int run_gemm(int fmt, const uint16_t* x, const uint8_t* wq, const uint16_t* scal
                           fmt == 0 ? TcFmt<0>::kWqRowBytes : TcFmt<1>::kWqRowBytes, kTcRows,
                           CU_TENSOR_MAP_SWIZZLE_NONE))
     return e;
+  CUtensorMap tm_x2 = tm_x, tm_w2 = tm_w;  // unused with one input
+  if (dual) {
+    if (int e = make_map_2d(&tm_x2, x16b, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, K2, M, kTcBox, kTcTok,
+                            CU_TENSOR_MAP_SWIZZLE_128B))
+      return e;
+    if (int e = make_map_2d(&tm_w2, in2.wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1,
+                            static_cast<uint64_t>(K2) / 4, N, TcFmt<0>::kWqRowBytes, kTcRows,
+                            CU_TENSOR_MAP_SWIZZLE_NONE))
+      return e;
+  }
   TcParams p;
   p.M = M;
   p.N = N;
   p.K = K;
+  p.K2 = K2;
+  p.scales2 = in2.d;
   p.tiles_m = sc.tiles_m;
   p.num_tiles = sc.num_tiles;
-  p.kt_main = (K + kTcBK - 1) / kTcBK;
+  p.kt1 = (K + kTcBK - 1) / kTcBK;
+  p.kt_main = p.kt1 + (K2 + kTcBK - 1) / kTcBK;
   p.kt_lora = lora ? ld.L : 0;
   p.ksteps = sc.ksteps;
   p.upc = sc.upc;
@@ -476,18 +527,18 @@ int run_gemm(int fmt, const uint16_t* x, const uint8_t* wq, const uint16_t* scal
   if (fmt == 0 && !lora) {
     if (int e = tc_prepare<0, false>()) return e;
     return launch(TGEMM_KIND_TC_Q2, st, [&] {
-      return pdl_launch(tc_gemm_kernel<0, false>, grid, kTcThreads, TcFmt<0>::kSmemBytes, st, tm_x, tm_u, tm_w, p);
+      return pdl_launch(tc_gemm_kernel<0, false>, grid, kTcThreads, TcFmt<0>::kSmemBytes, st, tm_x, tm_u, tm_w, tm_x2, tm_w2, p);
     });
   }
   if (fmt == 0) {
     if (int e = tc_prepare<0, true>()) return e;
     return launch(TGEMM_KIND_TC_Q2_LORA, st, [&] {
-      return pdl_launch(tc_gemm_kernel<0, true>, grid, kTcThreads, TcFmt<0>::kSmemBytes, st, tm_x, tm_u, tm_w, p);
+      return pdl_launch(tc_gemm_kernel<0, true>, grid, kTcThreads, TcFmt<0>::kSmemBytes, st, tm_x, tm_u, tm_w, tm_x2, tm_w2, p);
     });
   }
   if (int e = tc_prepare<1, false>()) return e;
   return launch(TGEMM_KIND_TC_Q4, st, [&] {
-    return pdl_launch(tc_gemm_kernel<1, false>, grid, kTcThreads, TcFmt<1>::kSmemBytes, st, tm_x, tm_u, tm_w, p);
+    return pdl_launch(tc_gemm_kernel<1, false>, grid, kTcThreads, TcFmt<1>::kSmemBytes, st, tm_x, tm_u, tm_w, tm_x2, tm_w2, p);
   });
 }
 
@@ -624,6 +675,29 @@ int tgemm_q2_noalloc(const uint16_t* x, const uint8_t* wq, const uint16_t* d, vo
   }
   return run_gemm(0, x, wq, d, nullptr, nullptr, 0, y, M, N, K, out_dtype, scratch,
                   need > 0 ? static_cast<size_t>(TGEMM_NOALLOC_SCRATCH_BYTES) : 0, stream);
+}
+
+size_t tgemm_q2_dual_workspace_size(int M, int N, int K1, int K2) {
+  if (M < 1 || N < 1 || K1 < 1 || K2 < 1) return 0;
+  return workspace_layout(TGEMM_OP_Q2, M, N, K1, 0, choose_path(M), sms_for_sizing(), K2).total;
+}
+
+size_t tgemm_q2_dual_workspace_size_min(int M, int N, int K1, int K2) {
+  if (M < 1 || N < 1 || K1 < 1 || K2 < 1) return 0;
+  return workspace_layout(TGEMM_OP_Q2, M, N, K1, 0, choose_path(M), kDefaultSms, K2).total_whole;
+}
+
+int tgemm_q2_dual(const uint16_t* x1, const uint8_t* wq1, const uint16_t* d1, int K1,
+                  const uint16_t* x2, const uint8_t* wq2, const uint16_t* d2, int K2, void* y,
+                  int M, int N, int out_dtype, void* workspace, size_t ws_bytes, void* stream) {
+  if (K2 < 1) return TGEMM_EINVAL;
+  SecondInput in2;
+  in2.x = x2;
+  in2.wq = wq2;
+  in2.d = d2;
+  in2.K = K2;
+  return run_gemm(0, x1, wq1, d1, nullptr, nullptr, 0, y, M, N, K1, out_dtype, workspace,
+                  ws_bytes, stream, in2);
 }
 
 int tgemm_q4(const uint16_t* x, const uint8_t* wq, const uint16_t* sz, void* y, int M, int N,

@@ -191,6 +191,25 @@ int tgemm_q2_noalloc(const uint16_t* x, const uint8_t* wq, const uint16_t* d, vo
                      int N, int K, int out_dtype, void* stream);
 
 /*
+ * tgemm_q2_dual -- y = x1 . W1^T + x2 . W2^T for Q2_0 weights: a projection whose input
+ *   is two activations concatenated per token, split along its input axis into two
+ *   matmuls that are summed ("We're Teaching Your Browser to Paint", section "The GPU
+ *   driver, and the bug that looked like broken math", "Slice weights, not
+ *   activations").  Both products accumulate into one f32 accumulator in one kernel (no
+ *   intermediate y).
+ *   x1 [M][K1] and x2 [M][K2] bf16 (16-byte aligned); wq1 [N][K1/4], d1 [N][K1/128] and
+ *   wq2 [N][K2/4], d2 [N][K2/128] as for tgemm_q2; y [M][N] (16-byte aligned).
+ *   Requires M, N >= 1, K1 and K2 multiples of 128.  Workspace of
+ *   tgemm_q2_dual_workspace_size(M, N, K1, K2) bytes, or at least
+ *   tgemm_q2_dual_workspace_size_min() (whole tiles per CTA); 256-byte aligned.
+ */
+int tgemm_q2_dual(const uint16_t* x1, const uint8_t* wq1, const uint16_t* d1, int K1,
+                  const uint16_t* x2, const uint8_t* wq2, const uint16_t* d2, int K2, void* y,
+                  int M, int N, int out_dtype, void* workspace, size_t ws_bytes, void* stream);
+size_t tgemm_q2_dual_workspace_size(int M, int N, int K1, int K2);
+size_t tgemm_q2_dual_workspace_size_min(int M, int N, int K1, int K2);
+
+/*
  * tgemm_q4 -- y = x . W^T for 4-bit group weights.
  *   x [M][K] bf16 (16-byte aligned), wq [N][K/2] (16-byte aligned), sz [N][K/64][2] f16
  *   (4-byte aligned), y [M][N] (16-byte aligned), workspace as for tgemm_q2 with
