@@ -197,7 +197,8 @@ __device__ __forceinline__ void q4_word_to_f16(uint32_t w, uint32_t s2, uint32_t
   }
 }
 
-template <int FMT, bool LORA>
+// DUAL: stages [kt1, kt_main) read a second input (tm_x2, tm_w2, scales2, K2).
+template <int FMT, bool LORA, bool DUAL>
 __global__ void __launch_bounds__(kTcThreads, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x,
                    const __grid_constant__ CUtensorMap tm_u,
@@ -241,11 +242,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tm_x);
     if (LORA) tma_prefetch_desc(&tm_u);
-    if (p.kt1 < p.kt_main) tma_prefetch_desc(&tm_x2);
+    if (DUAL) tma_prefetch_desc(&tm_x2);
   }
   if (warp == kTcWProdWarp && lane == 0) {
     tma_prefetch_desc(&tm_w);
-    if (p.kt1 < p.kt_main) tma_prefetch_desc(&tm_w2);
+    if (DUAL) tma_prefetch_desc(&tm_w2);
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_slot), kTcTmemCols);
@@ -257,6 +258,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   pdl_trigger_and_wait();  // everything above touched only shared and tensor memory
   const uint32_t tmem_base = *tmem_slot;
   const int ksteps = p.ksteps;
+  const int kt1 = DUAL ? p.kt1 : p.kt_main;  // stages of the first input
   const int u0 = static_cast<int>(blockIdx.x) * p.upc;  // this CTA's units [u0, u1)
   const int u1 = min(p.units, u0 + p.upc);
 
@@ -272,8 +274,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const uint32_t xdst = sbase + F::kXOff + s * kTcXBytes;
         mbar_arrive_expect_tx(full_bar(s), kTcXBytes);
         // stage ks: first input, second input, or the branch's u
-        const CUtensorMap* map = ks < p.kt1 ? &tm_x : (ks < p.kt_main ? &tm_x2 : &tm_u);
-        const int k0 = (ks < p.kt1 ? ks : (ks < p.kt_main ? ks - p.kt1 : ks - p.kt_main)) * kTcBK;
+        const CUtensorMap* map = ks < kt1 ? &tm_x : (ks < p.kt_main ? &tm_x2 : &tm_u);
+        const int k0 = (ks < kt1 ? ks : (ks < p.kt_main ? ks - kt1 : ks - p.kt_main)) * kTcBK;
         tma_load_2d(xdst, map, full_bar(s), k0, tm * kTcTok);
         tma_load_2d(xdst + kTcXBoxBytes, map, full_bar(s), k0 + kTcBox, tm * kTcTok);
       }
@@ -352,8 +354,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     // pair (0 where the item has none: a branch stage, a row past N, codes past K).
     auto scale_at = [&](int ks_, int row_, bool in) -> uint32_t {
       if (!in || row_ >= p.N || ks_ >= p.kt_main) return 0u;
-      const bool second = ks_ >= p.kt1;  // the second input's stages
-      if (second) ks_ -= p.kt1;
+      const bool second = DUAL && ks_ >= kt1;  // the second input's stages
+      if (second) ks_ -= kt1;
       const int k_first = ks_ * kTcBK + part * kC;
       if (k_first >= (second ? p.K2 : p.K)) return 0u;
       const uint16_t* srow = (second ? p.scales2 : p.scales) +
@@ -567,9 +569,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const uint32_t w = wit % F::kWStages, ph = (wit / F::kWStages) & 1u;
         if (!mbar_wait(wempty_bar(w), ph ^ 1u, abort_flag)) break;
         mbar_arrive_expect_tx(wfull_bar(w), F::kWBytes);
-        const bool second = ks >= p.kt1;
+        const bool second = DUAL && ks >= kt1;
         tma_load_2d(sbase + F::kWOff + w * F::kWBytes, second ? &tm_w2 : &tm_w, wfull_bar(w),
-                    (second ? ks - p.kt1 : ks) * F::kWqRowBytes, (tile / p.tiles_m) * kTcRows);
+                    (second ? ks - kt1 : ks) * F::kWqRowBytes, (tile / p.tiles_m) * kTcRows);
         ++wit;
       }
       // every load issued must land before the CTA may exit

@@ -172,12 +172,12 @@ int make_map_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dtype, i
 
 // ---- kernel attribute setup (once per instantiation) ------------------------------------
 
-template <int FMT, bool LORA>
+template <int FMT, bool LORA, bool DUAL = false>
 int tc_prepare() {
   static std::once_flag once;
   static cudaError_t err = cudaSuccess;
   std::call_once(once, [] {
-    err = cudaFuncSetAttribute(tc_gemm_kernel<FMT, LORA>,
+    err = cudaFuncSetAttribute(tc_gemm_kernel<FMT, LORA, DUAL>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize,
                                TcFmt<FMT>::kSmemBytes);
   });
@@ -524,21 +524,27 @@ int run_gemm(int fmt, const uint16_t* x, const uint8_t* wq, const uint16_t* scal
   p.part = sc.split ? reinterpret_cast<float*>(ws + wl.slots) : nullptr;
   p.cnt = cnt;
   const int grid = sc.grid;
+  if (dual) {
+    if (int e = tc_prepare<0, false, true>()) return e;
+    return launch(TGEMM_KIND_TC_Q2, st, [&] {
+      return pdl_launch(tc_gemm_kernel<0, false, true>, grid, kTcThreads, TcFmt<0>::kSmemBytes, st, tm_x, tm_u, tm_w, tm_x2, tm_w2, p);
+    });
+  }
   if (fmt == 0 && !lora) {
     if (int e = tc_prepare<0, false>()) return e;
     return launch(TGEMM_KIND_TC_Q2, st, [&] {
-      return pdl_launch(tc_gemm_kernel<0, false>, grid, kTcThreads, TcFmt<0>::kSmemBytes, st, tm_x, tm_u, tm_w, tm_x2, tm_w2, p);
+      return pdl_launch(tc_gemm_kernel<0, false, false>, grid, kTcThreads, TcFmt<0>::kSmemBytes, st, tm_x, tm_u, tm_w, tm_x2, tm_w2, p);
     });
   }
   if (fmt == 0) {
     if (int e = tc_prepare<0, true>()) return e;
     return launch(TGEMM_KIND_TC_Q2_LORA, st, [&] {
-      return pdl_launch(tc_gemm_kernel<0, true>, grid, kTcThreads, TcFmt<0>::kSmemBytes, st, tm_x, tm_u, tm_w, tm_x2, tm_w2, p);
+      return pdl_launch(tc_gemm_kernel<0, true, false>, grid, kTcThreads, TcFmt<0>::kSmemBytes, st, tm_x, tm_u, tm_w, tm_x2, tm_w2, p);
     });
   }
   if (int e = tc_prepare<1, false>()) return e;
   return launch(TGEMM_KIND_TC_Q4, st, [&] {
-    return pdl_launch(tc_gemm_kernel<1, false>, grid, kTcThreads, TcFmt<1>::kSmemBytes, st, tm_x, tm_u, tm_w, tm_x2, tm_w2, p);
+    return pdl_launch(tc_gemm_kernel<1, false, false>, grid, kTcThreads, TcFmt<1>::kSmemBytes, st, tm_x, tm_u, tm_w, tm_x2, tm_w2, p);
   });
 }
 
