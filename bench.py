@@ -505,10 +505,12 @@ def ours(args, world, rank, local):
     # ---- small-M stream: 64 distinct 3072x3072 weights (160 MB > L2), one graph of 64 GEMVs
     parts = {}
     if extras:
-        try:
-            parts["gemv_stream"] = gemv_stream(tg, torch, stream)
-        except Exception as exc:  # report, do not hide
-            parts["gemv_stream"] = {"error": str(exc)}
+        for key, fn in (("gemv_stream", gemv_stream), ("dual_out_projection", dual_out_projection),
+                        ("token_sweep", token_sweep)):
+            try:
+                parts[key] = fn(tg, torch, stream)
+            except Exception as exc:  # report, do not hide
+                parts[key] = {"error": str(exc)}
 
     dev_err = tg.device_error()
     cpu = None
@@ -551,6 +553,72 @@ def ours(args, world, rank, local):
     }
     if rank == 0:
         print(json.dumps(line), flush=True)
+
+
+def _time_calls(torch, fn, reps=20, warm=3):
+    """Median device time (seconds) of fn() over `reps` single calls, L2 flushed before each."""
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")
+    for _ in range(warm):
+        fn()
+    times = []
+    for _ in range(reps):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        fn()
+        b.record()
+        torch.cuda.synchronize()
+        times.append(a.elapsed_time(b) * 1e-3)
+    return statistics.median(times)
+
+
+def _q2_device_weights(tg, torch, N, K, seed):
+    g = torch.Generator(device="cuda").manual_seed(seed)
+    codes = torch.randint(0, 3, (N, K), dtype=torch.uint8, device="cuda", generator=g)
+    scale = (torch.rand(N, K // 128, device="cuda", generator=g) * 0.02).half().float()
+    wq, d, _ = tg.q2_pack(codes, scale)
+    return wq, d
+
+
+def dual_out_projection(tg, torch, stream):
+    """The MMDiT's fused out projection split along its input axis (page 2, 'Slice weights,
+    not activations'): 1536 tokens, N = 3072, K1 = 3072 (attention output) + K2 = 12288
+    (MLP output), bf16 out; one fused call against two separate calls plus an add."""
+    M, N, K1, K2 = 1536, 3072, 3072, 12288
+    wq1, d1 = _q2_device_weights(tg, torch, N, K1, 5)
+    wq2, d2 = _q2_device_weights(tg, torch, N, K2, 6)
+    x1 = torch.randn(M, K1, device="cuda").bfloat16()
+    x2 = torch.randn(M, K2, device="cuda").bfloat16()
+    y = torch.empty(M, N, device="cuda", dtype=torch.bfloat16)
+    ws = torch.empty(tg.dual_workspace_size(M, N, K1, K2), dtype=torch.uint8, device="cuda")
+    fused = _time_calls(torch, lambda: tg.gemm_q2_dual(x1, wq1, d1, x2, wq2, d2, y=y, workspace=ws))
+    y1 = torch.empty(M, N, device="cuda", dtype=torch.float32)
+    y2 = torch.empty(M, N, device="cuda", dtype=torch.float32)
+
+    def separate():
+        tg.gemm_q2(x1, wq1, d1, out_dtype=tg.OUT_F32, y=y1)
+        tg.gemm_q2(x2, wq2, d2, out_dtype=tg.OUT_F32, y=y2)
+        torch.add(y1, y2, out=y1)
+    sep = _time_calls(torch, separate)
+    flop = 2 * M * N * (K1 + K2)
+    return {"shape": f"{M} tokens x {N} x ({K1} + {K2})", "fused_us": fused * 1e6,
+            "fused_tflops": flop / fused / 1e12, "two_calls_plus_add_us": sep * 1e6}
+
+
+def token_sweep(tg, torch, stream):
+    """The 9216 x 3072 ternary matmul at the pages' step token counts (256 + text rows at
+    256^2, 384 = quarter-size first step, 1280 = 1024 patches + 256, 1536) and 4096."""
+    N, K = 9216, 3072
+    wq, d = _q2_device_weights(tg, torch, N, K, 7)
+    out = {}
+    for M in (256, 384, 1280, 1536, 4096):
+        x = torch.randn(M, K, device="cuda").bfloat16()
+        y = torch.empty(M, N, device="cuda", dtype=torch.bfloat16)
+        ws = torch.empty(max(tg.workspace_size(tg.OP_Q2, M, N, K), 256), dtype=torch.uint8,
+                         device="cuda")
+        t = _time_calls(torch, lambda: tg.gemm_q2(x, wq, d, y=y, workspace=ws), reps=10)
+        out[f"m{M}"] = {"us": t * 1e6, "tflops": 2 * M * N * K / t / 1e12}
+    return out
 
 
 def gemv_stream(tg, torch, stream):
