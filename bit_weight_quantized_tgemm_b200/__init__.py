@@ -12,5 +12,5 @@ from .binding import (  # noqa: F401
     workspace_size_min,
     KIND_GEMV_Q2, KIND_GEMV_Q4, KIND_PREP, KIND_TC_Q2, KIND_TC_Q2_LORA, KIND_TC_Q4,
     launch_count, profile_enable, profile_read, ETOOLARGE, NOALLOC_SCRATCH_BYTES,
-    gemm_q2_noalloc, gemm_q2_dual, dual_workspace_size,
+    gemm_q2_noalloc, gemm_q2_dual, dual_workspace_size, tc_plan, TC_PLAN_KEYS,
 )

@@ -39,6 +39,7 @@ _SIGS = {
     "tgemm_workspace_size_min": (_sz, [_i, _i, _i, _i, _i]),
     "tgemm_q2_dual_workspace_size": (_sz, [_i, _i, _i, _i]),
     "tgemm_q2_dual_workspace_size_min": (_sz, [_i, _i, _i, _i]),
+    "tgemm_tc_plan": (_i, [_i, _i, _i, _i, _i, _i, _i, _P]),
     "tgemm_q2": (_i, [_P, _P, _P, _P, _i, _i, _i, _i, _P, _sz, _P]),
     "tgemm_q2_lora": (_i, [_P, _P, _P, _P, _P, _i, _P, _i, _i, _i, _i, _P, _sz, _P]),
     "tgemm_q4": (_i, [_P, _P, _P, _P, _i, _i, _i, _i, _P, _sz, _P]),
@@ -173,6 +174,16 @@ def workspace_size(op: int, M: int, N: int, K: int, r: int = 0) -> int:
 def workspace_size_min(op: int, M: int, N: int, K: int, r: int = 0) -> int:
     """Smallest accepted workspace (whole tiles per CTA); see tgemm_workspace_size_min."""
     return int(lib().tgemm_workspace_size_min(op, M, N, K, r))
+
+
+TC_PLAN_KEYS = ("tiles_m", "num_tiles", "ksteps", "sk_t0", "upc", "dpc", "grid", "split")
+
+
+def tc_plan(op: int, M: int, N: int, K: int, r: int = 0, K2: int = 0, sms: int = 148) -> dict:
+    """The tensor-core kernel's schedule for these sizes on `sms` SMs (tgemm_tc_plan)."""
+    out = (ctypes.c_int * len(TC_PLAN_KEYS))()
+    _check(lib().tgemm_tc_plan(op, M, N, K, r, K2, sms, out), "tgemm_tc_plan")
+    return dict(zip(TC_PLAN_KEYS, out))
 
 
 _ws_cache = {}

@@ -1,11 +1,18 @@
 // gemm_tc.cuh -- large-M path: persistent tcgen05 (5th-generation tensor core) kernel.
 //
-// Schedule: a tile's work is `ksteps` units (its 128-k stages, then the branch's stages).
-// The units of all tiles, tile-major, are cut into equal contiguous ranges, one per CTA.
-// When the range length is a multiple of ksteps every CTA owns whole tiles; otherwise
-// (chosen by the host when tiles divide badly over the SMs, e.g. 40 or 152 tiles on 148
-// SMs) a tile can be shared by consecutive CTAs ("stream-K"): each writes its f32 partial
-// sum to a slot in the workspace and the last to arrive adds the slots in k order.
+// Schedule: a tile's work is `ksteps` units (its 128-k stages, then the branch's stages),
+// numbered tile-major.  The tiles are split in two regions:
+//   whole-tile region, tiles [0, sk_t0): CTA c owns the units [c * dpc, (c + 1) * dpc),
+//     a whole number of tiles;
+//   split region, tiles [sk_t0, num_tiles): its units are cut into equal contiguous ranges
+//     of `upc`, one per CTA, so a tile can be shared by consecutive CTAs ("stream-K"): each
+//     writes its f32 partial sum to a slot in the workspace and the last to arrive adds the
+//     slots in k order.
+// A CTA works through its split-region range first, then its whole tiles, so the split
+// tiles' partial sums and fix-ups overlap the whole tiles' MMAs and every CTA ends on a
+// whole tile stored straight from the accumulator.  The host picks sk_t0 = 0 with upc a
+// multiple of ksteps (whole tiles only), sk_t0 = 0 with dpc = 0 (all tiles shared, for
+// fewer tiles than SMs), or sk_t0 = floor(tiles / SMs) * SMs (the remainder shared).
 //
 // Tile: 128 weight rows (MMA M, TMEM lanes) x 256 tokens (MMA N, accumulator columns),
 // 128 k per stage (an M=128 MMA costs the same time for any N up to 256, so N is 256;
@@ -113,7 +120,7 @@ struct TcParams {
   int K2;          // the second input's width (0: one input)
   int kt_lora;     // extra stages for the low-rank branch (0 without it)
   int ksteps;      // kt_main + kt_lora: units of work per tile
-  int upc;         // units per CTA: CTA c owns units [c * upc, min(U, (c + 1) * upc))
+  int upc;         // split region: CTA c owns units sk_t0 * ksteps + [c * upc, (c + 1) * upc)
   int units;       // U = num_tiles * ksteps
   int lora_mmas;   // K=16 MMAs in those stages: 2 * round_up(r, 16) / 16
   int R;           // round_up(r, 16): width of u_hi (and of u_lo) in the concatenation
@@ -125,10 +132,12 @@ struct TcParams {
   const uint16_t* lb;      // low-rank B [N][r] (bf16)
   void* y;
   float* part;             // split tiles: 2 slots of 128 x 256 f32 per CTA
-  int* cnt;                // split tiles: 8 arrival counters per tile, zero at launch
+  int* cnt;                // split region: 8 arrival counters per tile, zero at launch
+  int sk_t0;               // first tile of the split region (tiles before it are whole per CTA)
+  int dpc;                 // whole-tile region: CTA c owns units [c * dpc, (c + 1) * dpc) (0: none)
 };
 
-// One tile's share of a CTA's unit range: tile `tile`, stages [ka, kb).
+// One tile's share of a CTA's unit range [u, u1): tile `tile`, stages [ka, kb).
 struct TcSeg {
   int tile, ka, kb;
 };
@@ -137,10 +146,25 @@ __device__ __forceinline__ TcSeg tc_seg_at(const TcParams& p, int u, int u1) {
   const int end = min(u1, (t + 1) * p.ksteps);
   return TcSeg{t, u - t * p.ksteps, end - t * p.ksteps};
 }
-// Slot of the partial sum that CTA c writes for its segment of tile t: a segment that
-// starts mid-tile (or at the tile's start) is the CTA's first, any other its last.
+// A CTA's two unit ranges: [a0, a1) in the split region, then [b0, b1) of whole tiles
+// (either may be empty).
+struct TcRanges {
+  int a0, a1, b0, b1;
+};
+__device__ __forceinline__ TcRanges tc_ranges(const TcParams& p, int c) {
+  const int sk_u0 = p.sk_t0 * p.ksteps;
+  TcRanges r;
+  r.a0 = sk_u0 + c * p.upc;
+  r.a1 = max(r.a0, min(p.units, r.a0 + p.upc));
+  r.b0 = c * p.dpc;
+  r.b1 = max(r.b0, min(sk_u0, r.b0 + p.dpc));
+  return r;
+}
+// Slot of the partial sum that CTA c writes for its segment of split-region tile t: a
+// segment that starts mid-tile (or at the tile's start) is the CTA's first, any other its
+// last.
 __device__ __forceinline__ int tc_slot(const TcParams& p, int c, int t) {
-  return c * p.upc >= t * p.ksteps ? 2 * c : 2 * c + 1;
+  return c * p.upc >= (t - p.sk_t0) * p.ksteps ? 2 * c : 2 * c + 1;
 }
 constexpr int kTcSlotFloats = kTcRows * kTcTok;
 
@@ -198,7 +222,9 @@ __device__ __forceinline__ void q4_word_to_f16(uint32_t w, uint32_t s2, uint32_t
 }
 
 // DUAL: stages [kt1, kt_main) read a second input (tm_x2, tm_w2, scales2, K2).
-template <int FMT, bool LORA, bool DUAL>
+// HYB: the schedule has a whole-tile region as well as the split region (p.dpc > 0); without
+// it every CTA runs one unit range and the loops compile to that alone.
+template <int FMT, bool LORA, bool DUAL, bool HYB>
 __global__ void __launch_bounds__(kTcThreads, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x,
                    const __grid_constant__ CUtensorMap tm_u,
@@ -259,18 +285,22 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const uint32_t tmem_base = *tmem_slot;
   const int ksteps = p.ksteps;
   const int kt1 = DUAL ? p.kt1 : p.kt_main;  // stages of the first input
-  const int u0 = static_cast<int>(blockIdx.x) * p.upc;  // this CTA's units [u0, u1)
-  const int u1 = min(p.units, u0 + p.upc);
+  const TcRanges rg = tc_ranges(p, static_cast<int>(blockIdx.x));  // this CTA's units
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       uint32_t it = 0;
-      for (int u = u0; u < u1; ++u, ++it) {
+      bool ok = true;
+      for (int r = 0; ok && r < (HYB ? 2 : 1); ++r)
+      for (int u = r ? rg.b0 : rg.a0, ue = r ? rg.b1 : rg.a1; u < ue; ++u, ++it) {
         const int tile = u / ksteps, ks = u - tile * ksteps;
         const int tm = tile % p.tiles_m;
         const uint32_t s = it % kTcStages, ph = (it / kTcStages) & 1u;
-        if (!mbar_wait(empty_bar(s), ph ^ 1u, abort_flag)) break;
+        if (!mbar_wait(empty_bar(s), ph ^ 1u, abort_flag)) {
+          ok = false;
+          break;
+        }
         const uint32_t xdst = sbase + F::kXOff + s * kTcXBytes;
         mbar_arrive_expect_tx(full_bar(s), kTcXBytes);
         // stage ks: first input, second input, or the branch's u
@@ -291,8 +321,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       constexpr uint32_t kIdescLora = make_idesc_f16(1u, kTcRows, kTcTok);  // bf16 x bf16
       uint32_t it = 0, scount = 0;
       bool ok = true;
-      for (int u = u0; ok && u < u1; ++scount) {
-        const TcSeg sg = tc_seg_at(p, u, u1);
+      for (int r = 0; ok && r < (HYB ? 2 : 1); ++r)
+      for (int u = r ? rg.b0 : rg.a0, ue = r ? rg.b1 : rg.a1; ok && u < ue; ++scount) {
+        const TcSeg sg = tc_seg_at(p, u, ue);
         u += sg.kb - sg.ka;
         if (!mbar_wait(accempty_bar, (scount & 1u) ^ 1u, abort_flag)) { ok = false; break; }
         tc_fence_after();
@@ -345,10 +376,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     uint32_t wit = 0;   // A stages written
     uint32_t wcnt = 0;  // weight stages consumed
     bool ok = true;
-    // This CTA's work is one stream of (tile, stage) items, item i being unit u0 + i; the
-    // position is advanced item by item (no divisions on the way).
-    const int n_items = u1 > u0 ? u1 - u0 : 0;
-    int tile = u0 / ksteps, ks = u0 - tile * ksteps;
+    // This CTA's work is one stream of (tile, stage) items: its split-region units, then
+    // its whole tiles.  The position is advanced item by item with one compare against
+    // the end of the current tile's segment (its last stage, or the first range's end);
+    // only there is the next tile (or the jump to the whole tiles) worked out.
+    const int n_first = rg.a1 - rg.a0;
+    const int n_items = HYB ? n_first + (rg.b1 - rg.b0) : n_first;
+    bool in_first = !HYB || n_first > 0;
+    const int u_start = in_first ? rg.a0 : rg.b0;
+    int tile = u_start / ksteps, ks = u_start - tile * ksteps;
+    int seg_end = HYB && in_first ? min(ksteps, rg.a1 - tile * ksteps) : ksteps;
     int row = (tile / p.tiles_m) * kTcRows + rt;
     // The scale of the item at (ks, row): Q2 block scale d, or the 4-bit group's (s, z)
     // pair (0 where the item has none: a branch stage, a row past N, codes past K).
@@ -368,9 +405,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const uint32_t sc = sc_next;
       const bool valid = row < p.N;
       int nks = ks + 1, ntile = tile, nrow = row;
-      if (nks == ksteps) {
+      if (nks == seg_end) {
         nks = 0;
-        ++ntile;
+        if (HYB && in_first && ntile * ksteps + seg_end == rg.a1) {
+          in_first = false;  // on to the whole tiles, which start on a tile boundary
+          ntile = rg.b0 / ksteps;
+        } else {
+          ++ntile;
+        }
+        if (HYB) seg_end = in_first ? min(ksteps, rg.a1 - ntile * ksteps) : ksteps;
         nrow = (ntile / p.tiles_m) * kTcRows + rt;
       }
       sc_next = scale_at(nks, nrow, i + 1 < n_items);
@@ -470,11 +513,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     constexpr int kChunks = kTcTok / 32 / 2;
     constexpr int kPieceFloats = kTcSlotFloats / kTcEpiWarps;
     uint32_t scount = 0;
-    for (int u = u0; u < u1; ++scount) {
-      const TcSeg sg = tc_seg_at(p, u, u1);
+    bool ok = true;
+    for (int r = 0; ok && r < (HYB ? 2 : 1); ++r)
+    for (int u = r ? rg.b0 : rg.a0, ue = r ? rg.b1 : rg.a1; u < ue; ++scount) {
+      const TcSeg sg = tc_seg_at(p, u, ue);
       u += sg.kb - sg.ka;
       const int tm = sg.tile % p.tiles_m, tn = sg.tile / p.tiles_m;
-      if (!mbar_wait_warp(accfull_bar, scount & 1u, abort_flag)) break;
+      if (!mbar_wait_warp(accfull_bar, scount & 1u, abort_flag)) {
+        ok = false;
+        break;
+      }
       tc_fence_after();
       const int n = tn * kTcRows + q * 32 + lane;  // this thread's weight row
       const bool nv = n < p.N;
@@ -533,10 +581,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       __threadfence();
       __syncwarp();
       int before = 0;
-      if (lane == 0) before = atomicAdd(p.cnt + sg.tile * kTcEpiWarps + piece, 1);
+      const int t_rel = sg.tile - p.sk_t0;  // the tile's place in the split region
+      if (lane == 0) before = atomicAdd(p.cnt + t_rel * kTcEpiWarps + piece, 1);
       before = __shfl_sync(0xFFFFFFFFu, before, 0);
-      const int c_lo = sg.tile * ksteps / p.upc;
-      const int c_hi = ((sg.tile + 1) * ksteps - 1) / p.upc;
+      const int c_lo = t_rel * ksteps / p.upc;
+      const int c_hi = ((t_rel + 1) * ksteps - 1) / p.upc;
       if (before != c_hi - c_lo) continue;  // another CTA's warp finishes this piece
       __threadfence();
 #pragma unroll 1
@@ -563,11 +612,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     // the weight ring, as far ahead of the dequant warps as the ring allows.
     if (lane == 0) {
       uint32_t wit = 0;
-      for (int u = u0; u < u1; ++u) {
+      bool ok = true;
+      for (int r = 0; ok && r < (HYB ? 2 : 1); ++r)
+      for (int u = r ? rg.b0 : rg.a0, ue = r ? rg.b1 : rg.a1; u < ue; ++u) {
         const int tile = u / ksteps, ks = u - tile * ksteps;
         if (ks >= p.kt_main) continue;  // branch stages carry no codes
         const uint32_t w = wit % F::kWStages, ph = (wit / F::kWStages) & 1u;
-        if (!mbar_wait(wempty_bar(w), ph ^ 1u, abort_flag)) break;
+        if (!mbar_wait(wempty_bar(w), ph ^ 1u, abort_flag)) {
+          ok = false;
+          break;
+        }
         mbar_arrive_expect_tx(wfull_bar(w), F::kWBytes);
         const bool second = DUAL && ks >= kt1;
         tma_load_2d(sbase + F::kWOff + w * F::kWBytes, second ? &tm_w2 : &tm_w, wfull_bar(w),

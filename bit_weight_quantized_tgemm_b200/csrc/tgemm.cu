@@ -8,6 +8,7 @@
 #include <cstdint>
 #include <cstdio>
 #include <mutex>
+#include <type_traits>
 #include <vector>
 
 #include "../../include/tgemm.h"
@@ -172,12 +173,12 @@ int make_map_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dtype, i
 
 // ---- kernel attribute setup (once per instantiation) ------------------------------------
 
-template <int FMT, bool LORA, bool DUAL = false>
+template <int FMT, bool LORA, bool DUAL, bool HYB>
 int tc_prepare() {
   static std::once_flag once;
   static cudaError_t err = cudaSuccess;
   std::call_once(once, [] {
-    err = cudaFuncSetAttribute(tc_gemm_kernel<FMT, LORA, DUAL>,
+    err = cudaFuncSetAttribute(tc_gemm_kernel<FMT, LORA, DUAL, HYB>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize,
                                TcFmt<FMT>::kSmemBytes);
   });
@@ -211,16 +212,30 @@ LoraDims lora_dims(int r, int K) {
   return d;
 }
 
-// Tensor-core schedule: units (tile, 128-k stage) cut into one contiguous range per CTA.
-// Whole tiles per CTA when the tiles fill the SMs evenly enough; otherwise ranges of
-// ceil(U / SMs) units that may split tiles between CTAs (see gemm_tc.cuh).
+// Tensor-core schedule (see gemm_tc.cuh): units (tile, 128-k stage), tile-major, in a
+// whole-tile region of floor(tiles / SMs) tiles per CTA and a split region where the
+// remaining tiles' units are cut into equal contiguous ranges, one per CTA.  It is the
+// split form only when it saves more than the split tiles' charge over whole tiles alone.
 constexpr int kDefaultSms = 148;    // sizes workspaces when no device is visible (B200)
 constexpr int kSplitPenalty = 2;    // units a split tile is charged (partial sums + fixup)
+constexpr int kMaxShare = 4;        // CTAs that may share a split tile next to whole tiles
 
 struct TcSchedule {
-  int ksteps = 0, tiles_m = 0, num_tiles = 0, units = 0, upc = 0, grid = 0;
+  int ksteps = 0, tiles_m = 0, num_tiles = 0, units = 0, grid = 0;
+  int sk_t0 = 0;  // first tile of the split region
+  int upc = 0;    // split-region units per CTA
+  int dpc = 0;    // whole-tile units per CTA before the split region (0: none)
   bool split = false;
 };
+
+// Whole tiles only: ceil(tiles / CTAs) per CTA, expressed as a split region of whole tiles.
+void tc_schedule_whole(TcSchedule& s, int sms) {
+  s.split = false;
+  s.sk_t0 = 0;
+  s.dpc = 0;
+  s.upc = (s.num_tiles + sms - 1) / sms * s.ksteps;
+  s.grid = (s.units + s.upc - 1) / s.upc;
+}
 
 TcSchedule tc_schedule(int M, int N, int K, int kt_lora, int sms) {
   TcSchedule s;
@@ -228,12 +243,21 @@ TcSchedule tc_schedule(int M, int N, int K, int kt_lora, int sms) {
   s.tiles_m = (M + kTcTok - 1) / kTcTok;
   s.num_tiles = s.tiles_m * ((N + kTcRows - 1) / kTcRows);
   s.units = s.num_tiles * s.ksteps;
-  const int waves = (s.num_tiles + sms - 1) / sms;
-  const int upc_whole = waves * s.ksteps;
-  const int upc_split = (s.units + sms - 1) / sms;
-  s.split = upc_split + kSplitPenalty < upc_whole;
-  s.upc = s.split ? upc_split : upc_whole;
-  s.grid = (s.units + s.upc - 1) / s.upc;
+  tc_schedule_whole(s, sms);
+  const int whole = s.upc;                       // the longest CTA's units, whole tiles
+  int wf = s.num_tiles / sms;                    // whole tiles every CTA gets
+  if (wf * sms == s.num_tiles) return s;         // the tiles fill the SMs evenly
+  // A few remainder tiles cut over all CTAs would each be summed from many partial sums
+  // by one CTA; give the split region one more wave of tiles instead.
+  if (wf > 0 && (s.num_tiles - wf * sms) * kMaxShare < sms) --wf;
+  const int sk_t0 = wf * sms;
+  const int upc = ((s.num_tiles - sk_t0) * s.ksteps + sms - 1) / sms;
+  if (wf * s.ksteps + upc + kSplitPenalty >= whole) return s;
+  s.split = true;
+  s.sk_t0 = sk_t0;
+  s.upc = upc;
+  s.dpc = wf * s.ksteps;
+  s.grid = wf > 0 ? sms : ((s.units + upc - 1) / upc);
   return s;
 }
 
@@ -287,7 +311,7 @@ Workspace workspace_layout(int op, int M, int N, int K, int r, int path, int sms
       w.slots_bytes = static_cast<size_t>(2) * sc.grid * kTcSlotFloats * 4;
       off = round_up(off + w.slots_bytes, 256);
       w.cnt = off;
-      w.cnt_bytes = static_cast<size_t>(sc.num_tiles) * kTcEpiWarps * 4;
+      w.cnt_bytes = static_cast<size_t>(sc.num_tiles - sc.sk_t0) * kTcEpiWarps * 4;
       off = round_up(off + w.cnt_bytes, 256);
     }
   }
@@ -424,12 +448,10 @@ int run_gemm(int fmt, const uint16_t* x, const uint8_t* wq, const uint16_t* scal
   TcSchedule sc = tc_schedule(M, N, K + K2, lora ? ld.L : 0, di.sms);
   if (sc.split && !split_ok) {
     // whole tiles per CTA (the workspace holds no partial-sum slots)
-    sc.split = false;
-    sc.upc = (sc.num_tiles + di.sms - 1) / di.sms * sc.ksteps;
-    sc.grid = (sc.units + sc.upc - 1) / sc.upc;
+    tc_schedule_whole(sc, di.sms);
   }
   int* cnt = sc.split ? reinterpret_cast<int*>(ws + wl.cnt) : nullptr;
-  const int ncnt = sc.split ? sc.num_tiles * kTcEpiWarps : 0;
+  const int ncnt = sc.split ? (sc.num_tiles - sc.sk_t0) * kTcEpiWarps : 0;
   uint16_t* x16 = reinterpret_cast<uint16_t*>(ws + wl.x16);
   uint16_t* ucat = nullptr;
   if (lora) {
@@ -511,7 +533,9 @@ int run_gemm(int fmt, const uint16_t* x, const uint8_t* wq, const uint16_t* scal
   p.kt_main = p.kt1 + (K2 + kTcBK - 1) / kTcBK;
   p.kt_lora = lora ? ld.L : 0;
   p.ksteps = sc.ksteps;
+  p.sk_t0 = sc.sk_t0;
   p.upc = sc.upc;
+  p.dpc = sc.dpc;
   p.units = sc.units;
   p.lora_mmas = lora ? 2 * ld.R / 16 : 0;
   p.R = ld.R;
@@ -524,28 +548,30 @@ int run_gemm(int fmt, const uint16_t* x, const uint8_t* wq, const uint16_t* scal
   p.part = sc.split ? reinterpret_cast<float*>(ws + wl.slots) : nullptr;
   p.cnt = cnt;
   const int grid = sc.grid;
-  if (dual) {
-    if (int e = tc_prepare<0, false, true>()) return e;
-    return launch(TGEMM_KIND_TC_Q2, st, [&] {
-      return pdl_launch(tc_gemm_kernel<0, false, true>, grid, kTcThreads, TcFmt<0>::kSmemBytes, st, tm_x, tm_u, tm_w, tm_x2, tm_w2, p);
+  // one instantiation per (format, branch, second input, whole-tile region)
+  auto run_tc = [&](auto fmt_c, auto lora_c, auto dual_c, auto hyb_c, int kind) -> int {
+    constexpr int kF = decltype(fmt_c)::value;
+    constexpr bool kL = decltype(lora_c)::value, kD = decltype(dual_c)::value;
+    constexpr bool kH = decltype(hyb_c)::value;
+    if (int e = tc_prepare<kF, kL, kD, kH>()) return e;
+    return launch(kind, st, [&] {
+      return pdl_launch(tc_gemm_kernel<kF, kL, kD, kH>, grid, kTcThreads, TcFmt<kF>::kSmemBytes, st,
+                        tm_x, tm_u, tm_w, tm_x2, tm_w2, p);
     });
-  }
-  if (fmt == 0 && !lora) {
-    if (int e = tc_prepare<0, false>()) return e;
-    return launch(TGEMM_KIND_TC_Q2, st, [&] {
-      return pdl_launch(tc_gemm_kernel<0, false, false>, grid, kTcThreads, TcFmt<0>::kSmemBytes, st, tm_x, tm_u, tm_w, tm_x2, tm_w2, p);
-    });
-  }
-  if (fmt == 0) {
-    if (int e = tc_prepare<0, true>()) return e;
-    return launch(TGEMM_KIND_TC_Q2_LORA, st, [&] {
-      return pdl_launch(tc_gemm_kernel<0, true, false>, grid, kTcThreads, TcFmt<0>::kSmemBytes, st, tm_x, tm_u, tm_w, tm_x2, tm_w2, p);
-    });
-  }
-  if (int e = tc_prepare<1, false>()) return e;
-  return launch(TGEMM_KIND_TC_Q4, st, [&] {
-    return pdl_launch(tc_gemm_kernel<1, false, false>, grid, kTcThreads, TcFmt<1>::kSmemBytes, st, tm_x, tm_u, tm_w, tm_x2, tm_w2, p);
-  });
+  };
+  using F0 = std::integral_constant<int, 0>;
+  using F1 = std::integral_constant<int, 1>;
+  using On = std::true_type;
+  using Off = std::false_type;
+  const bool hyb = sc.dpc > 0;
+  if (dual)
+    return hyb ? run_tc(F0{}, Off{}, On{}, On{}, TGEMM_KIND_TC_Q2) : run_tc(F0{}, Off{}, On{}, Off{}, TGEMM_KIND_TC_Q2);
+  if (fmt == 0 && !lora)
+    return hyb ? run_tc(F0{}, Off{}, Off{}, On{}, TGEMM_KIND_TC_Q2) : run_tc(F0{}, Off{}, Off{}, Off{}, TGEMM_KIND_TC_Q2);
+  if (fmt == 0)
+    return hyb ? run_tc(F0{}, On{}, Off{}, On{}, TGEMM_KIND_TC_Q2_LORA)
+               : run_tc(F0{}, On{}, Off{}, Off{}, TGEMM_KIND_TC_Q2_LORA);
+  return hyb ? run_tc(F1{}, Off{}, Off{}, On{}, TGEMM_KIND_TC_Q4) : run_tc(F1{}, Off{}, Off{}, Off{}, TGEMM_KIND_TC_Q4);
 }
 
 }  // namespace
@@ -653,6 +679,24 @@ size_t tgemm_workspace_size_min(int op, int M, int N, int K, int r) {
   if (op != TGEMM_OP_Q2 && op != TGEMM_OP_Q2_LORA && op != TGEMM_OP_Q4) return 0;
   if (op == TGEMM_OP_Q2_LORA && (r < 1 || r > 256)) return 0;
   return workspace_layout(op, M, N, K, r, choose_path(M), kDefaultSms).total_whole;
+}
+
+int tgemm_tc_plan(int op, int M, int N, int K, int r, int K2, int sms, int* plan) {
+  if (!plan || M < 1 || N < 1 || K < 1 || K2 < 0 || sms < 1) return TGEMM_EINVAL;
+  if (op != TGEMM_OP_Q2 && op != TGEMM_OP_Q2_LORA && op != TGEMM_OP_Q4) return TGEMM_EINVAL;
+  if (op == TGEMM_OP_Q2_LORA && (r < 1 || r > 256)) return TGEMM_EINVAL;
+  if (K2 > 0 && op != TGEMM_OP_Q2) return TGEMM_EINVAL;
+  const int kt_lora = op == TGEMM_OP_Q2_LORA ? lora_dims(r, K).L : 0;
+  const TcSchedule sc = tc_schedule(M, N, K + K2, kt_lora, sms);
+  plan[0] = sc.tiles_m;
+  plan[1] = sc.num_tiles;
+  plan[2] = sc.ksteps;
+  plan[3] = sc.sk_t0;
+  plan[4] = sc.upc;
+  plan[5] = sc.dpc;
+  plan[6] = sc.grid;
+  plan[7] = sc.split ? 1 : 0;
+  return TGEMM_OK;
 }
 
 int tgemm_q2(const uint16_t* x, const uint8_t* wq, const uint16_t* d, void* y, int M, int N,

@@ -144,6 +144,24 @@ size_t tgemm_workspace_size(int op, int M, int N, int K, int r);
 size_t tgemm_workspace_size_min(int op, int M, int N, int K, int r);
 
 /*
+ * tgemm_tc_plan -- the schedule the tensor-core kernel uses for matmul `op` with these
+ * sizes on a device of `sms` SMs, when the workspace has tgemm_workspace_size() bytes
+ * (with only the minimum it keeps whole tiles: plan[3] = 0, plan[5] = 0, plan[7] = 0).
+ * Host computation only; no device is touched.  K2 > 0 adds a second input of width K2
+ * (op must be TGEMM_OP_Q2, as for tgemm_q2_dual); r as for tgemm_workspace_size.
+ * A tile is 128 weight rows x 256 tokens; a unit is one of its 128-k stages (the
+ * low-rank branch adds its own stages).  Tiles and units are numbered tile-major; tile t
+ * covers tokens 256 (t % tiles_m) and rows 128 (t / tiles_m).  CTA c runs the split-region
+ * units sk_t0 * ksteps + [c * upc, (c + 1) * upc) first, then the whole-tile units
+ * [c * dpc, (c + 1) * dpc), both clipped to their region; a tile whose units are spread
+ * over several CTAs is summed from their f32 partial sums in k order.
+ *   plan[8] receives: tiles_m, num_tiles, ksteps, sk_t0, upc, dpc, grid (CTAs launched),
+ *   split (1 when some tile is shared between CTAs).
+ * Returns TGEMM_OK, or TGEMM_EINVAL for a NULL plan, sizes < 1, sms < 1 or an invalid op.
+ */
+int tgemm_tc_plan(int op, int M, int N, int K, int r, int K2, int sms, int* plan);
+
+/*
  * tgemm_q2 -- y = x . W^T for Q2_0 weights.
  *   x [M][K] bf16 (16-byte aligned), wq [N][K/4] (16-byte aligned), d [N][K/128] f16
  *   (2-byte aligned), y [M][N] (16-byte aligned), out_dtype TGEMM_OUT_*.

@@ -12,7 +12,7 @@ import torch
 
 import bit_weight_quantized_tgemm_b200 as tg
 from bit_weight_quantized_tgemm_b200 import synth
-from helpers import canary_intact, dev, gate_output, nan_filled, out_to_f64
+from helpers import canary_intact, dev, gate, gate_output, nan_filled, out_to_f64
 
 pytestmark = pytest.mark.gpu
 
@@ -104,6 +104,125 @@ def test_split_is_deterministic(oracle):
     """Same inputs, three calls in a row (counters re-zeroed each call): identical bits."""
     M, N, K = 256, 1024, 4096
     prob = synth.q2_problem((14, M, N, K), M, N, K)
+    wq, d, st = oracle.q2_pack(prob.codes, prob.scale)
+    x, twq, td = dev(prob.x, torch.bfloat16), dev(wq, torch.uint8), dev(d, torch.float16)
+    ws, _ = _workspaces(tg.OP_Q2, M, N, K)
+    ys = [tg.gemm_q2(x, twq, td, out_dtype=tg.OUT_F32, workspace=ws) for _ in range(3)]
+    torch.cuda.synchronize()
+    for y in ys[1:]:
+        assert torch.equal(y, ys[0])
+    assert tg.device_error() == 0
+
+
+# ---- hybrid form: whole tiles first in the numbering, the remainder split over all CTAs
+def _sms():
+    return torch.cuda.get_device_properties(0).multi_processor_count
+
+
+def _sample(M, N, seed, n=1500):
+    rng = np.random.default_rng(seed)
+    mi = np.concatenate([rng.integers(0, M, n), [0, M - 1, 0, M - 1]]).astype(np.int64)
+    ni = np.concatenate([rng.integers(0, N, n), [0, 0, N - 1, N - 1]]).astype(np.int64)
+    return mi, ni
+
+
+def _check_sampled(outs, ref_at, mi, ni, what):
+    split, whole = outs
+    ref = ref_at(mi, ni)
+    for y, form in ((split, "hybrid"), (whole, "whole tiles")):
+        gate(out_to_f64(y)[mi, ni], ref, f"{what} {form} ({mi.size} sampled outputs)")
+    a, b = out_to_f64(split), out_to_f64(whole)
+    assert np.all(np.isfinite(a)) and np.all(np.isfinite(b))
+    rel = np.linalg.norm(a - b) / np.linalg.norm(b)
+    assert rel < 1e-5, f"{what}: schedules differ by {rel:.2e}"
+
+
+def _hybrid(op, M, N, K, r=0, K2=0):
+    pl = tg.tc_plan(op, M, N, K, r, K2, sms=_sms())
+    assert pl["split"] and pl["dpc"] > 0, f"expected the hybrid form, got {pl}"
+    return pl
+
+
+# tiles: 200 (1 wave + 52), 2 x 130 with a ragged token edge, 360 (the 1280-token QKV)
+@pytest.mark.parametrize("M,N,K", [(256, 25600, 2048), (300, 16640, 3072), (1280, 9216, 3072)])
+def test_q2_hybrid_vs_whole(oracle, M, N, K):
+    _hybrid(tg.OP_Q2, M, N, K)
+    prob = synth.q2_problem((21, M, N, K), M, N, K)
+    wq, d, st = oracle.q2_pack(prob.codes, prob.scale)
+    assert st == 0
+    x, twq, td = dev(prob.x, torch.bfloat16), dev(wq, torch.uint8), dev(d, torch.float16)
+
+    def run(ws, y):
+        tg.gemm_q2(x, twq, td, out_dtype=tg.OUT_F32, y=y, workspace=ws)
+    run.workspaces = _workspaces(tg.OP_Q2, M, N, K)
+    mi, ni = _sample(M, N, 5)
+    _check_sampled(_both(run, M, N), lambda a, b: oracle.q2_gemm_at(prob.x, wq, d, N, a, b),
+                   mi, ni, f"q2 {M}x{N}x{K}")
+
+
+def test_q4_hybrid_vs_whole(oracle):
+    M, N, K = 512, 12800, 2048
+    _hybrid(tg.OP_Q4, M, N, K)
+    prob = synth.q4_problem((22, M, N, K), M, N, K)
+    wq, sz, st = oracle.q4_pack(prob.codes, prob.s, prob.z)
+    assert st == 0
+    x, twq, tsz = dev(prob.x, torch.bfloat16), dev(wq, torch.uint8), dev(sz, torch.float16)
+
+    def run(ws, y):
+        tg.gemm_q4(x, twq, tsz, out_dtype=tg.OUT_F32, y=y, workspace=ws)
+    run.workspaces = _workspaces(tg.OP_Q4, M, N, K)
+    mi, ni = _sample(M, N, 6)
+    _check_sampled(_both(run, M, N), lambda a, b: oracle.q4_gemm_at(prob.x, wq, sz, N, a, b),
+                   mi, ni, f"q4 {M}x{N}x{K}")
+
+
+@pytest.mark.parametrize("r", [4, 32])
+def test_q2_lora_hybrid_vs_whole(oracle, r):
+    M, N, K = 300, 12800, 1152
+    _hybrid(tg.OP_Q2_LORA, M, N, K, r)
+    prob = synth.q2_problem((23, M, N, K, r), M, N, K, r=r)
+    wq, d, st = oracle.q2_pack(prob.codes, prob.scale)
+    assert st == 0
+    x, twq, td = dev(prob.x, torch.bfloat16), dev(wq, torch.uint8), dev(d, torch.float16)
+    a, b = dev(prob.a, torch.bfloat16), dev(prob.b, torch.bfloat16)
+
+    def run(ws, y):
+        tg.gemm_q2_lora(x, twq, td, a, b, out_dtype=tg.OUT_F32, y=y, workspace=ws)
+    run.workspaces = _workspaces(tg.OP_Q2_LORA, M, N, K, r)
+    mi, ni = _sample(M, N, 7)
+    _check_sampled(_both(run, M, N),
+                   lambda i, j: oracle.q2_gemm_at(prob.x, wq, d, N, i, j, prob.a, prob.b),
+                   mi, ni, f"q2+branch r={r} {M}x{N}x{K}")
+
+
+def test_dual_hybrid_vs_whole(oracle):
+    M, N, K1, K2 = 256, 25600, 1024, 1024
+    _hybrid(tg.OP_Q2, M, N, K1, 0, K2)
+    p1 = synth.q2_problem((24, 1), M, N, K1)
+    p2 = synth.q2_problem((24, 2), M, N, K2)
+    wq1, d1, s1 = oracle.q2_pack(p1.codes, p1.scale)
+    wq2, d2, s2 = oracle.q2_pack(p2.codes, p2.scale)
+    assert s1 == 0 and s2 == 0
+    devs = (dev(p1.x, torch.bfloat16), dev(wq1, torch.uint8), dev(d1, torch.float16),
+            dev(p2.x, torch.bfloat16), dev(wq2, torch.uint8), dev(d2, torch.float16))
+    full = tg.dual_workspace_size(M, N, K1, K2)
+    small = tg.dual_workspace_size(M, N, K1, K2, minimum=True)
+    assert full > small > 0
+
+    def run(ws, y):
+        tg.gemm_q2_dual(*devs, out_dtype=tg.OUT_F32, y=y, workspace=ws)
+    run.workspaces = (torch.empty(full, dtype=torch.uint8, device="cuda"),
+                      torch.empty(small, dtype=torch.uint8, device="cuda"))
+    mi, ni = _sample(M, N, 8)
+    _check_sampled(_both(run, M, N),
+                   lambda i, j: oracle.q2_dual_gemm_at(p1.x, wq1, d1, p2.x, wq2, d2, N, i, j),
+                   mi, ni, f"dual {M}x{N}x({K1}+{K2})")
+
+
+def test_hybrid_is_deterministic(oracle):
+    M, N, K = 256, 25600, 2048
+    _hybrid(tg.OP_Q2, M, N, K)
+    prob = synth.q2_problem((25, M, N, K), M, N, K)
     wq, d, st = oracle.q2_pack(prob.codes, prob.scale)
     x, twq, td = dev(prob.x, torch.bfloat16), dev(wq, torch.uint8), dev(d, torch.float16)
     ws, _ = _workspaces(tg.OP_Q2, M, N, K)
