@@ -506,7 +506,7 @@ def ours(args, world, rank, local):
     parts = {}
     if extras:
         for key, fn in (("gemv_stream", gemv_stream), ("dual_out_projection", dual_out_projection),
-                        ("token_sweep", token_sweep)):
+                        ("token_sweep", token_sweep), ("mmdit_sequence", mmdit_sequence)):
             try:
                 parts[key] = fn(tg, torch, stream)
             except Exception as exc:  # report, do not hide
@@ -618,6 +618,58 @@ def token_sweep(tg, torch, stream):
                          device="cuda")
         t = _time_calls(torch, lambda: tg.gemm_q2(x, wq, d, y=y, workspace=ws), reps=10)
         out[f"m{M}"] = {"us": t * 1e6, "tflops": 2 * M * N * K / t / 1e12}
+    return out
+
+
+def mmdit_sequence(tg, torch, stream):
+    """All 81 token-path ternary linears of one MMDiT step (text conditioning projection,
+    5 joint blocks x 2 streams x 4, 20 single blocks x (stacked linear1 + two-input
+    linear2)), captured once in a CUDA graph and replayed, at the pages' token counts:
+    1024 image + 512 text (full size), 1024 + 256, and 256 + 128 (the quarter-size first
+    step). 0.91 GB of distinct packed weights per step, more than L2, so every replay
+    reads them from HBM."""
+    from bit_weight_quantized_tgemm_b200 import mmdit
+    weights = mmdit.make_weights(mmdit.weight_shapes(), seed=11)
+    sustained = load_peaks()["tflops_sustained"]
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+
+    def timed(fn, n):
+        a, b = ev(), ev()
+        a.record()
+        for _ in range(n):
+            fn()
+        b.record()
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) * 1e-3 / n
+
+    out = {}
+    for img, txt, sliced in ((1024, 512, False), (1024, 512, True), (1024, 256, False),
+                             (256, 128, False)):
+        seq = mmdit.StepSequence(mmdit.step_linears(img, txt, slice_rows=sliced), weights)
+        graph = seq.capture(warmup=2)
+        n0 = tg.launch_count()
+        seq.run()
+        torch.cuda.synchronize()
+        launches = tg.launch_count() - n0
+        # graph replays and eager runs alternate, so both see the same (power-capped) clocks
+        clocks = ClockSampler(torch.cuda.current_device())
+        clocks.mark_start()
+        g_t, e_t = [], []
+        for _ in range(3):
+            g_t.append(timed(graph.replay, 8))
+            e_t.append(timed(seq.run, 8))
+        clocks.mark_end()
+        clk = clocks.summary()
+        t, eager = statistics.median(g_t), statistics.median(e_t)
+        key = f"img{img}_txt{txt}" + ("_row_slices" if sliced else "")
+        out[key] = {"linears": len(seq.linears), "launches": launches, "gflop": seq.flops / 1e9,
+                    "us": t * 1e6, "tflops": seq.flops / t / 1e12,
+                    "frac_of_sustained": seq.flops / t / 1e12 / sustained,
+                    "weight_gbs": seq.weight_bytes / t / 1e9, "eager_us": eager * 1e6,
+                    "sm_mhz": clk.get("sm_mhz"), "reasons": clk.get("reasons")}
+        del graph, seq
+    del weights
+    torch.cuda.empty_cache()
     return out
 
 
