@@ -41,6 +41,7 @@ _SIGS = {
     "oracle_f64_to_bf16_array": (None, [_P, _I, _P]),
     "oracle_q2_unpack": (None, [_P, _I, _I, _P]),
     "oracle_q2_pack": (ctypes.c_uint32, [_P, _P, _I, _I, _P, _P]),
+    "oracle_q2_from_gemlite": (ctypes.c_uint32, [_P, _P, _P, _I, _I, _I, _P, _P]),
     "oracle_q2_dequant": (None, [_P, _P, _I, _I, _P]),
     "oracle_q4_unpack": (None, [_P, _I, _I, _P]),
     "oracle_q4_pack": (ctypes.c_uint32, [_P, _P, _P, _I, _I, _P, _P]),
@@ -109,6 +110,21 @@ class Oracle:
         wq = np.empty((N, K // 4), dtype=np.uint8)
         d = np.empty((N, K // 128), dtype=np.uint16)
         st = self.lib.oracle_q2_pack(pc, ps, N, K, wq.ctypes.data_as(_P), d.ctypes.data_as(_P))
+        return wq, d, int(st)
+
+    def q2_from_gemlite(self, wq_g: np.ndarray, scale: np.ndarray, zero: np.ndarray, g: int):
+        """gemlite-int2 (bytes [K/4][N], f32 scale and zero [N][K/g]) -> (wq, d, status)."""
+        wq_g, pw = self._c(wq_g, np.uint8)
+        scale, ps = self._c(scale, np.float32)
+        zero, pz = self._c(zero, np.float32)
+        K = wq_g.shape[0] * 4
+        N = wq_g.shape[1]
+        assert scale.shape == zero.shape == (N, K // g)
+        assert (128 % g == 0 and g % 4 == 0) or (g % 128 == 0 and K % g == 0)
+        wq = np.empty((N, K // 4), dtype=np.uint8)
+        d = np.empty((N, K // 128), dtype=np.uint16)
+        st = self.lib.oracle_q2_from_gemlite(pw, ps, pz, N, K, g, wq.ctypes.data_as(_P),
+                                             d.ctypes.data_as(_P))
         return wq, d, int(st)
 
     def q2_dequant(self, wq, d, N: int, K: int) -> np.ndarray:

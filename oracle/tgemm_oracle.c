@@ -178,6 +178,47 @@ uint32_t oracle_q2_pack(const uint8_t* codes, const float* scale, int64_t N, int
   return status;
 }
 
+uint32_t oracle_q2_from_gemlite(const uint8_t* wq_g, const float* scale, const float* zero,
+                                int64_t N, int64_t K, int64_t g, uint8_t* wq, uint16_t* d) {
+  const int64_t ng = K / g, nb = K / 128;
+  uint8_t* codes = (uint8_t*)malloc((size_t)(N * K));
+  float* bs = (float*)malloc((size_t)(N * nb) * sizeof(float));
+  uint32_t status = 0;
+  /* the transpose: gemlite's byte (k / 4, n) -> codes[n][k] */
+  for (int64_t n = 0; n < N; ++n)
+    for (int64_t k = 0; k < K; ++k) {
+#ifdef ORACLE_PLANT_GEMLITE_NO_TRANSPOSE
+      unsigned byte = wq_g[n * (K / 4) + k / 4];
+#else
+      unsigned byte = wq_g[(k / 4) * N + n];
+#endif
+      codes[n * K + k] = (uint8_t)((byte >> (2 * (k % 4))) & 3u);
+    }
+  /* zeros == -scales, every group */
+#ifndef ORACLE_PLANT_GEMLITE_ZERO_UNCHECKED
+  for (int64_t i = 0; i < N * ng; ++i)
+    if (!(zero[i] == -scale[i])) status |= ORACLE_PACK_ZERO_MISMATCH;
+#endif
+  /* the regroup: block b of row n takes the scale of the groups covering it */
+  for (int64_t n = 0; n < N; ++n)
+    for (int64_t b = 0; b < nb; ++b) {
+      const int64_t k0 = 128 * b, k1 = 128 * b + 128;
+#ifdef ORACLE_PLANT_GEMLITE_GROUP_INDEX
+      const int64_t j0 = b % ng;
+#else
+      const int64_t j0 = k0 / g;
+#endif
+      const float s = scale[n * ng + j0];
+      for (int64_t j = k0 / g; j * g < k1; ++j)
+        if (!(scale[n * ng + j] == s)) status |= ORACLE_PACK_GROUP_MISMATCH;
+      bs[n * nb + b] = s;
+    }
+  status |= oracle_q2_pack(codes, bs, N, K, wq, d);
+  free(codes);
+  free(bs);
+  return status;
+}
+
 void oracle_q2_dequant(const uint8_t* wq, const uint16_t* d, int64_t N, int64_t K, float* w) {
   for (int64_t n = 0; n < N; ++n) {
     for (int64_t k = 0; k < K; ++k) {

@@ -47,6 +47,8 @@ extern "C" {
 #define ORACLE_PACK_BAD_CODE  1u
 #define ORACLE_PACK_INEXACT   2u
 #define ORACLE_PACK_NONFINITE 4u
+#define ORACLE_PACK_ZERO_MISMATCH  8u   /* gemlite import: zero != -scale */
+#define ORACLE_PACK_GROUP_MISMATCH 16u  /* gemlite import: groups of one 128-block differ */
 
 /* IEEE 754 binary16 and bfloat16, converted bit by bit (round to nearest, ties to even). */
 float    oracle_f16_to_f32(uint16_t h);
@@ -61,6 +63,17 @@ void     oracle_q2_unpack(const uint8_t* wq, int64_t N, int64_t K, uint8_t* code
 uint32_t oracle_q2_pack(const uint8_t* codes, const float* scale, int64_t N, int64_t K,
                         uint8_t* wq, uint16_t* d);
 void     oracle_q2_dequant(const uint8_t* wq, const uint16_t* d, int64_t N, int64_t K, float* w);
+
+/* gemlite-int2 -> Q2_0 [P2-LB]: the pages give gemlite's codes ({0,1,2}, LSB-first, four
+ * per byte along the input axis), its dequant ((q - zero) * scale with zeros == -scales,
+ * i.e. (q - 1) * scale) and the conversion ("a transpose and regroup", scales f32 -> f16
+ * with an exact roundtrip).  Layout reading: wq_g[K/4][N] bytes, byte (i, n) holding the
+ * codes of k = 4i..4i+3 of output row n; scale and zero f32 [N][K/g], group j covering
+ * k in [j g, (j + 1) g).  Q2_0 block b takes the scale of the groups covering
+ * [128 b, 128 b + 128), which must all be equal.  g divides 128, or is a multiple of 128
+ * dividing K.  Returns the Q2 pack status plus the two import bits above. */
+uint32_t oracle_q2_from_gemlite(const uint8_t* wq_g, const float* scale, const float* zero,
+                                int64_t N, int64_t K, int64_t g, uint8_t* wq, uint16_t* d);
 
 /* 4-bit group format [P3-FB], [P2-WL] */
 void     oracle_q4_unpack(const uint8_t* wq, int64_t N, int64_t K, uint8_t* codes);

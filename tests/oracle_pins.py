@@ -264,6 +264,92 @@ def pin_pack_status(o):
     assert st == 2
 
 
+# ---- gemlite-int2 import ----------------------------------------------------------------
+
+def _gemlite_from_rows(rows):
+    N, K = 2, 128
+    wq_g = np.full((K // 4, N), 0x55, dtype=np.uint8)
+    scale = np.zeros((N, 1), np.float32)
+    zero = np.zeros((N, 1), np.float32)
+    d_want = np.zeros((N, 1), np.uint16)
+    w_want = []
+    for r in rows:
+        if r[0] == "byte":
+            wq_g[int(r[1]), int(r[2])] = int(r[3], 16)
+        elif r[0] == "scale":
+            n = int(r[1])
+            scale[n, 0], zero[n, 0], d_want[n, 0] = float(r[2]), float(r[3]), int(r[4], 16)
+        elif r[0] == "w":
+            w_want.append((int(r[1]), int(r[2]), float(r[3])))
+    return wq_g, scale, zero, d_want, w_want
+
+
+def pin_gemlite_hand_example(o):
+    """A hand-worked import: each gemlite byte (i, n) becomes Q2_0 byte (n, i) unchanged,
+    the scales become f16 d, and the dequantized weights are the hand-computed ones."""
+    wq_g, scale, zero, d_want, w_want = _gemlite_from_rows(_rows("gemlite_small.txt"))
+    wq, d, st = o.q2_from_gemlite(wq_g, scale, zero, 128)
+    assert st == 0, st
+    assert np.array_equal(wq, wq_g.T), "the import is a transpose of the packed bytes"
+    assert np.array_equal(d, d_want)
+    w = o.q2_dequant(wq, d, 2, 128)
+    for n, k, v in w_want:
+        assert w[n, k] == v, (n, k, w[n, k], v)
+
+
+def _gemlite_random(rng, N, K, g):
+    codes = rng.integers(0, 3, size=(N, K), dtype=np.uint8)
+    # gemlite bytes [K/4][N]: byte (i, n) = sum_j codes[n][4i + j] << 2j
+    c = codes.T.reshape(K // 4, 4, N).astype(np.uint32)
+    wq_g = (c[:, 0] | (c[:, 1] << 2) | (c[:, 2] << 4) | (c[:, 3] << 6)).astype(np.uint8)
+    per_block = np.abs(rng.standard_normal((N, K // 128))).astype(np.float16).astype(np.float32)
+    if g <= 128:
+        scale = np.repeat(per_block, 128 // g, axis=1)  # groups inside a block agree
+    else:
+        scale = np.abs(rng.standard_normal((N, K // g))).astype(np.float16).astype(np.float32)
+    return codes, wq_g, scale, -scale
+
+
+def pin_gemlite_dequant_definition(o):
+    """For every group size, Q2_0 dequant of the import equals gemlite's own definition
+    q * scale + zero evaluated from the gemlite bytes (exactly: both are one f32 product)."""
+    rng = np.random.default_rng(90)
+    N, K = 6, 1024
+    for g in (32, 64, 128, 256, 512, 1024):
+        codes, wq_g, scale, zero = _gemlite_random(rng, N, K, g)
+        wq, d, st = o.q2_from_gemlite(wq_g, scale, zero, g)
+        assert st == 0, (g, st)
+        # gemlite's dequant, from its bytes: the code of (n, k) is in byte (k / 4, n)
+        k = np.arange(K)
+        q = (wq_g[k // 4, :] >> (2 * (k % 4))[:, None]) & 3          # [K][N]
+        w_g = q.T.astype(np.float32) * np.repeat(scale, g, axis=1) + np.repeat(zero, g, axis=1)
+        assert np.array_equal(q.T, codes)
+        assert np.array_equal(o.q2_dequant(wq, d, N, K), w_g), g
+
+
+def pin_gemlite_status(o):
+    """zero != -scale, disagreeing groups in one block, a code 3 and an inexact f16 scale
+    are each reported; a clean import reports nothing."""
+    rng = np.random.default_rng(91)
+    N, K = 3, 256
+    codes, wq_g, scale, zero = _gemlite_random(rng, N, K, 64)
+    assert o.q2_from_gemlite(wq_g, scale, zero, 64)[2] == 0
+    z = zero.copy()
+    z[1, 2] = -z[1, 2]
+    if z[1, 2] == zero[1, 2]:
+        z[1, 2] = 1.0
+    assert o.q2_from_gemlite(wq_g, scale, z, 64)[2] == 8
+    s = scale.copy()
+    s[2, 1] = s[2, 0] * 2  # groups 0 and 1 form block 0 of row 2
+    assert o.q2_from_gemlite(wq_g, s, -s, 64)[2] == 16
+    bad = wq_g.copy()
+    bad[5, 1] |= 0x0C  # code 3 at k = 21 of row 1
+    assert o.q2_from_gemlite(bad, scale, zero, 64)[2] == 1
+    s = scale.copy()
+    s[0, :2] = np.float32(0.02)  # not an f16 value
+    assert o.q2_from_gemlite(wq_g, s, -s, 64)[2] == 2
+
+
 # ---- matmul: closed forms and brute force ---------------------------------------------
 
 def _rand_x(rng, M, K, scale=1.0):

@@ -20,6 +20,9 @@ PLANTS = [
     "ORACLE_PLANT_GEMM_TRANSPOSED",   # transposed weight operand
     "ORACLE_PLANT_LORA_DROPPED",      # side branch missing
     "ORACLE_PLANT_DUAL_SECOND_DROPPED",  # split projection: second product missing
+    "ORACLE_PLANT_GEMLITE_NO_TRANSPOSE",  # gemlite bytes read as [N][K/4]
+    "ORACLE_PLANT_GEMLITE_ZERO_UNCHECKED",  # zeros == -scales not checked
+    "ORACLE_PLANT_GEMLITE_GROUP_INDEX",  # block b takes group b mod (K/g)
 ]
 
 
