@@ -23,6 +23,7 @@ OUT_F32, OUT_BF16 = 0, 1
 OP_Q2, OP_Q2_LORA, OP_Q4 = 0, 1, 2
 PATH_AUTO, PATH_SMALL_M, PATH_TENSOR = 0, 1, 2
 PACK_BAD_CODE, PACK_INEXACT, PACK_NONFINITE = 1, 2, 4
+PACK_ZERO_MISMATCH, PACK_GROUP_MISMATCH = 8, 16
 DEVERR_TIMEOUT = 1
 KIND_TC_Q2, KIND_TC_Q2_LORA, KIND_TC_Q4, KIND_GEMV_Q2, KIND_GEMV_Q4, KIND_PREP = range(6)
 
@@ -33,6 +34,7 @@ _sz = ctypes.c_size_t
 _SIGS = {
     "q2_pack": (_i, [_P, _P, _P, _P, _i, _i, _P, _P]),
     "q4_pack": (_i, [_P, _P, _P, _P, _P, _i, _i, _P, _P]),
+    "q2_from_gemlite": (_i, [_P, _P, _P, _i, _i, _i, _P, _P, _P, _P]),
     "q2_dequant": (_i, [_P, _P, _P, _i, _i, _P]),
     "q4_dequant": (_i, [_P, _P, _P, _i, _i, _P]),
     "tgemm_workspace_size": (_sz, [_i, _i, _i, _i, _i]),
@@ -42,6 +44,7 @@ _SIGS = {
     "tgemm_tc_plan": (_i, [_i, _i, _i, _i, _i, _i, _i, _P]),
     "tgemm_q2": (_i, [_P, _P, _P, _P, _i, _i, _i, _i, _P, _sz, _P]),
     "tgemm_q2_lora": (_i, [_P, _P, _P, _P, _P, _i, _P, _i, _i, _i, _i, _P, _sz, _P]),
+    "tgemm_q2_lora_bt": (_i, [_P, _P, _P, _P, _P, _i, _P, _i, _i, _i, _i, _P, _sz, _P]),
     "tgemm_q4": (_i, [_P, _P, _P, _P, _i, _i, _i, _i, _P, _sz, _P]),
     "tgemm_q2_dual": (_i, [_P, _P, _P, _i, _P, _P, _P, _i, _P, _i, _i, _i, _P, _sz, _P]),
     "tgemm_q2_noalloc": (_i, [_P, _P, _P, _P, _i, _i, _i, _i, _P]),
@@ -128,6 +131,26 @@ def q2_pack(codes: torch.Tensor, scale: torch.Tensor, status: Optional[torch.Ten
         status = torch.zeros(1, dtype=torch.int32, device=codes.device)
     _check(lib().q2_pack(_ptr(codes), _ptr(scale), _ptr(wq), _ptr(d), N, K, _ptr(status),
                          _stream()), "q2_pack")
+    return wq, d, status
+
+
+def q2_from_gemlite(wq_g: torch.Tensor, scale: torch.Tensor, zero: torch.Tensor, g: int,
+                    status: Optional[torch.Tensor] = None):
+    """gemlite-int2 bytes uint8 [K/4, N], f32 scale and zero [N, K/g] -> Q2_0
+    (wq uint8 [N, K/4], d f16 [N, K/128], status); see q2_from_gemlite in tgemm.h."""
+    _need(wq_g, torch.uint8, "wq_g")
+    _need(scale, torch.float32, "scale")
+    _need(zero, torch.float32, "zero")
+    K4, N = wq_g.shape
+    K = 4 * K4
+    if g < 1 or K % g or tuple(scale.shape) != (N, K // g) or tuple(zero.shape) != (N, K // g):
+        raise ValueError("scale and zero must be [N, K/g]")
+    wq = torch.empty((N, K4), dtype=torch.uint8, device=wq_g.device)
+    d = torch.empty((N, K // 128), dtype=torch.float16, device=wq_g.device)
+    if status is None:
+        status = torch.zeros(1, dtype=torch.int32, device=wq_g.device)
+    _check(lib().q2_from_gemlite(_ptr(wq_g), _ptr(scale), _ptr(zero), N, K, g, _ptr(wq), _ptr(d),
+                                 _ptr(status), _stream()), "q2_from_gemlite")
     return wq, d, status
 
 
@@ -256,10 +279,31 @@ def gemm_q2_lora(x, wq, d, a, b, *, out_dtype: int = OUT_BF16, y=None, workspace
     M, K = x.shape
     N = wq.shape[0]
     r = a.shape[0]
+    if tuple(a.shape) != (r, K) or tuple(b.shape) != (N, r):
+        raise ValueError(f"a must be [r, K] and b [N, r]; got {tuple(a.shape)}, {tuple(b.shape)}")
     y = _out(y, M, N, out_dtype, x.device)
     ws, nbytes = _workspace(OP_Q2_LORA, M, N, K, r, x.device, workspace)
     _check(lib().tgemm_q2_lora(_ptr(x), _ptr(wq), _ptr(d), _ptr(a), _ptr(b), r, _ptr(y), M, N,
                                K, out_dtype, _ptr(ws), nbytes, _stream()), "tgemm_q2_lora")
+    return y
+
+
+def gemm_q2_lora_bt(x, wq, d, a, bt, *, out_dtype: int = OUT_BF16, y=None, workspace=None):
+    """gemm_q2_lora with B given transposed: bt bf16 [r, N] (see tgemm_q2_lora_bt)."""
+    _need(x, torch.bfloat16, "x")
+    _need(wq, torch.uint8, "wq")
+    _need(d, torch.float16, "d")
+    _need(a, torch.bfloat16, "a")
+    _need(bt, torch.bfloat16, "bt")
+    M, K = x.shape
+    N = wq.shape[0]
+    r = a.shape[0]
+    if tuple(a.shape) != (r, K) or tuple(bt.shape) != (r, N):
+        raise ValueError(f"a must be [r, K] and bt [r, N]; got {tuple(a.shape)}, {tuple(bt.shape)}")
+    y = _out(y, M, N, out_dtype, x.device)
+    ws, nbytes = _workspace(OP_Q2_LORA, M, N, K, r, x.device, workspace)
+    _check(lib().tgemm_q2_lora_bt(_ptr(x), _ptr(wq), _ptr(d), _ptr(a), _ptr(bt), r, _ptr(y), M,
+                                  N, K, out_dtype, _ptr(ws), nbytes, _stream()), "tgemm_q2_lora_bt")
     return y
 
 

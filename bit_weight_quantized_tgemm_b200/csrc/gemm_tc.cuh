@@ -129,12 +129,13 @@ struct TcParams {
   const uint8_t* wq;       // packed codes [N][K/4] (Q2) or [N][K/2] (4-bit)
   const uint16_t* scales;  // Q2: d [N][K/128]; 4-bit: sz [N][K/64][2]
   const uint16_t* scales2; // the second input's scales (two inputs only)
-  const uint16_t* lb;      // low-rank B [N][r] (bf16)
+  const uint16_t* lb;      // low-rank B (bf16): element (n, i) at lb[n * lb_sn + i * lb_si]
   void* y;
   float* part;             // split tiles: 2 slots of 128 x 256 f32 per CTA
   int* cnt;                // split region: 8 arrival counters per tile, zero at launch
   int sk_t0;               // first tile of the split region (tiles before it are whole per CTA)
   int dpc;                 // whole-tile region: CTA c owns units [c * dpc, (c + 1) * dpc) (0: none)
+  int lb_sn, lb_si;        // B's element strides: (r, 1) for B [N][r], (1, N) for B^T [r][N]
 };
 
 // One tile's share of a CTA's unit range [u, u1): tile `tile`, stages [ka, kb).
@@ -457,14 +458,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       } else {
         // low-rank stage: weight-side values [j0, j0 + kC) of [B | B], zero beyond 2R
         const int j0 = (ks - p.kt_main) * kTcBK + part * kC;
-        const bool vec = (p.r & 7) == 0 && (reinterpret_cast<uintptr_t>(p.lb) & 15) == 0;
+        const bool vec = p.lb_si == 1 && (p.lb_sn & 7) == 0 &&
+                         (reinterpret_cast<uintptr_t>(p.lb) & 15) == 0;
 #pragma unroll
         for (int cq = 0; cq < kC / 8; ++cq) {
           const int jc = j0 + 8 * cq;
           const int ic = jc < p.R ? jc : jc - p.R;
           if (vec && jc < 2 * p.R && ic + 8 <= p.r) {
             uint4 v = make_uint4(0, 0, 0, 0);
-            if (valid) v = *reinterpret_cast<const uint4*>(p.lb + static_cast<int64_t>(row) * p.r + ic);
+            if (valid) v = *reinterpret_cast<const uint4*>(p.lb + static_cast<int64_t>(row) * p.lb_sn + ic);
             o[4 * cq] = v.x;
             o[4 * cq + 1] = v.y;
             o[4 * cq + 2] = v.z;
@@ -479,7 +481,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
               const int j = jc + 2 * e + h;
               const int ii = j < p.R ? j : j - p.R;
               uint32_t v = 0;
-              if (valid && j < 2 * p.R && ii < p.r) v = p.lb[static_cast<int64_t>(row) * p.r + ii];
+              if (valid && j < 2 * p.R && ii < p.r)
+                v = p.lb[static_cast<int64_t>(row) * p.lb_sn + static_cast<int64_t>(ii) * p.lb_si];
               v2 |= v << (16 * h);
             }
             o[4 * cq + e] = v2;

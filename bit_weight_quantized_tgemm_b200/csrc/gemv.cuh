@@ -108,7 +108,8 @@ template <int FMT, bool LORA, bool DUAL>
 __global__ void __launch_bounds__(256) gemv_kernel(
     const uint16_t* __restrict__ x, const uint8_t* __restrict__ wq,
     const uint16_t* __restrict__ scales, void* __restrict__ y, int M, int N, int K, int out_f32,
-    const float* __restrict__ u, const uint16_t* __restrict__ lb, int r, int mrows, int kp,
+    const float* __restrict__ u, const uint16_t* __restrict__ lb, int r, int lb_sn, int lb_si,
+    int mrows, int kp,
     const uint16_t* __restrict__ x2, const uint8_t* __restrict__ wq2,
     const uint16_t* __restrict__ scales2, int K2) {
   extern __shared__ __align__(16) uint8_t gv_smem[];
@@ -328,7 +329,8 @@ __global__ void __launch_bounds__(256) gemv_kernel(
       if (LORA) {
         float br = 0.f;
         for (int i = 0; i < r; ++i)
-          br = fmaf(bf16_bits_to_f32(lb[static_cast<int64_t>(n) * r + i]), u[static_cast<int64_t>(m) * r + i], br);
+          br = fmaf(bf16_bits_to_f32(lb[static_cast<int64_t>(n) * lb_sn + static_cast<int64_t>(i) * lb_si]),
+                    u[static_cast<int64_t>(m) * r + i], br);
         v += br;
       }
       if (out_f32)

@@ -15,6 +15,8 @@ namespace tgemm {
 constexpr uint32_t kPackBadCode = 1u;
 constexpr uint32_t kPackInexact = 2u;
 constexpr uint32_t kPackNonFinite = 4u;
+constexpr uint32_t kPackZeroMismatch = 8u;
+constexpr uint32_t kPackGroupMismatch = 16u;
 
 // OR `bits` into *status once per warp (only lanes with something to report take part).
 __device__ __forceinline__ void report_status(uint32_t* status, uint32_t bits) {
@@ -69,6 +71,79 @@ __global__ void __launch_bounds__(256) q2_pack_kernel(const uint8_t* __restrict_
     }
     if (u < n_scales) d[u] = scale_to_f16(scale[u], flags);
     report_status(status, flags);
+  }
+}
+
+// gemlite-int2 -> Q2_0 ("We're Teaching Your Browser to Paint...", section "The lucky
+// break that wasn't luck": same codes, same bit order, dequant (q - zero) * scale with
+// zeros == -scales, so the conversion is a transpose and regroup).  The gemlite bytes are
+// [K/4][N] (byte (i, n): codes of k = 4i..4i+3 of row n), so byte (i, n) moves unchanged
+// to wq[n][i].  Each CTA transposes one tile of 32 byte-rows x 128 rows n through shared
+// memory; then all threads regroup the f32 scales [N][K/g] into f16 block scales, checking
+// zero == -scale for every group and that the groups of one 128-block agree.
+constexpr int kGlTileI = 32;   // gemlite byte-rows (4 k each) per tile
+constexpr int kGlTileN = 128;  // output rows per tile
+
+__global__ void __launch_bounds__(256) q2_from_gemlite_kernel(
+    const uint8_t* __restrict__ wq_g, const float* __restrict__ scale,
+    const float* __restrict__ zero, uint8_t* __restrict__ wq, uint16_t* __restrict__ d, int N,
+    int K, int g, int tiles_n, uint32_t* status) {
+  __shared__ uint8_t tile[kGlTileI][kGlTileN + 4];
+  pdl_trigger_and_wait();
+  const int kq = K / 4;
+  const int i0 = (static_cast<int>(blockIdx.x) / tiles_n) * kGlTileI;
+  const int n0 = (static_cast<int>(blockIdx.x) % tiles_n) * kGlTileN;
+  uint32_t flags = 0;
+  // load: 32 byte-rows x 128 bytes along n (lanes read consecutive n)
+#pragma unroll
+  for (int r = 0; r < kGlTileI * kGlTileN / 256; ++r) {
+    const int idx = r * 256 + static_cast<int>(threadIdx.x);
+    const int ii = idx / kGlTileN, nn = idx % kGlTileN;
+    uint32_t byte = 0x55u;  // rows past N: four codes 1, never stored
+    if (n0 + nn < N) {
+      byte = __ldg(wq_g + static_cast<int64_t>(i0 + ii) * N + n0 + nn);
+      if (byte & (byte >> 1) & 0x55u) flags |= kPackBadCode;  // a 2-bit field equal to 3
+    }
+    tile[ii][nn] = static_cast<uint8_t>(byte);
+  }
+  __syncthreads();
+  // store: row n0 + nn gets bytes [i0, i0 + 32) as eight 4-byte words
+#pragma unroll
+  for (int r = 0; r < kGlTileI * kGlTileN / 4 / 256; ++r) {
+    const int w = r * 256 + static_cast<int>(threadIdx.x);
+    const int nn = w / (kGlTileI / 4), wi = w % (kGlTileI / 4);
+    if (n0 + nn < N) {
+      const uint32_t word = static_cast<uint32_t>(tile[4 * wi][nn]) |
+                            (static_cast<uint32_t>(tile[4 * wi + 1][nn]) << 8) |
+                            (static_cast<uint32_t>(tile[4 * wi + 2][nn]) << 16) |
+                            (static_cast<uint32_t>(tile[4 * wi + 3][nn]) << 24);
+      *reinterpret_cast<uint32_t*>(wq + static_cast<int64_t>(n0 + nn) * kq + i0 + 4 * wi) = word;
+    }
+  }
+  report_status(status, flags);
+  // regroup the scales: block b of row n takes the scale of the groups covering it
+  const int nb = K / 128, ng = K / g;
+  const int64_t n_blocks = static_cast<int64_t>(N) * nb;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  const int64_t tid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  for (int64_t base = 0; base < n_blocks; base += stride) {
+    const int64_t u = base + tid;
+    uint32_t f = 0;
+    if (u < n_blocks) {
+      const int64_t n = u / nb;
+      const int b = static_cast<int>(u - n * nb);
+      const float* srow = scale + n * ng;
+      const float* zrow = zero + n * ng;
+      const int j0 = 128 * b / g;
+      const float sv = __ldg(srow + j0);
+      for (int j = j0; j * g < 128 * b + 128; ++j) {
+        const float sj = __ldg(srow + j);
+        if (!(sj == sv)) f |= kPackGroupMismatch;
+        if (!(__ldg(zrow + j) == -sj)) f |= kPackZeroMismatch;
+      }
+      d[u] = scale_to_f16(sv, f);
+    }
+    report_status(status, f);
   }
 }
 

@@ -367,10 +367,11 @@ struct SecondInput {
   int K = 0;
 };
 
+// lb_t: the branch's B is given transposed, [r][N] instead of [N][r].
 int run_gemm(int fmt, const uint16_t* x, const uint8_t* wq, const uint16_t* scales,
              const uint16_t* la, const uint16_t* lb, int r, void* y, int M, int N, int K,
              int out_dtype, void* workspace, size_t ws_bytes, void* stream,
-             const SecondInput& in2 = SecondInput()) {
+             const SecondInput& in2 = SecondInput(), bool lb_t = false) {
   const bool lora = la != nullptr;
   const bool dual = in2.K > 0;
   const int K2 = in2.K;
@@ -387,6 +388,7 @@ int run_gemm(int fmt, const uint16_t* x, const uint8_t* wq, const uint16_t* scal
     if (fmt != 0 || lora || !in2.x || !in2.wq || !in2.d || K2 < 128 || K2 % 128) return TGEMM_EINVAL;
     if (!aligned(in2.x, 16) || !aligned(in2.wq, 16) || !aligned(in2.d, 2)) return TGEMM_EALIGN;
   }
+  const int lb_sn = lb_t ? 1 : r, lb_si = lb_t ? N : 1;  // B's element strides
   const int path = choose_path(M);
   // the required size does not depend on the device (only the optional split-tile part does)
   const size_t required = workspace_layout(op, M, N, K, r, path, kDefaultSms, K2).total_whole;
@@ -418,28 +420,28 @@ int run_gemm(int fmt, const uint16_t* x, const uint8_t* wq, const uint16_t* scal
     if (fmt == 0 && lora) {
       if (int e = gemv_prepare<0, true>()) return e;
       return launch(TGEMM_KIND_GEMV_Q2, st, [&] {
-        return pdl_launch(gemv_kernel<0, true, false>, grid, 256, smem, st, x, wq, scales, y, M, N, K, out_f32, u32, lb, r, mrows, kp,
+        return pdl_launch(gemv_kernel<0, true, false>, grid, 256, smem, st, x, wq, scales, y, M, N, K, out_f32, u32, lb, r, lb_sn, lb_si, mrows, kp,
                           nullptr, nullptr, nullptr, 0);
       });
     }
     if (fmt == 0 && dual) {
       if (int e = gemv_prepare<0, false, true>()) return e;
       return launch(TGEMM_KIND_GEMV_Q2, st, [&] {
-        return pdl_launch(gemv_kernel<0, false, true>, grid, 256, smem, st, x, wq, scales, y, M, N, K, out_f32, nullptr, nullptr, 0, mrows, kp,
+        return pdl_launch(gemv_kernel<0, false, true>, grid, 256, smem, st, x, wq, scales, y, M, N, K, out_f32, nullptr, nullptr, 0, 0, 0, mrows, kp,
                           in2.x, in2.wq, in2.d, K2);
       });
     }
     if (fmt == 0) {
       if (int e = gemv_prepare<0, false>()) return e;
       return launch(TGEMM_KIND_GEMV_Q2, st, [&] {
-        return pdl_launch(gemv_kernel<0, false, false>, grid, 256, smem, st, x, wq, scales, y, M, N, K, out_f32, nullptr, nullptr, 0, mrows, kp,
+        return pdl_launch(gemv_kernel<0, false, false>, grid, 256, smem, st, x, wq, scales, y, M, N, K, out_f32, nullptr, nullptr, 0, 0, 0, mrows, kp,
                           static_cast<const uint16_t*>(nullptr), static_cast<const uint8_t*>(nullptr),
                           static_cast<const uint16_t*>(nullptr), 0);
       });
     }
     if (int e = gemv_prepare<1, false>()) return e;
     return launch(TGEMM_KIND_GEMV_Q4, st, [&] {
-      return pdl_launch(gemv_kernel<1, false, false>, grid, 256, smem, st, x, wq, scales, y, M, N, K, out_f32, nullptr, nullptr, 0, mrows, kp,
+      return pdl_launch(gemv_kernel<1, false, false>, grid, 256, smem, st, x, wq, scales, y, M, N, K, out_f32, nullptr, nullptr, 0, 0, 0, mrows, kp,
                         nullptr, nullptr, nullptr, 0);
     });
   }
@@ -544,6 +546,8 @@ int run_gemm(int fmt, const uint16_t* x, const uint8_t* wq, const uint16_t* scal
   p.wq = wq;
   p.scales = scales;
   p.lb = lb;
+  p.lb_sn = lb_sn;
+  p.lb_si = lb_si;
   p.y = y;
   p.part = sc.split ? reinterpret_cast<float*>(ws + wl.slots) : nullptr;
   p.cnt = cnt;
@@ -621,6 +625,28 @@ int q2_pack(const uint8_t* codes, const float* scale, uint8_t* wq, uint16_t* d, 
   const cudaStream_t st = as_stream(stream);
   return launch(TGEMM_KIND_PREP, st, [&] {
     return pdl_launch(q2_pack_kernel, grid_for(units, 256, di.sms), 256, 0, st, codes, scale, wq, d, units, scales, status);
+  });
+}
+
+int q2_from_gemlite(const uint8_t* wq_g, const float* scale, const float* zero, int N, int K,
+                    int g, uint8_t* wq, uint16_t* d, uint32_t* status, void* stream) {
+  if (!wq_g || !scale || !zero || !wq || !d || !status) return TGEMM_EINVAL;
+  if (N < 1 || K < 128 || K % 128 || g < 4) return TGEMM_EINVAL;
+  const bool small_groups = 128 % g == 0 && g % 4 == 0;
+  const bool large_groups = g % 128 == 0 && K % g == 0;
+  if (!small_groups && !large_groups) return TGEMM_EINVAL;
+  if (!aligned(wq, 16) || !aligned(scale, 4) || !aligned(zero, 4) || !aligned(d, 2) ||
+      !aligned(status, 4))
+    return TGEMM_EALIGN;
+  DeviceInfo di;
+  if (int st = current_device_info(&di)) return st;
+  const int tiles_n = (N + kGlTileN - 1) / kGlTileN;
+  const int64_t tiles = static_cast<int64_t>(K / 4 / kGlTileI) * tiles_n;
+  if (tiles > 0x7FFFFFFF) return TGEMM_ETOOLARGE;
+  const cudaStream_t st = as_stream(stream);
+  return launch(TGEMM_KIND_PREP, st, [&] {
+    return pdl_launch(q2_from_gemlite_kernel, static_cast<int>(tiles), 256, 0, st, wq_g, scale, zero,
+                      wq, d, N, K, g, tiles_n, status);
   });
 }
 
@@ -710,6 +736,14 @@ int tgemm_q2_lora(const uint16_t* x, const uint8_t* wq, const uint16_t* d, const
                   void* workspace, size_t ws_bytes, void* stream) {
   if (!a) return TGEMM_EINVAL;
   return run_gemm(0, x, wq, d, a, b, r, y, M, N, K, out_dtype, workspace, ws_bytes, stream);
+}
+
+int tgemm_q2_lora_bt(const uint16_t* x, const uint8_t* wq, const uint16_t* d, const uint16_t* a,
+                     const uint16_t* bt, int r, void* y, int M, int N, int K, int out_dtype,
+                     void* workspace, size_t ws_bytes, void* stream) {
+  if (!a) return TGEMM_EINVAL;
+  return run_gemm(0, x, wq, d, a, bt, r, y, M, N, K, out_dtype, workspace, ws_bytes, stream,
+                  SecondInput(), true);
 }
 
 int tgemm_q2_noalloc(const uint16_t* x, const uint8_t* wq, const uint16_t* d, void* y, int M,

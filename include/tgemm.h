@@ -73,6 +73,8 @@ extern "C" {
 #define TGEMM_PACK_BAD_CODE  1u /* a Q2 code > 2 or a 4-bit code > 15 (stored masked) */
 #define TGEMM_PACK_INEXACT   2u /* a scale/zero is not exactly representable in f16 */
 #define TGEMM_PACK_NONFINITE 4u /* a scale/zero is inf or NaN */
+#define TGEMM_PACK_ZERO_MISMATCH  8u  /* q2_from_gemlite: some zero != -scale */
+#define TGEMM_PACK_GROUP_MISMATCH 16u /* q2_from_gemlite: groups of one 128-block differ */
 
 /* ---- device error word bits (tgemm_device_error) ----------------------------------- */
 #define TGEMM_DEVERR_TIMEOUT 1u /* a pipeline wait in a matmul kernel ran out of time */
@@ -101,6 +103,27 @@ extern "C" {
  */
 int q2_pack(const uint8_t* codes, const float* scale, uint8_t* wq, uint16_t* d, int N, int K,
             uint32_t* status, void* stream);
+
+/*
+ * q2_from_gemlite -- import a gemlite-int2 matrix as Q2_0, on the device ("We're Teaching
+ * Your Browser to Paint...", "The lucky break that wasn't luck": gemlite's codes are
+ * {0,1,2}, LSB-first, four per byte along the input axis, dequantized as
+ * (q - zero) * scale with zeros == -scales, so the conversion is a transpose and regroup
+ * with no numeric change; the scale's f32 -> f16 rounding must be exact).
+ *   wq_g   uint8 [K/4][N]: byte (i, n) holds the codes of k = 4i..4i+3 of output row n
+ *          (the input axis is the outer one; this layout is a reading, the pages do not
+ *          print it)                                   (any alignment)
+ *   scale, zero  f32 [N][K/g]: group j of a row covers k in [j g, (j + 1) g)  (4-byte aligned)
+ *   wq, d  Q2_0 out, as from q2_pack: byte (i, n) of wq_g becomes wq[n][i] unchanged, and
+ *          block b of row n gets the f16 of the scale of the groups covering
+ *          [128 b, 128 b + 128)                       (16- and 2-byte aligned)
+ *   status as for q2_pack, plus ZERO_MISMATCH (a zero that is not -scale) and
+ *          GROUP_MISMATCH (g < 128 and the groups of one block have different scales).
+ *   Requires N >= 1, K % 128 == 0, and g a multiple of 4 dividing 128 or a multiple of
+ *   128 dividing K.  Load-time work.
+ */
+int q2_from_gemlite(const uint8_t* wq_g, const float* scale, const float* zero, int N, int K,
+                    int g, uint8_t* wq, uint16_t* d, uint32_t* status, void* stream);
 
 /*
  * q4_pack -- 4-bit packing ("You Can Now Just Ask...", "The bug that hid in one flipped bit").
@@ -184,6 +207,17 @@ int tgemm_q2(const uint16_t* x, const uint8_t* wq, const uint16_t* d, void* y, i
 int tgemm_q2_lora(const uint16_t* x, const uint8_t* wq, const uint16_t* d, const uint16_t* a,
                   const uint16_t* b, int r, void* y, int M, int N, int K, int out_dtype,
                   void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * tgemm_q2_lora_bt -- tgemm_q2_lora with B given transposed: bt [r][N] bf16 (2-byte
+ * aligned), element (i, n) = B[n][i].  The branches in the model file are stored as
+ * <branch>.<matrix>.a and <branch>.<matrix>.bt ("mindview-t2i-turbo", "Running it"),
+ * so they load without a transpose.  The same workspace as tgemm_q2_lora; the
+ * result is bit-identical to tgemm_q2_lora on the transposed copy.
+ */
+int tgemm_q2_lora_bt(const uint16_t* x, const uint8_t* wq, const uint16_t* d, const uint16_t* a,
+                     const uint16_t* bt, int r, void* y, int M, int N, int K, int out_dtype,
+                     void* workspace, size_t ws_bytes, void* stream);
 
 /*
  * tgemm_q2_noalloc -- tgemm_q2 for callers that cannot allocate device memory.

@@ -103,6 +103,14 @@ P = ctypes.c_void_p
     lambda L: L.q2_pack(P(16), P(16), P(16), P(16), 4, 64, P(16), None),
     lambda L: L.q4_pack(P(16), P(16), P(16), P(16), P(16), 4, 32, P(16), None),
     lambda L: L.q2_dequant(None, P(16), P(16), 4, 128, None),
+    # gemlite import: K not a multiple of 128, g neither dividing 128 nor a multiple of
+    # 128 dividing K, g below 4, no rows, a missing pointer
+    lambda L: L.q2_from_gemlite(P(16), P(16), P(16), 4, 96, 32, P(16), P(16), P(16), None),
+    lambda L: L.q2_from_gemlite(P(16), P(16), P(16), 4, 256, 48, P(16), P(16), P(16), None),
+    lambda L: L.q2_from_gemlite(P(16), P(16), P(16), 4, 256, 384, P(16), P(16), P(16), None),
+    lambda L: L.q2_from_gemlite(P(16), P(16), P(16), 4, 256, 2, P(16), P(16), P(16), None),
+    lambda L: L.q2_from_gemlite(P(16), P(16), P(16), 0, 256, 128, P(16), P(16), P(16), None),
+    lambda L: L.q2_from_gemlite(P(16), None, P(16), 4, 256, 128, P(16), P(16), P(16), None),
 ])
 def test_argument_errors_return_einval(call):
     assert call(tg.lib()) == tg.EINVAL
@@ -114,6 +122,8 @@ def test_argument_errors_return_einval(call):
     lambda L: L.tgemm_q2(P(16), P(16), P(17), P(16), 4, 4, 128, 0, None, 0, None),
     lambda L: L.tgemm_q4(P(16), P(16), P(18), P(16), 4, 4, 128, 0, None, 0, None),
     lambda L: L.q2_pack(P(8), P(16), P(16), P(16), 4, 128, P(16), None),
+    lambda L: L.q2_from_gemlite(P(16), P(16), P(16), 4, 256, 128, P(20), P(16), P(16), None),
+    lambda L: L.q2_from_gemlite(P(16), P(18), P(16), 4, 256, 128, P(16), P(16), P(16), None),
 ])
 def test_misaligned_pointers_return_ealign(call):
     assert call(tg.lib()) == tg.EALIGN
