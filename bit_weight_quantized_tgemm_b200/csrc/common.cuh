@@ -86,6 +86,19 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
   }
 }
 
+// Wait for a phase that must complete (copies or MMAs this thread issued), giving up after
+// kWaitLimitNs with a recorded timeout; used on the way out, where nothing else can help.
+__device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      atomicOr(&g_device_error, kDevErrTimeout);
+      return false;
+    }
+  }
+  return true;
+}
+
 // ---- TMA ---------------------------------------------------------------------------
 
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {

@@ -169,17 +169,6 @@ __device__ __forceinline__ int tc_slot(const TcParams& p, int c, int t) {
 }
 constexpr int kTcSlotFloats = kTcRows * kTcTok;
 
-__device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity) {
-  const uint64_t t0 = globaltimer_ns();
-  while (!mbar_try_wait(bar, parity)) {
-    if (globaltimer_ns() - t0 > kWaitLimitNs) {
-      atomicOr(&g_device_error, kDevErrTimeout);
-      return false;
-    }
-  }
-  return true;
-}
-
 // A warp-uniform bounded wait: every lane gets the same answer, so the .sync.aligned
 // tcgen05 instructions that follow never run with part of a warp.
 __device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity,

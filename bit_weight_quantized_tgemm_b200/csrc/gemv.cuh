@@ -1,27 +1,40 @@
-// gemv.cuh -- small-M path (up to 16 tokens per tile): HBM-bound on the packed weights.
+// gemv.cuh -- small-M path (up to 16 tokens per pass over the weights): HBM-bound on the
+// packed weights, and at these sizes bound by the latency of one trip to memory, so the
+// kernel is laid out to need exactly one such trip after its dependency wait.
 //
-// Each CTA owns 16 weight rows (two 8-row n-tiles of mma.sync m16n8k16); its 8 warps split
-// K in units of 128 weights.  Per pass of up to kp weights along K:
-//   * every lane issues all of its packed-weight loads for the pass first: lane (g, c)
-//     loads the c-th quarter of row g's packed bytes of each of its units, so the warp
-//     reads each row-unit once and a whole pass costs one memory round trip;
-//   * the CTA stages the pass's activation rows in shared memory, converted to the
-//     fragment order of the codes (below), so one ldmatrix.x4 yields a whole A fragment;
-//     tokens past the tile read a shared row of zeros;
-//   * codes are unpacked in registers (the word a lane needs comes from the lane of its
-//     quad that loaded it, by shuffle) into exact bf16 integers for the mma;
-//   * block scales are applied to the f32 partial sums after each block:
-//       Q2_0:  B = q - 1 in {-1, 0, 1}, then y += d * sum              (128-weight block)
-//       4-bit: B = q in 0..15, S = sum of x over the group (an mma against ones),
-//              then y += s * (sum - z * S)                              (64-weight group)
-//     which equals sum_k (q - 1) d x  and  sum_k (q - z) s x  with only f32 rounding.
+// Each CTA owns 16 weight rows (the M side of mma.sync m16n8k16); its 8 warps split K in
+// units of 128 weights; the tokens are the mma's N side (8 per tile, one or two tiles).
+// Per pass over up to kp weights along K:
+//   * lanes of warp 0 start one bulk copy (cp.async.bulk) per token row of the pass's
+//     activations into shared memory, in their natural order, completing on an mbarrier;
+//   * meanwhile every lane loads, straight into registers, all the packed codes it needs
+//     for the pass (lane (g, c): rows g and g+8, bytes [8c, 8c+8) of each of its 32-byte
+//     Q2 row-units, or bytes [8c, 8c+8) and [32+8c, 32+8c+8) of its 64-byte 4-bit
+//     row-units: each 32-byte sector is requested once), and the CTA loads the pass's
+//     scales of its 16 rows with consecutive threads on consecutive scales;
+//   * the codes of one byte (Q2) or byte pair (4-bit) become an A fragment pair with a
+//     byte permute, a mask-and-or that sets a bf16 exponent (the code then reads as an
+//     exact integer plus a known offset), and one subtraction;
+//   * the B fragments (activations) are one 8-byte shared-memory load per k16 step.
+// Block scales are applied to the f32 partial sums after each block:
+//   Q2_0:  A = base + q (base 128 or 32 by k slot), C = sum of (base + 1) x (an mma against
+//          constants), then y += d * (sum - C)                    (128-weight block)
+//   4-bit: A = 128 + q, S = sum of x over the group (an mma against ones),
+//          then y += s * (sum - (128 + z) * S)                      (64-weight group)
+// which equals sum_k (q - 1) d x  and  sum_k (q - z) s x  up to f32 rounding (all products
+// of the bf16 operands are exact in the f32 accumulators).
 // The warps' partial sums are reduced through shared memory; the optional low-rank
 // branch adds sum_i B[n][i] u[m][i] (u = A x in f32, from the lora kernels).
 //
-// Fragment order: a 32-bit word of Q2 codes unpacks with one shift and mask per pair into
-// codes (i, i+8); a word of 4-bit codes into codes (i, i+4).  The staged activations hold,
-// in each 16-group (Q2) or 8-group (4-bit), x[i] and x[i+8] (x[i] and x[i+4]) side by
-// side, so the mma's k pair (2i, 2i+1) is the same pair of weights on both operands.
+// k order inside an mma.  Lane (g, c) supplies the k slots {2c, 2c+1, 2c+8, 2c+9} of A
+// (weight rows g, g+8) and of B (token g).  In k16 step s of a 128-k unit those slots hold
+// four consecutive codes -- one Q2 byte, or two 4-bit bytes -- in the slot order
+//   Q2:    codes 32c + 4s + (0, 1 | 2, 3)
+//   4-bit: codes 16c + 4s + (0, 2 | 1, 3)  (steps 0-3, the first 64-weight group), and
+//          64 + 16c + 4(s-4) + (0, 2 | 1, 3)  (steps 4-7, the second group)
+// so that all codes of a 4-bit step share one group.  Any assignment of codes to slots
+// gives the same contraction as long as A and B agree, and every lane's codes for all eight
+// steps are the 8 (Q2) or 16 (4-bit) bytes it loaded.
 #pragma once
 
 #include "common.cuh"
@@ -30,46 +43,31 @@ namespace tgemm {
 
 constexpr int kGvRows = 16;   // weight rows per CTA
 constexpr int kGvWarps = 8;   // warps per CTA, splitting K
-constexpr int kGvUnit = 128;  // K per unit
-constexpr int kGvMaxU = 6;    // units per warp per pass
-constexpr int kGvKPMax = kGvMaxU * kGvWarps * kGvUnit;  // 6144
-// Dynamic shared memory per CTA: the staged activations (two CTAs per SM, 16 tokens x
-// 3072 in one pass); after the last pass it holds the warps' partial sums instead.
+constexpr int kGvUnit = 128;  // K per unit (one Q2 block, two 4-bit groups)
+// units per warp per pass: the codes of a pass are held in registers
+template <int FMT>
+struct GvFmt {
+  static constexpr int kMaxU = FMT == 0 ? 6 : 4;
+  static constexpr int kKPMax = kMaxU * kGvWarps * kGvUnit;  // 6144 (Q2), 4096 (4-bit)
+  static constexpr int kUnitBytes = FMT == 0 ? 32 : 64;      // packed bytes of a row-unit
+  static constexpr int kWords = FMT == 0 ? 2 : 4;             // 32-bit code words per lane
+};
+// Dynamic shared memory per CTA (the staged activations): two CTAs fit on one SM with 16
+// tokens x 3072 in one pass.
 constexpr int kGvXBudget = 104960;
-constexpr int kGvRedBytes = kGvWarps * 16 * (kGvRows + 1) * 4;
 
 __host__ __device__ constexpr int gemv_row_stride_bytes(int kp) { return 2 * kp + 16; }
-// K per pass: the largest multiple of 128 (at most kGvKPMax) whose staged activation rows
-// (`mrows` tokens plus one row of zeros) fit kGvXBudget; never more than K needs.
-__host__ __device__ inline int gemv_pass_k(int mrows, int K) {
+// K per pass: the largest multiple of 128 (at most the format's kKPMax) whose staged
+// activation rows (`mrows` tokens) fit kGvXBudget; never more than K needs.
+__host__ __device__ inline int gemv_pass_k(int fmt, int mrows, int K) {
+  const int kmax = fmt == 0 ? GvFmt<0>::kKPMax : GvFmt<1>::kKPMax;
   int kp = (K + kGvUnit - 1) / kGvUnit * kGvUnit;
-  if (kp > kGvKPMax) kp = kGvKPMax;
-  while (kp > kGvUnit && (mrows + 1) * gemv_row_stride_bytes(kp) > kGvXBudget) kp -= kGvUnit;
+  if (kp > kmax) kp = kmax;
+  while (kp > kGvUnit && mrows * gemv_row_stride_bytes(kp) > kGvXBudget) kp -= kGvUnit;
   return kp;
 }
 __host__ __device__ constexpr int gemv_smem_bytes(int mrows, int kp) {
-  return (mrows + 1) * gemv_row_stride_bytes(kp) > kGvRedBytes
-             ? (mrows + 1) * gemv_row_stride_bytes(kp)
-             : kGvRedBytes;
-}
-
-// bf16x2 a - b (exact for the small integers used here)
-__device__ __forceinline__ uint32_t bsub2(uint32_t a, uint32_t b) {
-  __nv_bfloat162 r =
-      __hsub2(*reinterpret_cast<__nv_bfloat162*>(&a), *reinterpret_cast<__nv_bfloat162*>(&b));
-  return *reinterpret_cast<uint32_t*>(&r);
-}
-
-// Two 2-bit codes (bits s..s+1 and s+16..s+17 of w) -> bf16x2 (q - 1).
-__device__ __forceinline__ uint32_t q2_pair_bf16(uint32_t w, int s) {
-  const uint32_t t = lop3_and_or(w >> s, 0x00030003u, 0x43004300u);  // 128 + q
-  return bsub2(t, 0x43014301u);                                       // - 129
-}
-
-// Two 4-bit codes (bits s..s+3 and s+16..s+19 of w) -> bf16x2 q.
-__device__ __forceinline__ uint32_t q4_pair_bf16(uint32_t w, int s) {
-  const uint32_t t = lop3_and_or(w >> s, 0x000F000Fu, 0x43004300u);  // 128 + q
-  return bsub2(t, 0x43004300u);                                       // - 128
+  return mrows * gemv_row_stride_bytes(kp);
 }
 
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
@@ -78,83 +76,97 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
   return r;
 }
 
-__device__ __forceinline__ void st_shared_v4(uint32_t saddr, uint32_t a, uint32_t b, uint32_t c,
-                                             uint32_t d) {
-  asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(saddr), "r"(a), "r"(b), "r"(c),
-               "r"(d)
-               : "memory");
+// Q2: byte `b` of w (codes q0..q3 at bits 0-1, 2-3, 4-5, 6-7) -> two bf16x2 pairs
+// (128 + q0, 32 + q1) and (128 + q2, 32 + q3).  The byte is copied into both halves; the
+// low half keeps bits 0-1 under the exponent of 128 (ulp 1), the high half bits 2-3 (its
+// bits 18-19) under the exponent of 32 (ulp 1/4, so bit 2 is worth 1).  The offsets are
+// removed after the mma: sum_k (q - 1) x = sum_k (base_k + q) x - sum_k (base_k + 1) x,
+// the last term being one more mma of x against the constant pairs (129, 33).
+constexpr uint32_t kQ2Offset1 = 0x42044301u;  // bf16x2 (129, 33)
+__device__ __forceinline__ void q2_byte_pairs(uint32_t w, int b, uint32_t& lo, uint32_t& hi) {
+  const uint32_t p = prmt(w, 0u, static_cast<uint32_t>(b) | 0x4040u | (static_cast<uint32_t>(b) << 8));
+  lo = lop3_and_or(p, 0x000C0003u, 0x42004300u);
+  hi = lop3_and_or(p >> 4, 0x000C0003u, 0x42004300u);
 }
 
-// 16 bf16 activations (v: pairs (0,1) .. (14,15)) -> the fragment order of format FMT.
-//   Q2:    word i = (x[i], x[i+8])                         i < 8
-//   4-bit: word 4h+i = (x[8h+i], x[8h+i+4])                h < 2, i < 4
-template <int FMT>
-__device__ __forceinline__ void x_fragment_order(const uint32_t (&v)[8], uint32_t (&o)[8]) {
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    if (FMT == 0) {
-      const uint32_t sel = (i & 1) ? 0x7632u : 0x5410u;  // odd i: the high halves
-      o[i] = prmt(v[i >> 1], v[4 + (i >> 1)], sel);
-    } else {
-      const int h = i >> 2, j = i & 3;
-      const uint32_t sel = (j & 1) ? 0x7632u : 0x5410u;
-      o[i] = prmt(v[4 * h + (j >> 1)], v[4 * h + 2 + (j >> 1)], sel);
-    }
-  }
+// 4-bit: bytes 2h and 2h+1 of w (codes q0, q1 | q2, q3, low nibble first) -> bf16x2 pairs
+// (128 + q0, 128 + q2) and (128 + q1, 128 + q3), each nibble under the exponent of 128;
+// the offset joins the zero point: (q - z) = (128 + q) - (128 + z).
+__device__ __forceinline__ void q4_bytes_pairs(uint32_t w, int h, uint32_t& lo, uint32_t& hi) {
+  const uint32_t sel = static_cast<uint32_t>(2 * h) | 0x40u | (static_cast<uint32_t>(2 * h + 1) << 8) | 0x4000u;
+  const uint32_t p = prmt(w, 0u, sel);
+  lo = lop3_and_or(p, 0x000F000Fu, 0x43004300u);
+  hi = lop3_and_or(p >> 4, 0x000F000Fu, 0x43004300u);
+}
+
+// Bulk copy of `bytes` (a multiple of 16, both addresses 16-byte aligned) from global to
+// this CTA's shared memory, completing on `bar`.
+__device__ __forceinline__ void bulk_copy_g2s(uint32_t dst, const void* src, uint32_t bytes,
+                                              uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+      : "memory");
 }
 
 // DUAL: a second input (x2, wq2, scales2, K2) whose product adds into the same sums.
-template <int FMT, bool LORA, bool DUAL>
-__global__ void __launch_bounds__(256) gemv_kernel(
+// T: token tiles of 8 per pass (1 for up to 8 tokens, 2 for up to 16).
+template <int FMT, int T, bool LORA, bool DUAL>
+__global__ void __launch_bounds__(256, 2) gemv_kernel(
     const uint16_t* __restrict__ x, const uint8_t* __restrict__ wq,
     const uint16_t* __restrict__ scales, void* __restrict__ y, int M, int N, int K, int out_f32,
     const float* __restrict__ u, const uint16_t* __restrict__ lb, int r, int lb_sn, int lb_si,
-    int mrows, int kp,
+    int kp,
     const uint16_t* __restrict__ x2, const uint8_t* __restrict__ wq2,
     const uint16_t* __restrict__ scales2, int K2) {
-  extern __shared__ __align__(16) uint8_t gv_smem[];
-  // the warps' partial sums, over the staged activations once all passes are done
-  auto red = reinterpret_cast<float(*)[16][kGvRows + 1]>(gv_smem);
-  // scales of this CTA's rows for one pass: Q2 d per unit, 4-bit (s, z) per group
-  constexpr int kScl = FMT == 0 ? kGvKPMax / 128 : kGvKPMax / 64;
+  using F = GvFmt<FMT>;
+  constexpr int kTok = 8 * T;  // tokens per pass over the weights
+  extern __shared__ __align__(128) uint8_t gv_smem[];
+  __shared__ float red[kGvWarps][kGvRows][kTok + 1];  // the warps' partial sums
+  __shared__ __align__(8) uint64_t xbar;              // the activation copies of a pass
+  __shared__ uint32_t abort_word;
+  // the pass's scales of the CTA's rows: Q2 d per unit, 4-bit (s, z) per group
+  constexpr int kScl = FMT == 0 ? F::kMaxU * kGvWarps : 2 * F::kMaxU * kGvWarps;
+  constexpr int kSclPerThread = kGvRows * kScl / 256;
   __shared__ uint32_t scl[kGvRows][kScl];
-  pdl_trigger();
-  {
-    // the first pass's packed rows -> L2 while the previous kernel finishes (no data
-    // reaches the SM before the wait below)
-    const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
-    const int64_t rb = FMT == 0 ? K / 4 : K / 2;
-    const int units0 = min((K + kGvUnit - 1) / kGvUnit, kp / kGvUnit);
-    const int row = blockIdx.x * kGvRows + (l & 15);
-    if (row < N)
-      for (int un = w + kGvWarps * (l >> 4); un < units0; un += 2 * kGvWarps)
-        prefetch_l2(wq + static_cast<int64_t>(row) * rb + static_cast<int64_t>(un) * (FMT == 0 ? 32 : 64));
-  }
-  pdl_wait();
-  const uint32_t xs = smem_u32(gv_smem);
-  const int rs = gemv_row_stride_bytes(kp);
-  const uint32_t zrow = xs + mrows * rs;  // zeros: the rows of tokens past the tile
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, c = lane & 3;
   const int n0 = blockIdx.x * kGvRows;
-  constexpr int kUnitBytes = FMT == 0 ? 32 : 64;  // packed bytes of one row per unit
-  constexpr int kQW = FMT == 0 ? 2 : 4;           // 32-bit words a lane loads per row-unit
+  const uint32_t xs = smem_u32(gv_smem);
+  const uint32_t bar = smem_u32(&xbar);
+  const int rs = gemv_row_stride_bytes(kp);
+  volatile uint32_t* abort_flag = &abort_word;
+  if (tid == 0) {
+    mbar_init(bar, 1);
+    abort_word = 0u;
+    fence_mbar_init();
+  }
+  pdl_trigger();
+  {
+    // the first pass's packed rows and scales -> L2 while the previous kernel finishes
+    // (no data reaches the SM before the wait below)
+    const int64_t rb = FMT == 0 ? K / 4 : K / 2;
+    const int pass_bytes = static_cast<int>(rb < (FMT == 0 ? kp / 4 : kp / 2) ? rb : (FMT == 0 ? kp / 4 : kp / 2));
+    const int lines = (pass_bytes + 127) / 128;
+    for (int i = tid; i < kGvRows * lines; i += blockDim.x) {
+      const int row = n0 + i / lines;
+      if (row < N) prefetch_l2(wq + static_cast<int64_t>(row) * rb + (i % lines) * 128);
+    }
+    if (tid < kGvRows && n0 + tid < N)
+      prefetch_l2(scales + static_cast<int64_t>(n0 + tid) * (FMT == 0 ? K / 128 : K / 32));
+  }
+  __syncthreads();  // the barrier's initialisation is visible to every thread
+  pdl_wait();
 
-  // ldmatrix.x4 row address of this lane: matrices (tokens 0-7 | 8-15) x (k 0-7 | 8-15)
-  const int mi = lane >> 3, arow = (mi & 1) * 8 + (lane & 7);
-  const uint32_t a_col = (mi >> 1) * 16;
-
-  for (int m0 = 0; m0 < M; m0 += 16) {
-    const int mt = min(16, M - m0);  // tokens in this tile (<= mrows)
-    const uint32_t a_row = (arow < mt ? xs + arow * rs : zrow) + a_col;
-    // (re)zero the zero row: the previous tile's partial sums may have covered it
-    for (int i = tid; i < rs / 16; i += blockDim.x) st_shared_v4(zrow + 16 * i, 0u, 0u, 0u, 0u);
-    float acc[2][4];
+  uint32_t phase = 0;  // completed activation copies (the mbarrier's phase parity)
+  for (int m0 = 0; m0 < M; m0 += kTok) {
+    const int mt = min(kTok, M - m0);  // tokens in this pass over the weights
+    float acc[T][4];
 #pragma unroll
-    for (int j = 0; j < 2; ++j)
+    for (int t = 0; t < T; ++t)
 #pragma unroll
-      for (int e = 0; e < 4; ++e) acc[j][e] = 0.f;
+      for (int e = 0; e < 4; ++e) acc[t][e] = 0.f;
 
     // one input, or two (a projection split along its input axis: their products add
     // into the same partial sums)
@@ -163,169 +175,198 @@ __global__ void __launch_bounds__(256) gemv_kernel(
       const uint8_t* wqq = part ? wq2 : wq;
       const uint16_t* sq = part ? scales2 : scales;
       const int Kq = part ? K2 : K;
-      const int nunitsq = (Kq + kGvUnit - 1) / kGvUnit;
-      const int64_t row_bytesq = FMT == 0 ? Kq / 4 : Kq / 2;
-      const int nscaleq = FMT == 0 ? Kq / 128 : Kq / 64;
+      const int64_t row_bytes = FMT == 0 ? Kq / 4 : Kq / 2;
+      const int nscale = FMT == 0 ? Kq / 128 : Kq / 64;
       for (int k0 = 0; k0 < Kq; k0 += kp) {
         const int kpass = min(kp, Kq - k0);
         const int u_base = k0 / kGvUnit;
-        const int u_end = min(nunitsq, (k0 + kpass + kGvUnit - 1) / kGvUnit);
-        // ---- every packed-weight load of this pass (lane (g, c): quarter c of row g)
-        uint32_t wreg[kGvMaxU][2][kQW];
+        const int u_end = (k0 + kpass + kGvUnit - 1) / kGvUnit;
+        // ---- the pass's activation rows -> shared memory (async)
+        if (warp == 0) {
+          if (lane == 0) mbar_arrive_expect_tx(bar, static_cast<uint32_t>(mt * kpass * 2));
+          __syncwarp();
+          if (lane < mt)
+            bulk_copy_g2s(xs + lane * rs, xq + static_cast<int64_t>(m0 + lane) * Kq + k0,
+                          static_cast<uint32_t>(kpass * 2), bar);
+        }
+        // the next pass's rows -> L2
+        if (k0 + kp < Kq) {
+          const int nb = FMT == 0 ? min(kp, Kq - k0 - kp) / 4 : min(kp, Kq - k0 - kp) / 2;
+          const int lines = (nb + 127) / 128;
+          for (int i = tid; i < kGvRows * lines; i += blockDim.x) {
+            const int row = n0 + i / lines;
+            if (row < N)
+              prefetch_l2(wqq + static_cast<int64_t>(row) * row_bytes +
+                          (FMT == 0 ? (k0 + kp) / 4 : (k0 + kp) / 2) + (i % lines) * 128);
+          }
+        }
+        // ---- every packed-code load of this pass, straight into registers
+        uint32_t wreg[F::kMaxU][2][F::kWords];
 #pragma unroll
-        for (int i = 0; i < kGvMaxU; ++i) {
-          const int unit = u_base + i * kGvWarps + warp;
+        for (int i = 0; i < F::kMaxU; ++i) {
+          const int unit = u_base + warp + kGvWarps * i;
 #pragma unroll
           for (int j = 0; j < 2; ++j) {
             const int row = n0 + 8 * j + g;
             const bool ok = unit < u_end && row < N;
-            const uint8_t* base = wqq + static_cast<int64_t>(row) * row_bytesq +
-                                  static_cast<int64_t>(unit) * kUnitBytes;
+            const uint8_t* base = wqq + static_cast<int64_t>(row) * row_bytes +
+                                  static_cast<int64_t>(unit) * F::kUnitBytes;
             if (FMT == 0) {
-              uint2 v = make_uint2(0x55555555u, 0x55555555u);  // code 1 everywhere = weight 0
-              if (ok) v = __ldg(reinterpret_cast<const uint2*>(base + 8 * c));
-              wreg[i][j][0] = v.x;
-              wreg[i][j][1] = v.y;
+              // codes 32c..32c+31 of the unit (code 1 = weight 0 where there is no row)
+              uint2 a = make_uint2(0x55555555u, 0x55555555u);
+              if (ok) a = __ldg(reinterpret_cast<const uint2*>(base + 8 * c));
+              wreg[i][j][0] = a.x;
+              wreg[i][j][1] = a.y;
             } else {
-              // a unit's second 32 bytes exist only where K reaches its second group
-              uint4 v = make_uint4(0u, 0u, 0u, 0u);
-              if (ok && (c < 2 || static_cast<int64_t>(unit) * kGvUnit + 64 < Kq))
-                v = __ldg(reinterpret_cast<const uint4*>(base + 16 * c));
-              wreg[i][j][0] = v.x;
-              wreg[i][j][1] = v.y;
-              wreg[i][j][2] = v.z;
-              wreg[i][j][3] = v.w;
+              // codes 16c..16c+15 and 64+16c..64+16c+15; the unit's second 64 codes exist
+              // only where K reaches them
+              const bool ok2 = ok && static_cast<int64_t>(unit) * kGvUnit + 64 < Kq;
+              uint2 a = make_uint2(0u, 0u), b = make_uint2(0u, 0u);
+              if (ok) a = __ldg(reinterpret_cast<const uint2*>(base + 8 * c));
+              if (ok2) b = __ldg(reinterpret_cast<const uint2*>(base + 32 + 8 * c));
+              wreg[i][j][0] = a.x;
+              wreg[i][j][1] = a.y;
+              wreg[i][j][2] = b.x;
+              wreg[i][j][3] = b.y;
             }
           }
         }
-        // ---- this pass's sq for the CTA's rows
+        // ---- the pass's scales (consecutive threads, consecutive scales), then to shared
         {
           const int s_base = FMT == 0 ? u_base : 2 * u_base;
-          const int s_cnt = FMT == 0 ? (u_end - u_base) : min(nscaleq - s_base, 2 * (u_end - u_base));
-          for (int it = tid; it < kGvRows * s_cnt; it += blockDim.x) {
+          const int s_cnt = FMT == 0 ? u_end - u_base : min(nscale - s_base, 2 * (u_end - u_base));
+          uint32_t sv[kSclPerThread];
+#pragma unroll
+          for (int e = 0; e < kSclPerThread; ++e) {
+            const int it = tid + 256 * e;
             const int rl = it / s_cnt, si = it - rl * s_cnt;
             const int n = n0 + rl;
-            uint32_t v = 0;
-            if (n < N) {
-              const int64_t idx = static_cast<int64_t>(n) * nscaleq + s_base + si;
-              v = FMT == 0 ? static_cast<uint32_t>(sq[idx])
-                           : reinterpret_cast<const uint32_t*>(sq)[idx];
+            sv[e] = 0u;
+            if (rl < kGvRows && n < N) {
+              const int64_t idx = static_cast<int64_t>(n) * nscale + s_base + si;
+              sv[e] = FMT == 0 ? static_cast<uint32_t>(__ldg(sq + idx))
+                               : __ldg(reinterpret_cast<const uint32_t*>(sq) + idx);
             }
-            scl[rl][si] = v;
           }
-        }
-        // ---- the pass's activations, in fragment order
-        {
-          const int ng = kpass / 16;  // 16-element groups per token row
-          for (int gi = tid; gi < mt * ng; gi += blockDim.x) {
-            const int row = gi / ng, grp = gi - row * ng;
-            const uint4* src = reinterpret_cast<const uint4*>(
-                xq + static_cast<int64_t>(m0 + row) * Kq + k0 + 16 * grp);
-            const uint4 a = __ldg(src), b = __ldg(src + 1);
-            const uint32_t v[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-            uint32_t o[8];
-            x_fragment_order<FMT>(v, o);
-            const uint32_t dst = xs + row * rs + 32 * grp;
-            st_shared_v4(dst, o[0], o[1], o[2], o[3]);
-            st_shared_v4(dst + 16, o[4], o[5], o[6], o[7]);
-          }
-        }
-        __syncthreads();
-        // ---- the warp's units: A fragments by ldmatrix, B fragments from the codes
 #pragma unroll
-        for (int i = 0; i < kGvMaxU; ++i) {
-          const int unit = u_base + i * kGvWarps + warp;
+          for (int e = 0; e < kSclPerThread; ++e) {
+            const int it = tid + 256 * e;
+            const int rl = it / s_cnt, si = it - rl * s_cnt;
+            if (rl < kGvRows) scl[rl][si] = sv[e];
+          }
+        }
+        // ---- wait for the activations (bounded); every thread must agree before going on
+        const bool got = mbar_wait(bar, phase, abort_flag);
+        phase ^= 1u;
+        if (!__syncthreads_and(got)) {
+          // give the copies in flight a bounded time to land before the CTA leaves
+          if (tid == 0) mbar_wait_drain(bar, phase ^ 1u);
+          return;
+        }
+        // ---- the warp's units
+#pragma unroll
+        for (int i = 0; i < F::kMaxU; ++i) {
+          const int unit = u_base + warp + kGvWarps * i;
           if (unit >= u_end) break;
-          const int ku = (unit - u_base) * kGvUnit;  // unit offset within the pass
+          const int ui = unit - u_base;  // the unit within the pass
           if (FMT == 0) {
-            float part[2][4];
+            float pacc[T][4], corr[T][4];
 #pragma unroll
-            for (int j = 0; j < 2; ++j)
+            for (int t = 0; t < T; ++t)
 #pragma unroll
-              for (int e = 0; e < 4; ++e) part[j][e] = 0.f;
+              for (int e = 0; e < 4; ++e) pacc[t][e] = corr[t][e] = 0.f;
+            const uint32_t off[4] = {kQ2Offset1, kQ2Offset1, kQ2Offset1, kQ2Offset1};
 #pragma unroll
-            for (int s = 0; s < 8; ++s) {  // k16 step s: word s of the row-unit
+            for (int s = 0; s < 8; ++s) {
               uint32_t af[4];
-              ldmatrix_x4(a_row + 2 * (ku + 16 * s), af);
-              const int src = (lane & ~3) | (s >> 1);  // the quad lane that loaded word s
+              q2_byte_pairs(wreg[i][0][s >> 2], s & 3, af[0], af[2]);
+              q2_byte_pairs(wreg[i][1][s >> 2], s & 3, af[1], af[3]);
+              // activations 32c + 4s .. +3 of the unit, token g (+8t)
+              const uint32_t xo = xs + 2 * (ui * kGvUnit + 32 * c + 4 * s);
 #pragma unroll
-              for (int j = 0; j < 2; ++j) {
-                const uint32_t w = __shfl_sync(0xFFFFFFFFu, wreg[i][j][s & 1], src);
-                mma_bf16_16816(part[j], af, q2_pair_bf16(w, 2 * c), q2_pair_bf16(w, 2 * c + 8));
+              for (int t = 0; t < T; ++t) {
+                uint2 bv = make_uint2(0u, 0u);
+                if (g + 8 * t < mt) bv = ld_shared_v2(xo + (g + 8 * t) * rs);
+                mma_bf16_16816(pacc[t], af, bv.x, bv.y);
+                mma_bf16_16816(corr[t], off, bv.x, bv.y);
               }
             }
-            // part[j][e]: token g (+8 for e >= 2), weight row 8j + 2c + (e & 1)
+            // pacc[t][e]: weight row g (+8 for e >= 2), token 2c + (e & 1) + 8t; corr[t][e]
+            // is the same for every row
+            const float d0 = __half2float(__ushort_as_half(static_cast<uint16_t>(scl[g][ui])));
+            const float d1 = __half2float(__ushort_as_half(static_cast<uint16_t>(scl[g + 8][ui])));
 #pragma unroll
-            for (int j = 0; j < 2; ++j) {
-              const int rl = 8 * j + 2 * c, ui = unit - u_base;
-              const float d0 = __half2float(__ushort_as_half(static_cast<uint16_t>(scl[rl][ui])));
-              const float d1 = __half2float(__ushort_as_half(static_cast<uint16_t>(scl[rl + 1][ui])));
-              acc[j][0] = fmaf(d0, part[j][0], acc[j][0]);
-              acc[j][1] = fmaf(d1, part[j][1], acc[j][1]);
-              acc[j][2] = fmaf(d0, part[j][2], acc[j][2]);
-              acc[j][3] = fmaf(d1, part[j][3], acc[j][3]);
+            for (int t = 0; t < T; ++t) {
+              acc[t][0] = fmaf(d0, pacc[t][0] - corr[t][0], acc[t][0]);
+              acc[t][1] = fmaf(d0, pacc[t][1] - corr[t][1], acc[t][1]);
+              acc[t][2] = fmaf(d1, pacc[t][2] - corr[t][0], acc[t][2]);
+              acc[t][3] = fmaf(d1, pacc[t][3] - corr[t][1], acc[t][3]);
             }
           } else {
 #pragma unroll
-            for (int h2 = 0; h2 < 2; ++h2) {
-              const int grp = 2 * unit + h2;
-              if (grp * 64 >= Kq) break;
-              float part[2][4], ssum[4] = {0.f, 0.f, 0.f, 0.f};
+            for (int h2 = 0; h2 < 2; ++h2) {  // the unit's two 64-weight groups
+              if (h2 == 1 && static_cast<int64_t>(unit) * kGvUnit + 64 >= Kq) break;
+              float pacc[T][4], ssum[T][4];
 #pragma unroll
-              for (int j = 0; j < 2; ++j)
+              for (int t = 0; t < T; ++t)
 #pragma unroll
-                for (int e = 0; e < 4; ++e) part[j][e] = 0.f;
+                for (int e = 0; e < 4; ++e) pacc[t][e] = ssum[t][e] = 0.f;
 #pragma unroll
-              for (int sq = 0; sq < 4; ++sq) {  // k16 step s: words 2s, 2s+1 of the row-unit
-                const int s = 4 * h2 + sq;
+              for (int sq4 = 0; sq4 < 4; ++sq4) {
+                const int s = 4 * h2 + sq4;
                 uint32_t af[4];
-                ldmatrix_x4(a_row + 2 * (ku + 16 * s), af);
-                mma_bf16_16816(ssum, af, 0x3F803F80u, 0x3F803F80u);  // xq against ones
-                const int src = (lane & ~3) | (s >> 1);
+                q4_bytes_pairs(wreg[i][0][s >> 1], s & 1, af[0], af[2]);
+                q4_bytes_pairs(wreg[i][1][s >> 1], s & 1, af[1], af[3]);
+                // activations 64 h2 + 16c + 4 sq4 .. +3 of the unit, token g (+8t)
+                const uint32_t xo = xs + 2 * (ui * kGvUnit + 64 * h2 + 16 * c + 4 * sq4);
+                const uint32_t ones[4] = {0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u};
 #pragma unroll
-                for (int j = 0; j < 2; ++j) {
-                  const uint32_t w0 = __shfl_sync(0xFFFFFFFFu, wreg[i][j][2 * (s & 1)], src);
-                  const uint32_t w1 = __shfl_sync(0xFFFFFFFFu, wreg[i][j][2 * (s & 1) + 1], src);
-                  mma_bf16_16816(part[j], af, q4_pair_bf16(w0, 4 * c), q4_pair_bf16(w1, 4 * c));
+                for (int t = 0; t < T; ++t) {
+                  uint2 bv = make_uint2(0u, 0u);
+                  if (g + 8 * t < mt) bv = ld_shared_v2(xo + (g + 8 * t) * rs);
+                  const uint32_t b0 = prmt(bv.x, bv.y, 0x5410u);  // (x0, x2)
+                  const uint32_t b1 = prmt(bv.x, bv.y, 0x7632u);  // (x1, x3)
+                  mma_bf16_16816(pacc[t], af, b0, b1);
+                  mma_bf16_16816(ssum[t], ones, b0, b1);  // S: sum of x per token
                 }
               }
-              // ssum[0] = S for token g, ssum[2] = S for token g + 8
+              // ssum[t][0] = S of token 2c + 8t, ssum[t][1] = S of token 2c + 1 + 8t
+              const uint32_t v0 = scl[g][2 * ui + h2], v1 = scl[g + 8][2 * ui + h2];
+              // codes arrive as 128 + q: the zero point becomes 128 + z (exact in f32)
+              const float s0 = __half2float(__ushort_as_half(static_cast<uint16_t>(v0 & 0xFFFFu)));
+              const float z0 = 128.f + __half2float(__ushort_as_half(static_cast<uint16_t>(v0 >> 16)));
+              const float s1 = __half2float(__ushort_as_half(static_cast<uint16_t>(v1 & 0xFFFFu)));
+              const float z1 = 128.f + __half2float(__ushort_as_half(static_cast<uint16_t>(v1 >> 16)));
 #pragma unroll
-              for (int j = 0; j < 2; ++j) {
-                const int rl = 8 * j + 2 * c, gi = grp - 2 * u_base;
-                const uint32_t v0 = scl[rl][gi], v1 = scl[rl + 1][gi];
-                const float s0 = __half2float(__ushort_as_half(static_cast<uint16_t>(v0 & 0xFFFFu)));
-                const float z0 = __half2float(__ushort_as_half(static_cast<uint16_t>(v0 >> 16)));
-                const float s1 = __half2float(__ushort_as_half(static_cast<uint16_t>(v1 & 0xFFFFu)));
-                const float z1 = __half2float(__ushort_as_half(static_cast<uint16_t>(v1 >> 16)));
-                acc[j][0] = fmaf(s0, fmaf(-z0, ssum[0], part[j][0]), acc[j][0]);
-                acc[j][1] = fmaf(s1, fmaf(-z1, ssum[0], part[j][1]), acc[j][1]);
-                acc[j][2] = fmaf(s0, fmaf(-z0, ssum[2], part[j][2]), acc[j][2]);
-                acc[j][3] = fmaf(s1, fmaf(-z1, ssum[2], part[j][3]), acc[j][3]);
+              for (int t = 0; t < T; ++t) {
+                acc[t][0] = fmaf(s0, fmaf(-z0, ssum[t][0], pacc[t][0]), acc[t][0]);
+                acc[t][1] = fmaf(s0, fmaf(-z0, ssum[t][1], pacc[t][1]), acc[t][1]);
+                acc[t][2] = fmaf(s1, fmaf(-z1, ssum[t][0], pacc[t][2]), acc[t][2]);
+                acc[t][3] = fmaf(s1, fmaf(-z1, ssum[t][1], pacc[t][3]), acc[t][3]);
               }
             }
           }
         }
-        __syncthreads();  // everyone is done with this pass's activations and sq
+        __syncthreads();  // everyone is done with this pass's activations
       }
     }
 
     // ---- reduce the warps' partial sums and write y ---------------------------------
 #pragma unroll
-    for (int j = 0; j < 2; ++j) {
-      red[warp][g][8 * j + 2 * c] = acc[j][0];
-      red[warp][g][8 * j + 2 * c + 1] = acc[j][1];
-      red[warp][g + 8][8 * j + 2 * c] = acc[j][2];
-      red[warp][g + 8][8 * j + 2 * c + 1] = acc[j][3];
+    for (int t = 0; t < T; ++t) {
+      red[warp][g][2 * c + 8 * t] = acc[t][0];
+      red[warp][g][2 * c + 1 + 8 * t] = acc[t][1];
+      red[warp][g + 8][2 * c + 8 * t] = acc[t][2];
+      red[warp][g + 8][2 * c + 1 + 8 * t] = acc[t][3];
     }
     __syncthreads();
-    for (int o = tid; o < 16 * kGvRows; o += blockDim.x) {
+    for (int o = tid; o < kTok * kGvRows; o += blockDim.x) {
       const int mm = o / kGvRows, nn = o % kGvRows;
       const int m = m0 + mm, n = n0 + nn;
-      if (m >= M || n >= N) continue;
+      if (mm >= mt || n >= N) continue;
       float v = 0.f;
 #pragma unroll
-      for (int w = 0; w < kGvWarps; ++w) v += red[w][mm][nn];
+      for (int w = 0; w < kGvWarps; ++w) v += red[w][nn][mm];
       if (LORA) {
         float br = 0.f;
         for (int i = 0; i < r; ++i)

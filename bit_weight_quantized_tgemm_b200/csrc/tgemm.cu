@@ -346,15 +346,28 @@ int prep_lora_prepare() {
   return err == cudaSuccess ? TGEMM_OK : TGEMM_ECUDA;
 }
 
-template <int FMT, bool LORA, bool DUAL = false>
+template <int FMT, int T, bool LORA, bool DUAL = false>
 int gemv_prepare() {
   static std::once_flag once;
   static cudaError_t err = cudaSuccess;
   std::call_once(once, [] {
-    err = cudaFuncSetAttribute(gemv_kernel<FMT, LORA, DUAL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    err = cudaFuncSetAttribute(gemv_kernel<FMT, T, LORA, DUAL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                kGvXBudget);
   });
   return err == cudaSuccess ? TGEMM_OK : TGEMM_ECUDA;
+}
+
+// One small-M launch: T token tiles of 8 per pass over the weights.
+template <int FMT, int T, bool LORA, bool DUAL>
+int launch_gemv(int grid, size_t smem, cudaStream_t st, const uint16_t* x, const uint8_t* wq,
+                const uint16_t* scales, void* y, int M, int N, int K, int out_f32, const float* u32,
+                const uint16_t* lb, int r, int lb_sn, int lb_si, int kp, const uint16_t* x2,
+                const uint8_t* wq2, const uint16_t* d2, int K2) {
+  if (int e = gemv_prepare<FMT, T, LORA, DUAL>()) return e;
+  return launch(FMT == 0 ? TGEMM_KIND_GEMV_Q2 : TGEMM_KIND_GEMV_Q4, st, [&] {
+    return pdl_launch(gemv_kernel<FMT, T, LORA, DUAL>, grid, 256, smem, st, x, wq, scales, y, M, N, K,
+                      out_f32, u32, lb, r, lb_sn, lb_si, kp, x2, wq2, d2, K2);
+  });
 }
 
 // ---- the matmul driver ---------------------------------------------------------------
@@ -415,35 +428,23 @@ int run_gemm(int fmt, const uint16_t* x, const uint8_t* wq, const uint16_t* scal
     }
     const int grid = (N + kGvRows - 1) / kGvRows;
     const int mrows = M < 16 ? M : 16;
-    const int kp = gemv_pass_k(mrows, K > K2 ? K : K2);
+    const int kp = gemv_pass_k(fmt, mrows, K > K2 ? K : K2);
     const size_t smem = gemv_smem_bytes(mrows, kp);
-    if (fmt == 0 && lora) {
-      if (int e = gemv_prepare<0, true>()) return e;
-      return launch(TGEMM_KIND_GEMV_Q2, st, [&] {
-        return pdl_launch(gemv_kernel<0, true, false>, grid, 256, smem, st, x, wq, scales, y, M, N, K, out_f32, u32, lb, r, lb_sn, lb_si, mrows, kp,
-                          nullptr, nullptr, nullptr, 0);
-      });
-    }
-    if (fmt == 0 && dual) {
-      if (int e = gemv_prepare<0, false, true>()) return e;
-      return launch(TGEMM_KIND_GEMV_Q2, st, [&] {
-        return pdl_launch(gemv_kernel<0, false, true>, grid, 256, smem, st, x, wq, scales, y, M, N, K, out_f32, nullptr, nullptr, 0, 0, 0, mrows, kp,
-                          in2.x, in2.wq, in2.d, K2);
-      });
-    }
-    if (fmt == 0) {
-      if (int e = gemv_prepare<0, false>()) return e;
-      return launch(TGEMM_KIND_GEMV_Q2, st, [&] {
-        return pdl_launch(gemv_kernel<0, false, false>, grid, 256, smem, st, x, wq, scales, y, M, N, K, out_f32, nullptr, nullptr, 0, 0, 0, mrows, kp,
-                          static_cast<const uint16_t*>(nullptr), static_cast<const uint8_t*>(nullptr),
-                          static_cast<const uint16_t*>(nullptr), 0);
-      });
-    }
-    if (int e = gemv_prepare<1, false>()) return e;
-    return launch(TGEMM_KIND_GEMV_Q4, st, [&] {
-      return pdl_launch(gemv_kernel<1, false, false>, grid, 256, smem, st, x, wq, scales, y, M, N, K, out_f32, nullptr, nullptr, 0, 0, 0, mrows, kp,
-                        nullptr, nullptr, nullptr, 0);
-    });
+    const bool t1 = M <= 8;  // one token tile of 8, else two
+    const uint16_t* x2 = in2.x;
+    const uint8_t* wq2 = in2.wq;
+    const uint16_t* d2 = in2.d;
+    if (fmt == 0 && lora)
+      return t1 ? launch_gemv<0, 1, true, false>(grid, smem, st, x, wq, scales, y, M, N, K, out_f32, u32, lb, r, lb_sn, lb_si, kp, nullptr, nullptr, nullptr, 0)
+                : launch_gemv<0, 2, true, false>(grid, smem, st, x, wq, scales, y, M, N, K, out_f32, u32, lb, r, lb_sn, lb_si, kp, nullptr, nullptr, nullptr, 0);
+    if (fmt == 0 && dual)
+      return t1 ? launch_gemv<0, 1, false, true>(grid, smem, st, x, wq, scales, y, M, N, K, out_f32, nullptr, nullptr, 0, 0, 0, kp, x2, wq2, d2, K2)
+                : launch_gemv<0, 2, false, true>(grid, smem, st, x, wq, scales, y, M, N, K, out_f32, nullptr, nullptr, 0, 0, 0, kp, x2, wq2, d2, K2);
+    if (fmt == 0)
+      return t1 ? launch_gemv<0, 1, false, false>(grid, smem, st, x, wq, scales, y, M, N, K, out_f32, nullptr, nullptr, 0, 0, 0, kp, nullptr, nullptr, nullptr, 0)
+                : launch_gemv<0, 2, false, false>(grid, smem, st, x, wq, scales, y, M, N, K, out_f32, nullptr, nullptr, 0, 0, 0, kp, nullptr, nullptr, nullptr, 0);
+    return t1 ? launch_gemv<1, 1, false, false>(grid, smem, st, x, wq, scales, y, M, N, K, out_f32, nullptr, nullptr, 0, 0, 0, kp, nullptr, nullptr, nullptr, 0)
+              : launch_gemv<1, 2, false, false>(grid, smem, st, x, wq, scales, y, M, N, K, out_f32, nullptr, nullptr, 0, 0, 0, kp, nullptr, nullptr, nullptr, 0);
   }
 
   // ---- tensor-core path
