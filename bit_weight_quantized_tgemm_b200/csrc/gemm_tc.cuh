@@ -168,6 +168,9 @@ __device__ __forceinline__ int tc_slot(const TcParams& p, int c, int t) {
   return c * p.upc >= (t - p.sk_t0) * p.ksteps ? 2 * c : 2 * c + 1;
 }
 constexpr int kTcSlotFloats = kTcRows * kTcTok;
+// The dequant warps prefetch a row's low-rank B values this many stages before the
+// tile's branch stage.
+constexpr int kLoraPrefetchStages = 4;
 
 // A warp-uniform bounded wait: every lane gets the same answer, so the .sync.aligned
 // tcgen05 instructions that follow never run with part of a warp.
@@ -407,6 +410,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         nrow = (ntile / p.tiles_m) * kTcRows + rt;
       }
       sc_next = scale_at(nks, nrow, i + 1 < n_items);
+      if (LORA && valid && ks == (p.kt_main > kLoraPrefetchStages ? p.kt_main - kLoraPrefetchStages : 0)) {
+        // the row's B values for this tile's branch stage -> L1, a few stages ahead
+        if (p.lb_si == 1) {
+          const uint16_t* br = p.lb + static_cast<int64_t>(row) * p.lb_sn;
+          prefetch_l1(br);
+          if (((reinterpret_cast<uintptr_t>(br) & 127) + 2 * p.r) > 128) prefetch_l1(br + 64);
+        } else {
+          for (int ii = part; ii < p.r; ii += kTcDeqParts)
+            prefetch_l1(p.lb + static_cast<int64_t>(ii) * p.lb_si + static_cast<int64_t>(row) * p.lb_sn);
+        }
+      }
       uint32_t o[kC / 2];
       if (!LORA || ks < p.kt_main) {
         // codes from the weight ring (rows past N and k past K arrive zero-filled)
@@ -445,36 +459,35 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           for (int j = 0; j < kWords; ++j) q4_word_to_f16(cw[j], s2, z2, o + 4 * j);
         }
       } else {
-        // low-rank stage: weight-side values [j0, j0 + kC) of [B | B], zero beyond 2R
+        // low-rank stage: weight-side values [j0, j0 + kC) of [B | B], zero beyond 2R and
+        // in each copy's padding (columns r..R-1); a chunk of 8 columns is either all
+        // padding (skipped, warp-uniform), a 16-byte load, or up to 8 element loads
         const int j0 = (ks - p.kt_main) * kTcBK + part * kC;
-        const bool vec = p.lb_si == 1 && (p.lb_sn & 7) == 0 &&
-                         (reinterpret_cast<uintptr_t>(p.lb) & 15) == 0;
 #pragma unroll
-        for (int cq = 0; cq < kC / 8; ++cq) {
-          const int jc = j0 + 8 * cq;
-          const int ic = jc < p.R ? jc : jc - p.R;
-          if (vec && jc < 2 * p.R && ic + 8 <= p.r) {
-            uint4 v = make_uint4(0, 0, 0, 0);
-            if (valid) v = *reinterpret_cast<const uint4*>(p.lb + static_cast<int64_t>(row) * p.lb_sn + ic);
-            o[4 * cq] = v.x;
-            o[4 * cq + 1] = v.y;
-            o[4 * cq + 2] = v.z;
-            o[4 * cq + 3] = v.w;
-            continue;
-          }
+        for (int q = 0; q < kC / 2; ++q) o[q] = 0u;
+        if (j0 < 2 * p.R) {
+          const uint16_t* br = p.lb + static_cast<int64_t>(valid ? row : 0) * p.lb_sn;
+          const bool vec = p.lb_si == 1 && (p.lb_sn & 7) == 0 &&
+                           (reinterpret_cast<uintptr_t>(p.lb) & 15) == 0;
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            uint32_t v2 = 0;
+          for (int cq = 0; cq < kC / 8; ++cq) {
+            const int jc = j0 + 8 * cq;
+            if (jc >= 2 * p.R) break;
+            const int ic = jc < p.R ? jc : jc - p.R;
+            if (ic >= p.r || !valid) continue;
+            if (vec && ic + 8 <= p.r) {
+              const uint4 v = *reinterpret_cast<const uint4*>(br + ic);
+              o[4 * cq] = v.x;
+              o[4 * cq + 1] = v.y;
+              o[4 * cq + 2] = v.z;
+              o[4 * cq + 3] = v.w;
+            } else {
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              const int j = jc + 2 * e + h;
-              const int ii = j < p.R ? j : j - p.R;
-              uint32_t v = 0;
-              if (valid && j < 2 * p.R && ii < p.r)
-                v = p.lb[static_cast<int64_t>(row) * p.lb_sn + static_cast<int64_t>(ii) * p.lb_si];
-              v2 |= v << (16 * h);
+              for (int e = 0; e < 8; ++e)
+                if (ic + e < p.r)
+                  o[4 * cq + e / 2] |= static_cast<uint32_t>(br[static_cast<int64_t>(ic + e) * p.lb_si])
+                                       << (16 * (e & 1));
             }
-            o[4 * cq + e] = v2;
           }
         }
       }
