@@ -99,16 +99,6 @@ __device__ __forceinline__ void q4_bytes_pairs(uint32_t w, int h, uint32_t& lo, 
   hi = lop3_and_or(p >> 4, 0x000F000Fu, 0x43004300u);
 }
 
-// Bulk copy of `bytes` (a multiple of 16, both addresses 16-byte aligned) from global to
-// this CTA's shared memory, completing on `bar`.
-__device__ __forceinline__ void bulk_copy_g2s(uint32_t dst, const void* src, uint32_t bytes,
-                                              uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
-      : "memory");
-}
-
 // DUAL: a second input (x2, wq2, scales2, K2) whose product adds into the same sums.
 // T: token tiles of 8 per pass (1 for up to 8 tokens, 2 for up to 16).
 template <int FMT, int T, bool LORA, bool DUAL>
