@@ -343,13 +343,27 @@ def oracle_sample(items, seconds: float, seed: int = 0):
     return OracleSampler(items).run(seconds, seed)
 
 
+def step_config(world: int, step_flops: float, step_wbytes: float) -> dict:
+    """The workload both arms report (the same object in both JSON lines)."""
+    return {
+        "workload": "mmdit_step: 1536-token ternary 9216x3072, 3072x12288, 12288x3072; "
+                    "rank 4/32/64 branch on 9216x3072; 512-token 4-bit 9728x2560, "
+                    "2560x9728; 3072x3072 ternary GEMV at M=1,4,16",
+        "tokens": 1536, "encoder_tokens": 512, "out_dtype": "bf16",
+        "step_gflop": step_flops / 1e9, "step_weight_mb": step_wbytes / 1e6,
+        "l2": "flushed before every timed step (256 MB write, outside the step events)",
+        "parallelism": f"independent replicas x{world} (weak scaling, no collective)",
+    }
+
+
 def reference_arm(args, world, rank):
     """The oracle as the reference arm: K timed steps, each a bounded sample."""
     if rank != 0:
         return
     from bit_weight_quantized_tgemm_b200 import synth
 
-    sampler = OracleSampler([synth.ALL[n] for n in STEP_ORDER])
+    items = [synth.ALL[n] for n in STEP_ORDER]
+    sampler = OracleSampler(items)
     per_step = max(0.2, 90.0 / max(1, args.steps + args.warmup))
     for i in range(args.warmup):
         sampler.run(per_step, seed=1000 + i)
@@ -368,7 +382,8 @@ def reference_arm(args, world, rank):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * sec / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": "mmdit_step (see bench.py docstring)", "sample": sample},
+        "config": dict(step_config(world, sum(w.flops for w in items), sum(w.weight_bytes for w in items)),
+                       sample=sample),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -542,15 +557,7 @@ def ours(args, world, rank, local):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f16", "data": "synthetic",
-        "config": {
-            "workload": "mmdit_step: 1536-token ternary 9216x3072, 3072x12288, 12288x3072; "
-                        "rank 4/32/64 branch on 9216x3072; 512-token 4-bit 9728x2560, "
-                        "2560x9728; 3072x3072 ternary GEMV at M=1,4,16",
-            "tokens": 1536, "encoder_tokens": 512, "out_dtype": "bf16",
-            "step_gflop": step_flops / 1e9, "step_weight_mb": step_wbytes / 1e6,
-            "l2": "flushed before every timed step (256 MB write, outside the step events)",
-            "parallelism": f"independent replicas x{world} (weak scaling, no collective)",
-        },
+        "config": step_config(world, step_flops, step_wbytes),
         "weight_gbs": world * step_wbytes / (step_ms * 1e-3) / 1e9,
         "e2e": {"value": world * step_flops / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
