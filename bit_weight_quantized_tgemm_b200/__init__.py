@@ -14,4 +14,5 @@ from .binding import (  # noqa: F401
     launch_count, profile_enable, profile_read, ETOOLARGE, NOALLOC_SCRATCH_BYTES,
     gemm_q2_noalloc, gemm_q2_dual, dual_workspace_size, tc_plan, TC_PLAN_KEYS,
     q2_from_gemlite, PACK_ZERO_MISMATCH, PACK_GROUP_MISMATCH, gemm_q2_lora_bt,
+    selftest_wait_timeout,
 )

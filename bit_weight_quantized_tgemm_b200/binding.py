@@ -37,6 +37,7 @@ _SIGS = {
     "q2_from_gemlite": (_i, [_P, _P, _P, _i, _i, _i, _P, _P, _P, _P]),
     "q2_dequant": (_i, [_P, _P, _P, _i, _i, _P]),
     "q4_dequant": (_i, [_P, _P, _P, _i, _i, _P]),
+    "tgemm_selftest_wait_timeout": (_i, [_P]),
     "tgemm_workspace_size": (_sz, [_i, _i, _i, _i, _i]),
     "tgemm_workspace_size_min": (_sz, [_i, _i, _i, _i, _i]),
     "tgemm_q2_dual_workspace_size": (_sz, [_i, _i, _i, _i]),
@@ -189,6 +190,12 @@ def q4_dequant(wq: torch.Tensor, sz: torch.Tensor) -> torch.Tensor:
 
 
 # ---- matmuls --------------------------------------------------------------------------------
+
+def selftest_wait_timeout() -> None:
+    """Launch the failure-detection self test on the current stream: a wait that can never
+    be satisfied gives up after the library's wait limit (1 s) and sets DEVERR_TIMEOUT."""
+    _check(lib().tgemm_selftest_wait_timeout(_stream()), "tgemm_selftest_wait_timeout")
+
 
 def workspace_size(op: int, M: int, N: int, K: int, r: int = 0) -> int:
     return int(lib().tgemm_workspace_size(op, M, N, K, r))

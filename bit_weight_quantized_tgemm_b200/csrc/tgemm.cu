@@ -579,6 +579,22 @@ int run_gemm(int fmt, const uint16_t* x, const uint8_t* wq, const uint16_t* scal
   return hyb ? run_tc(F1{}, Off{}, Off{}, On{}, TGEMM_KIND_TC_Q4) : run_tc(F1{}, Off{}, Off{}, Off{}, TGEMM_KIND_TC_Q4);
 }
 
+// Failure-detection self test: one CTA waits on an mbarrier phase that nothing ever
+// completes.  The library's bounded wait gives up after kWaitLimitNs, records
+// TGEMM_DEVERR_TIMEOUT in the device error word and returns; the context stays usable.
+__global__ void __launch_bounds__(32) selftest_wait_kernel() {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ uint32_t abort_word;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    abort_word = 0u;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  pdl_trigger_and_wait();
+  mbar_wait(smem_u32(&bar), 0u, &abort_word);  // no thread arrives on `bar`
+}
+
 }  // namespace
 }  // namespace tgemm
 
@@ -692,6 +708,13 @@ int q4_dequant(const uint8_t* wq, const uint16_t* sz, float* w, int N, int K, vo
   return launch(TGEMM_KIND_PREP, st, [&] {
     return pdl_launch(q4_dequant_kernel, grid_for(words, 256, di.sms), 256, 0, st, wq, sz, w, words, K);
   });
+}
+
+int tgemm_selftest_wait_timeout(void* stream) {
+  DeviceInfo di;
+  if (int st = current_device_info(&di)) return st;
+  const cudaStream_t st = as_stream(stream);
+  return launch(TGEMM_KIND_PREP, st, [&] { return pdl_launch(selftest_wait_kernel, 1, 32, 0, st); });
 }
 
 size_t tgemm_workspace_size(int op, int M, int N, int K, int r) {

@@ -147,6 +147,16 @@ int q2_dequant(const uint8_t* wq, const uint16_t* d, float* w, int N, int K, voi
 int q4_dequant(const uint8_t* wq, const uint16_t* sz, float* w, int N, int K, void* stream);
 
 /*
+ * tgemm_selftest_wait_timeout -- test hook for failure detection.  Launches one CTA
+ * whose wait (the same bounded mbarrier wait every pipeline of the library uses) can
+ * never be satisfied: after the wait limit (1 s) it gives up, sets TGEMM_DEVERR_TIMEOUT
+ * in the device error word and returns.  Nothing faults, traps or hangs, and the
+ * context stays usable; read and clear the bit with tgemm_device_error.  The pages have
+ * no counterpart: it checks this library's own error reporting.
+ */
+int tgemm_selftest_wait_timeout(void* stream);
+
+/*
  * tgemm_workspace_size -- bytes of workspace the matmul `op` (TGEMM_OP_*) needs for
  * these sizes under the current path setting to run its fastest schedule (0 when it
  * needs none).  On the tensor-core path that schedule may split tiles between CTAs
