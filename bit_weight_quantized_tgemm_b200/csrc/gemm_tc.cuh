@@ -271,6 +271,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     tmem_alloc(smem_u32(tmem_slot), kTcTmemCols);
     tmem_relinquish();
   }
+  __syncwarp();  // reconverge after the single-thread set-up above
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -640,6 +641,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   }
 
   // ------------------------------------------------------------ teardown
+  // Warps 0, 1 and the weight producer run their roles on lane 0 alone; the other lanes
+  // wait here for it, so that every warp reaches the CTA barrier converged (an aligned
+  // barrier must not be executed by part of a warp) and TMEM is released only after the
+  // last MMA has drained.
+  __syncwarp();
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
