@@ -186,8 +186,9 @@ __device__ __forceinline__ uint4 ld_shared_v4(uint32_t saddr) {
   return v;
 }
 
-// Make this thread's generic-proxy shared-memory writes visible to the async proxy
-// (tensor core reads of operands written with st.shared).
+// Order this thread's earlier generic-proxy shared-memory accesses (st.shared writes of
+// operands the tensor core reads, or ld.shared reads of a buffer that a TMA or bulk copy
+// refills next) before later async-proxy accesses to the same memory.
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }

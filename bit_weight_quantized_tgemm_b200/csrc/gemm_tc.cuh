@@ -446,6 +446,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             cw[j + 3] = v.w;
           }
         }
+        // the ring slot is refilled by TMA (the async proxy) once every dequant warp has
+        // released it: order these generic-proxy reads before that write
+        fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(wempty_bar(w));
         ++wcnt;

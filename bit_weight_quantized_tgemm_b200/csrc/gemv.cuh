@@ -337,6 +337,9 @@ __global__ void __launch_bounds__(256, 2) gemv_kernel(
             }
           }
         }
+        // the next pass's bulk copies (the async proxy) overwrite these activations: order
+        // this thread's generic-proxy reads of them before those writes
+        fence_proxy_async_smem();
         __syncthreads();  // everyone is done with this pass's activations
       }
     }
