@@ -215,9 +215,15 @@ LoraDims lora_dims(int r, int K) {
 // Tensor-core schedule (see gemm_tc.cuh): units (tile, 128-k stage), tile-major, in a
 // whole-tile region of floor(tiles / SMs) tiles per CTA and a split region where the
 // remaining tiles' units are cut into equal contiguous ranges, one per CTA.  It is the
-// split form only when it saves more than the split tiles' charge over whole tiles alone.
+// split form only when it saves more than the split tiles' charge over whole tiles alone
+// (a larger charge when the CTAs also run whole tiles).
 constexpr int kDefaultSms = 148;    // sizes workspaces when no device is visible (B200)
 constexpr int kSplitPenalty = 2;    // units a split tile is charged (partial sums + fixup)
+// Next to whole tiles a CTA's split share costs more: writing its partial sums and fixing
+// up shared tiles keeps the epilogue warps from draining the following whole tile, which
+// stalls the MMAs (measured: 4096 tokens x 9216 x 3072 ran 6 % slower split than whole at
+// a 2-unit charge, 1280 tokens with the r = 64 branch ran 5 % faster split).
+constexpr int kHybridPenalty = 8;
 constexpr int kMaxShare = 4;        // CTAs that may share a split tile next to whole tiles
 
 struct TcSchedule {
@@ -252,7 +258,7 @@ TcSchedule tc_schedule(int M, int N, int K, int kt_lora, int sms) {
   if (wf > 0 && (s.num_tiles - wf * sms) * kMaxShare < sms) --wf;
   const int sk_t0 = wf * sms;
   const int upc = ((s.num_tiles - sk_t0) * s.ksteps + sms - 1) / sms;
-  if (wf * s.ksteps + upc + kSplitPenalty >= whole) return s;
+  if (wf * s.ksteps + upc + (wf > 0 ? kHybridPenalty : kSplitPenalty) >= whole) return s;
   s.split = true;
   s.sk_t0 = sk_t0;
   s.upc = upc;

@@ -143,8 +143,8 @@ def _hybrid(op, M, N, K, r=0, K2=0):
     return pl
 
 
-# tiles: 200 (1 wave + 52), 2 x 130 with a ragged token edge, 360 (the 1280-token QKV)
-@pytest.mark.parametrize("M,N,K", [(256, 25600, 2048), (300, 16640, 3072), (1280, 9216, 3072)])
+# tiles: 200 (1 wave + 52), 2 x 104 with ragged token and row edges, 360 (the 1280-token QKV)
+@pytest.mark.parametrize("M,N,K", [(256, 25600, 2048), (300, 13300, 3072), (1280, 9216, 3072)])
 def test_q2_hybrid_vs_whole(oracle, M, N, K):
     _hybrid(tg.OP_Q2, M, N, K)
     prob = synth.q2_problem((21, M, N, K), M, N, K)
@@ -178,7 +178,7 @@ def test_q4_hybrid_vs_whole(oracle):
 
 @pytest.mark.parametrize("r", [4, 32])
 def test_q2_lora_hybrid_vs_whole(oracle, r):
-    M, N, K = 300, 12800, 1152
+    M, N, K = 300, 13300, 3072
     _hybrid(tg.OP_Q2_LORA, M, N, K, r)
     prob = synth.q2_problem((23, M, N, K, r), M, N, K, r=r)
     wq, d, st = oracle.q2_pack(prob.codes, prob.scale)

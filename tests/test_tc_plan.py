@@ -116,7 +116,9 @@ def _form(pl):
     (tg.OP_Q4, 512, 9728, 2560, 0, 0, "split"),      # 152 tiles: 4 left over, cut over all CTAs
     (tg.OP_Q4, 512, 2560, 9728, 0, 0, "split"),      # 40 tiles
     (tg.OP_Q2, 1280, 9216, 3072, 0, 0, "hybrid"),    # 360 tiles: 2 waves + 64
-    (tg.OP_Q2, 4096, 9216, 3072, 0, 0, "hybrid"),    # 1152 tiles: 7 waves + 116
+    (tg.OP_Q2, 4096, 9216, 3072, 0, 0, "whole"),     # 1152 tiles: 7 waves + 116, split saves < its charge
+    (tg.OP_Q2, 1536, 21504, 3072, 0, 0, "whole"),    # 1008 tiles: 6 waves + 120, likewise
+    (tg.OP_Q2, 300, 13300, 3072, 0, 0, "hybrid"),    # 208 tiles: 1 wave + 60, ragged edges
     (tg.OP_Q2_LORA, 1280, 9216, 3072, 32, 0, "hybrid"),
     (tg.OP_Q2, 1536, 3072, 3072, 0, 12288, "split"),  # fused out projection: 144 tiles of 120 stages
     (tg.OP_Q2, 256, 9216, 3072, 0, 0, "split"),      # 72 tiles
