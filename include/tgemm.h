@@ -195,7 +195,10 @@ size_t tgemm_workspace_size_min(int op, int M, int N, int K, int r);
 int tgemm_tc_plan(int op, int M, int N, int K, int r, int K2, int sms, int* plan);
 
 /*
- * tgemm_q2 -- y = x . W^T for Q2_0 weights.
+ * tgemm_q2 -- y = x . W^T for Q2_0 weights, W = (q - 1) * d ("We're Teaching...", "The
+ * lucky break that wasn't luck"; the ternary linears of "A Browser Tab Just Rendered
+ * This Fox...", "The claim").  M <= 16 runs the small-M kernel, larger M the tensor-core
+ * kernel (tgemm_set_path overrides this for tests).
  *   x [M][K] bf16 (16-byte aligned), wq [N][K/4] (16-byte aligned), d [N][K/128] f16
  *   (2-byte aligned), y [M][N] (16-byte aligned), out_dtype TGEMM_OUT_*.
  *   workspace: device memory of tgemm_workspace_size(TGEMM_OP_Q2, M, N, K, 0) bytes, or
@@ -272,7 +275,9 @@ size_t tgemm_q2_dual_workspace_size(int M, int N, int K1, int K2);
 size_t tgemm_q2_dual_workspace_size_min(int M, int N, int K1, int K2);
 
 /*
- * tgemm_q4 -- y = x . W^T for 4-bit group weights.
+ * tgemm_q4 -- y = x . W^T for 4-bit group weights, W = (q - z) * s with the codes unpacked
+ * as in q4_pack ("You Can Now Just Ask...", "The bug that hid in one flipped bit";
+ * "We're Teaching...", "What's left").  Dispatch as for tgemm_q2.
  *   x [M][K] bf16 (16-byte aligned), wq [N][K/2] (16-byte aligned), sz [N][K/64][2] f16
  *   (4-byte aligned), y [M][N] (16-byte aligned), workspace as for tgemm_q2 with
  *   TGEMM_OP_Q4.  Requires M, N >= 1, K % 64 == 0.
