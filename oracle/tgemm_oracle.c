@@ -116,7 +116,11 @@ uint16_t oracle_f64_to_bf16_rne(double v) {
   int lead = e - 1;
   if (lead < -126) lead = -126; /* bf16 subnormals share f32's minimum exponent */
   /* 8 significant bits: units of 2^(lead-7); rint rounds to nearest, ties to even */
+#ifdef ORACLE_PLANT_BF16_TRUNCATE
+  double q = trunc(ldexp(a, 7 - lead));
+#else
   double q = rint(ldexp(a, 7 - lead));
+#endif
   double r = ldexp(q, lead - 7);
   if (r >= 0x1p128) return sign ? 0xFF80u : 0x7F80u;
   float rf = (float)r; /* exact: at most 8 significant bits inside f32's range */
@@ -288,8 +292,13 @@ void oracle_q4_dequant(const uint8_t* wq, const uint16_t* sz, int64_t N, int64_t
   for (int64_t n = 0; n < N; ++n) {
     for (int64_t t = 0; t < K; ++t) {
       float q = (float)q4_code_of(wq[n * (K / 2) + t / 2], t);
-      float sc = oracle_f16_to_f32(sz[(n * (K / 64) + t / 64) * 2 + 0]);
-      float ze = oracle_f16_to_f32(sz[(n * (K / 64) + t / 64) * 2 + 1]);
+#ifdef ORACLE_PLANT_Q4_GROUP32
+      int64_t g = (t / 32) % (K / 64); /* groups of 32 weights, kept inside the row */
+#else
+      int64_t g = t / 64;
+#endif
+      float sc = oracle_f16_to_f32(sz[(n * (K / 64) + g) * 2 + 0]);
+      float ze = oracle_f16_to_f32(sz[(n * (K / 64) + g) * 2 + 1]);
 #ifdef ORACLE_PLANT_Q4_ZERO_SIGN
       float diff = q + ze;
 #else
@@ -337,7 +346,12 @@ void oracle_lora_add_f64(const uint16_t* x, const uint16_t* a, const uint16_t* b
     for (int64_t i = 0; i < r; ++i) {
       double acc = 0.0;
       for (int64_t k = 0; k < K; ++k)
+#ifdef ORACLE_PLANT_LORA_A_TRANSPOSED
+        /* reads A as if it were stored [K][r]; the index stays inside the buffer */
+        acc += (double)oracle_bf16_to_f32(a[k * r + i]) * (double)oracle_bf16_to_f32(x[m * K + k]);
+#else
         acc += (double)oracle_bf16_to_f32(a[i * K + k]) * (double)oracle_bf16_to_f32(x[m * K + k]);
+#endif
       u[m * r + i] = acc;
     }
   }
@@ -346,7 +360,12 @@ void oracle_lora_add_f64(const uint16_t* x, const uint16_t* a, const uint16_t* b
   for (int64_t n = 0; n < N; ++n) {
     for (int64_t m = 0; m < M; ++m) {
       double acc = 0.0;
+#ifdef ORACLE_PLANT_LORA_B_TRANSPOSED
+      /* reads B as if it were stored [r][N]; the index stays inside the buffer */
+      for (int64_t i = 0; i < r; ++i) acc += (double)oracle_bf16_to_f32(b[i * N + n]) * u[m * r + i];
+#else
       for (int64_t i = 0; i < r; ++i) acc += (double)oracle_bf16_to_f32(b[n * r + i]) * u[m * r + i];
+#endif
       y[m * N + n] += acc;
     }
   }

@@ -23,6 +23,10 @@ PLANTS = [
     "ORACLE_PLANT_GEMLITE_NO_TRANSPOSE",  # gemlite bytes read as [N][K/4]
     "ORACLE_PLANT_GEMLITE_ZERO_UNCHECKED",  # zeros == -scales not checked
     "ORACLE_PLANT_GEMLITE_GROUP_INDEX",  # block b takes group b mod (K/g)
+    "ORACLE_PLANT_Q4_GROUP32",        # 4-bit group indexed per 32 instead of per 64 weights
+    "ORACLE_PLANT_BF16_TRUNCATE",     # f64 -> bf16 output truncates instead of rounding
+    "ORACLE_PLANT_LORA_A_TRANSPOSED",  # branch reads A as [K][r]
+    "ORACLE_PLANT_LORA_B_TRANSPOSED",  # branch reads B as [r][N]
 ]
 
 
