@@ -42,6 +42,8 @@ STEP_ORDER = ["mmdit_9216x3072", "gemv_m1", "gemv_m4", "gemv_m16", "mmdit_3072x1
 DOMINANT = ["mmdit_9216x3072", "mmdit_3072x12288", "mmdit_12288x3072"]
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "tc_gemm_q2_mmdit.md")
 TC_SOURCE = os.path.join(ROOT, "bit_weight_quantized_tgemm_b200", "csrc", "gemm_tc.cuh")
+# CPU seconds the reference arm spends over all its steps (warm-up included)
+REFERENCE_SECONDS = 90.0
 
 
 def parse_args():
@@ -364,7 +366,7 @@ def reference_arm(args, world, rank):
 
     items = [synth.ALL[n] for n in STEP_ORDER]
     sampler = OracleSampler(items)
-    per_step = max(0.2, 90.0 / max(1, args.steps + args.warmup))
+    per_step = max(0.2, REFERENCE_SECONDS / max(1, args.steps + args.warmup))
     for i in range(args.warmup):
         sampler.run(per_step, seed=1000 + i)
     fl, sec, samples, cores = 0, 0.0, 0, 1
