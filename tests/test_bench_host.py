@@ -1,10 +1,12 @@
-"""bench.py's reference arm (the CPU oracle) prints the contract's JSON line (no GPU).
+"""bench.py's host logic (no GPU): the reference arm's JSON line, and the roofline's
+traffic figure being dropped once the kernel source no longer matches its ncu capture.
 
-The arm runs on a two-matmul subset of the step with a shortened CPU budget, so that the
+The reference arm runs on a two-matmul subset of the step with a shortened CPU budget, so that the
 line's keys and their consistency are checked in seconds; the full arm differs only in
 the matmuls it samples and the time it spends.
 """
 import argparse
+import hashlib
 import json
 
 import bench
@@ -43,3 +45,25 @@ def test_reference_other_ranks_print_nothing(monkeypatch, capsys):
     monkeypatch.setattr(bench, "REFERENCE_SECONDS", 0.2)
     bench.reference_arm(_args(gpus=2), world=2, rank=1)
     assert capsys.readouterr().out.strip() == ""
+
+
+def test_traffic_follows_the_kernel_source(monkeypatch, tmp_path):
+    src = tmp_path / "kernel.cuh"
+    src.write_bytes(b"// a kernel\n")
+    sha = hashlib.sha256(src.read_bytes()).hexdigest()
+    prof = tmp_path / "profile.md"
+    prof.write_text(f"kernel_source_sha256: {sha}\ntraffic_bytes_per_launch_full: 1234\n")
+    monkeypatch.setattr(bench, "TC_SOURCE", str(src))
+    monkeypatch.setattr(bench, "TRAFFIC_FILE", str(prof))
+    assert bench.ncu_traffic() == (1234.0, None)
+    src.write_bytes(b"// a kernel, changed\n")
+    traffic, note = bench.ncu_traffic()
+    assert traffic is None and note
+    monkeypatch.setattr(bench, "TRAFFIC_FILE", str(tmp_path / "missing.md"))
+    assert bench.ncu_traffic() == (None, None)
+
+
+def test_peaks_come_from_the_measured_file():
+    peaks = bench.load_peaks()
+    assert peaks["hbm_gbs"] > 0 and peaks["tflops_burst"] >= peaks["tflops_sustained"] > 0
+    assert peaks["source"] in ("measured", "fallback")
