@@ -63,7 +63,8 @@ extern "C" {
 #define TGEMM_EARCH      -4 /* the current device is not compute capability 10.0 */
 #define TGEMM_EWORKSPACE -5 /* workspace missing or smaller than tgemm_workspace_size_min() */
 #define TGEMM_ETOOLARGE  -6 /* tgemm_q2_noalloc: the problem needs more scratch than its
-                               built-in buffer (TGEMM_NOALLOC_SCRATCH_BYTES) holds */
+                               built-in buffer (TGEMM_NOALLOC_SCRATCH_BYTES) holds;
+                               q2_from_gemlite: more than 2^31 - 1 transpose tiles */
 
 /* ---- output element types ---------------------------------------------------------- */
 #define TGEMM_OUT_F32  0
@@ -95,10 +96,10 @@ extern "C" {
  *   scale  f32   [N][K/128], the block scales         (4-byte aligned)
  *   wq     uint8 [N][K/4]  out: code k of a row goes to bits 2*(k%4) of byte k/4 (16-byte aligned)
  *   d      f16   [N][K/128] out: scale rounded to f16 (nearest even)  (2-byte aligned)
- *   status uint32 device word, zeroed by the caller; receives TGEMM_PACK_* bits.  A code
- *          above 2 is stored as (code & 3) and sets BAD_CODE; a scale whose f16 value
- *          differs from it sets INEXACT (NONFINITE for inf/NaN).  A caller following the
- *          pages aborts on any nonzero status.
+ *   status uint32 device word (4-byte aligned), zeroed by the caller; receives
+ *          TGEMM_PACK_* bits.  A code above 2 is stored as (code & 3) and sets BAD_CODE;
+ *          a scale whose f16 value differs from it sets INEXACT (NONFINITE for inf/NaN).
+ *          A caller following the pages aborts on any nonzero status.
  *   Requires N >= 1, K >= 128, K % 128 == 0.
  */
 int q2_pack(const uint8_t* codes, const float* scale, uint8_t* wq, uint16_t* d, int N, int K,
@@ -141,7 +142,8 @@ int q4_pack(const uint8_t* codes, const float* s, const float* z, uint8_t* wq, u
 /*
  * q2_dequant / q4_dequant -- the weights a packed matrix stands for, in f32 [N][K]
  * (16-byte aligned): (q - 1) * d, or (q - z) * s computed as two rounded f32 operations.
- * Test hooks: they use the same unpacking as the matmul kernels.
+ * wq 4-byte aligned; d 2-byte, sz 4-byte aligned.  Requires N >= 1 and K a multiple of
+ * 128 (Q2) or 64 (4-bit).  Test hooks: they unpack the codes as the matmul kernels do.
  */
 int q2_dequant(const uint8_t* wq, const uint16_t* d, float* w, int N, int K, void* stream);
 int q4_dequant(const uint8_t* wq, const uint16_t* sz, float* w, int N, int K, void* stream);
@@ -202,8 +204,8 @@ int tgemm_tc_plan(int op, int M, int N, int K, int r, int K2, int sms, int* plan
  *   x [M][K] bf16 (16-byte aligned), wq [N][K/4] (16-byte aligned), d [N][K/128] f16
  *   (2-byte aligned), y [M][N] (16-byte aligned), out_dtype TGEMM_OUT_*.
  *   workspace: device memory of tgemm_workspace_size(TGEMM_OP_Q2, M, N, K, 0) bytes, or
- *   at least tgemm_workspace_size_min() (256-byte aligned; may be NULL when that is 0).  The call overwrites it;
- *   calls sharing a workspace must not overlap on the GPU.
+ *   at least tgemm_workspace_size_min() (256-byte aligned; may be NULL when that is 0).
+ *   The call overwrites it; calls sharing a workspace must not overlap on the GPU.
  *   Requires M, N >= 1, K % 128 == 0.
  */
 int tgemm_q2(const uint16_t* x, const uint8_t* wq, const uint16_t* d, void* y, int M, int N,
