@@ -828,7 +828,7 @@ const char* tgemm_strerror(int status) {
     case TGEMM_ECUDA: return "CUDA runtime or launch failure";
     case TGEMM_EARCH: return "device is not compute capability 10.0 (sm_100)";
     case TGEMM_EWORKSPACE: return "workspace missing or too small";
-    case TGEMM_ETOOLARGE: return "problem needs more scratch than the built-in buffer holds";
+    case TGEMM_ETOOLARGE: return "problem too large for this call (built-in scratch or tile count)";
     default: return "unknown status";
   }
 }

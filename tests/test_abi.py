@@ -39,6 +39,8 @@ def test_strerror_and_version():
     lib = tg.lib()
     assert lib.tgemm_strerror(0) == b"success"
     assert lib.tgemm_strerror(-5) == b"workspace missing or too small"
+    assert lib.tgemm_strerror(-6).startswith(b"problem too large")
+    assert lib.tgemm_strerror(-7) == b"unknown status"
     assert tg.version() >= 100
 
 
