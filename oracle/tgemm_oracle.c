@@ -444,7 +444,12 @@ void oracle_q2_gemm_at(const uint16_t* x, const uint8_t* wq, const uint16_t* d,
           double ui = 0.0;
           for (int64_t k = 0; k < K; ++k)
             ui += (double)oracle_bf16_to_f32(a[i * K + k]) * (double)oracle_bf16_to_f32(x[m * K + k]);
+#ifdef ORACLE_PLANT_SAMPLED_B_TRANSPOSED
+          /* the sampled path alone reads B as [r][N]; the index stays inside the buffer */
+          br += (double)oracle_bf16_to_f32(b[i * N + n]) * ui;
+#else
           br += (double)oracle_bf16_to_f32(b[n * r + i]) * ui;
+#endif
         }
         acc += br;
 #endif

@@ -27,6 +27,7 @@ PLANTS = [
     "ORACLE_PLANT_BF16_TRUNCATE",     # f64 -> bf16 output truncates instead of rounding
     "ORACLE_PLANT_LORA_A_TRANSPOSED",  # branch reads A as [K][r]
     "ORACLE_PLANT_LORA_B_TRANSPOSED",  # branch reads B as [r][N]
+    "ORACLE_PLANT_SAMPLED_B_TRANSPOSED",  # sampled outputs alone read B as [r][N]
 ]
 
 
