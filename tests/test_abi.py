@@ -140,3 +140,20 @@ def test_missing_workspace_is_reported():
         assert st == tg.EWORKSPACE
     finally:
         tg.set_path(prev)
+
+
+def test_no_fallback_without_the_library(monkeypatch, tmp_path):
+    """With libtgemm.so absent and no way to build it, the binding raises: there is no
+    other implementation to fall back to."""
+    from bit_weight_quantized_tgemm_b200 import build as pkg_build
+
+    def cannot_build(*a, **k):
+        raise RuntimeError("nvcc unavailable")
+
+    monkeypatch.setattr(binding, "_lib", None)
+    monkeypatch.setattr(pkg_build, "LIB", str(tmp_path / "libtgemm.so"))
+    monkeypatch.setattr(pkg_build, "build", cannot_build)
+    with pytest.raises(RuntimeError):
+        binding.lib()
+    with pytest.raises(RuntimeError):
+        tg.version()
