@@ -118,6 +118,8 @@ __global__ void __launch_bounds__(256, 2) gemv_kernel(
   // the pass's scales of the CTA's rows: Q2 d per unit, 4-bit (s, z) per group
   constexpr int kScl = FMT == 0 ? F::kMaxU * kGvWarps : 2 * F::kMaxU * kGvWarps;
   constexpr int kSclPerThread = kGvRows * kScl / 256;
+  static_assert(kSclPerThread * 256 == kGvRows * kScl,
+                "the 256 threads must stage every scale of a pass, none twice");
   __shared__ uint32_t scl[kGvRows][kScl];
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
