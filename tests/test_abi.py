@@ -126,6 +126,22 @@ def test_argument_errors_return_einval(call):
     lambda L: L.q2_pack(P(8), P(16), P(16), P(16), 4, 128, P(16), None),
     lambda L: L.q2_from_gemlite(P(16), P(16), P(16), 4, 256, 128, P(20), P(16), P(16), None),
     lambda L: L.q2_from_gemlite(P(16), P(18), P(16), 4, 256, 128, P(16), P(16), P(16), None),
+    # the branch factors: a 4-byte, b (or bt) 2-byte aligned
+    lambda L: L.tgemm_q2_lora(P(16), P(16), P(16), P(18), P(16), 4, P(16), 4, 4, 128, 0, P(256), 1 << 20, None),
+    lambda L: L.tgemm_q2_lora(P(16), P(16), P(16), P(16), P(17), 4, P(16), 4, 4, 128, 0, P(256), 1 << 20, None),
+    lambda L: L.tgemm_q2_lora_bt(P(16), P(16), P(16), P(16), P(17), 4, P(16), 4, 4, 128, 0, P(256), 1 << 20, None),
+    # the second input of a split projection
+    lambda L: L.tgemm_q2_dual(P(16), P(16), P(16), 128, P(24), P(16), P(16), 128, P(16), 4, 4, 0, P(256), 1 << 20, None),
+    lambda L: L.tgemm_q2_dual(P(16), P(16), P(16), 128, P(16), P(16), P(17), 128, P(16), 4, 4, 0, P(256), 1 << 20, None),
+    # a workspace that is large enough but not 256-byte aligned (tensor-core path, M = 64)
+    lambda L: L.tgemm_q2(P(16), P(16), P(16), P(16), 64, 64, 128, 0, P(128), 1 << 20, None),
+    # 4-bit pack: s, and the status word
+    lambda L: L.q4_pack(P(16), P(18), P(16), P(16), P(16), 4, 64, P(16), None),
+    lambda L: L.q4_pack(P(16), P(16), P(16), P(16), P(16), 4, 64, P(18), None),
+    # the dequant hooks: wq 4-byte, w 16-byte, sz 4-byte
+    lambda L: L.q2_dequant(P(18), P(16), P(16), 4, 128, None),
+    lambda L: L.q2_dequant(P(16), P(16), P(24), 4, 128, None),
+    lambda L: L.q4_dequant(P(16), P(18), P(16), 4, 64, None),
 ])
 def test_misaligned_pointers_return_ealign(call):
     assert call(tg.lib()) == tg.EALIGN
