@@ -113,6 +113,18 @@ P = ctypes.c_void_p
     lambda L: L.q2_from_gemlite(P(16), P(16), P(16), 4, 256, 2, P(16), P(16), P(16), None),
     lambda L: L.q2_from_gemlite(P(16), P(16), P(16), 0, 256, 128, P(16), P(16), P(16), None),
     lambda L: L.q2_from_gemlite(P(16), None, P(16), 4, 256, 128, P(16), P(16), P(16), None),
+    # B given transposed: no A, r out of range
+    lambda L: L.tgemm_q2_lora_bt(P(16), P(16), P(16), None, P(16), 4, P(16), 4, 4, 128, 0, P(256), 1 << 20, None),
+    lambda L: L.tgemm_q2_lora_bt(P(16), P(16), P(16), P(16), P(16), 0, P(16), 4, 4, 128, 0, P(256), 1 << 20, None),
+    # split projection: K2 not a multiple of 128, K2 = 0, a missing second input
+    lambda L: L.tgemm_q2_dual(P(16), P(16), P(16), 128, P(16), P(16), P(16), 100, P(16), 4, 4, 0, P(256), 1 << 20, None),
+    lambda L: L.tgemm_q2_dual(P(16), P(16), P(16), 128, P(16), P(16), P(16), 0, P(16), 4, 4, 0, P(256), 1 << 20, None),
+    lambda L: L.tgemm_q2_dual(P(16), P(16), P(16), 128, None, P(16), P(16), 128, P(16), 4, 4, 0, P(256), 1 << 20, None),
+    # the dequant hooks and the no-allocation call
+    lambda L: L.q4_dequant(P(16), P(16), P(16), 4, 96, None),
+    lambda L: L.q2_dequant(P(16), P(16), P(16), 0, 128, None),
+    lambda L: L.tgemm_q2_noalloc(P(16), P(16), P(16), P(16), 0, 4, 128, 0, None),
+    lambda L: L.tgemm_q2_noalloc(P(16), P(16), None, P(16), 4, 4, 128, 0, None),
 ])
 def test_argument_errors_return_einval(call):
     assert call(tg.lib()) == tg.EINVAL
@@ -173,3 +185,24 @@ def test_no_fallback_without_the_library(monkeypatch, tmp_path):
         binding.lib()
     with pytest.raises(RuntimeError):
         tg.version()
+
+
+def test_noalloc_refuses_large_problems_on_the_host():
+    """The no-allocation call rejects a problem whose f16 copy of x exceeds its built-in
+    buffer before touching the device (2048 x 12288 x 2 bytes = 48 MiB > 40 MiB)."""
+    prev = tg.set_path(tg.PATH_AUTO)
+    try:
+        st = tg.lib().tgemm_q2_noalloc(P(16), P(16), P(16), P(16), 2048, 64, 12288, 0, None)
+        assert st == tg.ETOOLARGE
+    finally:
+        tg.set_path(prev)
+
+
+def test_profile_read_rejects_unknown_kinds():
+    import ctypes as C
+
+    ms, n = C.c_double(), C.c_int64()
+    L = tg.lib()
+    assert L.tgemm_profile_read(6, C.byref(ms), C.byref(n), 0) == tg.EINVAL
+    assert L.tgemm_profile_read(-1, C.byref(ms), C.byref(n), 0) == tg.EINVAL
+    assert L.tgemm_profile_read(0, None, C.byref(n), 0) == tg.EINVAL
