@@ -38,6 +38,7 @@ _SIGS = {
     "q2_dequant": (_i, [_P, _P, _P, _i, _i, _P]),
     "q4_dequant": (_i, [_P, _P, _P, _i, _i, _P]),
     "tgemm_selftest_wait_timeout": (_i, [_P]),
+    "tgemm_selftest_bad_launch": (_i, [_P]),
     "tgemm_workspace_size": (_sz, [_i, _i, _i, _i, _i]),
     "tgemm_workspace_size_min": (_sz, [_i, _i, _i, _i, _i]),
     "tgemm_q2_dual_workspace_size": (_sz, [_i, _i, _i, _i]),

@@ -60,10 +60,6 @@ inline size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
 
-inline int launch_status() {
-  return cudaGetLastError() == cudaSuccess ? TGEMM_OK : TGEMM_ECUDA;
-}
-
 // ---- launch accounting and optional per-launch event timing ---------------------------
 
 std::atomic<int64_t> g_launches{0};
@@ -117,15 +113,17 @@ int launch(int kind, cudaStream_t st, Fn&& launch_fn) {
     e = take_event();
     if (b && e) cudaEventRecord(b, st);
   }
+  // The launch's own return value is its status.  The runtime's last-error slot is left
+  // alone: reading it (cudaGetLastError) would clear, and blame this call for, an error
+  // that an earlier, unrelated launch left there.
   const cudaError_t le = launch_fn();
   g_launches.fetch_add(1, std::memory_order_relaxed);
-  const int status = launch_status();
   if (b && e) {
     cudaEventRecord(e, st);
     std::lock_guard<std::mutex> lock(g_prof_mu);
     g_records.push_back({kind, b, e});
   }
-  return le == cudaSuccess ? status : TGEMM_ECUDA;
+  return le == cudaSuccess ? TGEMM_OK : TGEMM_ECUDA;
 }
 
 int grid_for(int64_t work_items, int per_block, int sms) {
@@ -601,6 +599,8 @@ __global__ void __launch_bounds__(32) selftest_wait_kernel() {
   mbar_wait(smem_u32(&bar), 0u, &abort_word);  // no thread arrives on `bar`
 }
 
+__global__ void selftest_noop_kernel() {}
+
 }  // namespace
 }  // namespace tgemm
 
@@ -612,19 +612,60 @@ static __device__ __align__(256) uint8_t g_noalloc_scratch[TGEMM_NOALLOC_SCRATCH
 
 namespace tgemm {
 namespace {
-void* g_noalloc_ptr[kMaxDevices] = {};
+// The buffer's device address, looked up once per device and context.  The address
+// belongs to the context the module was loaded in: after a device reset the primary
+// context (and the module) is created anew, with a new context id, and the address is
+// looked up again.
+struct NoallocScratch {
+  unsigned long long ctx_id = 0;
+  void* ptr = nullptr;
+};
+NoallocScratch g_noalloc[kMaxDevices];
+
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+
+// The current context's unique id (never reused within a process).
+int current_context_id(unsigned long long* id) {
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<CtxGetCurrentFn>(f);
+    f = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(f);
+  });
+  if (!get_current || !get_id) return TGEMM_ECUDA;
+  CUcontext ctx = nullptr;
+  if (get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return TGEMM_ECUDA;
+  if (get_id(ctx, id) != CUDA_SUCCESS) return TGEMM_ECUDA;
+  return TGEMM_OK;
+}
 
 int noalloc_scratch(void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return TGEMM_ECUDA;
+  // No context may be current yet (the runtime creates the primary context lazily);
+  // then the lookup below creates it, and its id is read afterwards.
+  unsigned long long id = 0;
+  const bool have_id = current_context_id(&id) == TGEMM_OK;
   std::lock_guard<std::mutex> lock(g_mu);
-  if (g_noalloc_ptr[dev] == nullptr) {
+  NoallocScratch& s = g_noalloc[dev];
+  if (!have_id || s.ptr == nullptr || s.ctx_id != id) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
       return TGEMM_ECUDA;
-    g_noalloc_ptr[dev] = p;
+    if (!have_id && current_context_id(&id) != TGEMM_OK) return TGEMM_ECUDA;
+    s.ptr = p;
+    s.ctx_id = id;
   }
-  *out = g_noalloc_ptr[dev];
+  *out = s.ptr;
   return TGEMM_OK;
 }
 }  // namespace
@@ -721,6 +762,20 @@ int tgemm_selftest_wait_timeout(void* stream) {
   if (int st = current_device_info(&di)) return st;
   const cudaStream_t st = as_stream(stream);
   return launch(TGEMM_KIND_PREP, st, [&] { return pdl_launch(selftest_wait_kernel, 1, 32, 0, st); });
+}
+
+int tgemm_selftest_bad_launch(void* stream) {
+  DeviceInfo di;
+  if (int st = current_device_info(&di)) return st;
+  const cudaStream_t st = as_stream(stream);
+  // 2048 threads per block is over the 1024 limit: the runtime refuses the launch on the
+  // host, returns the error and leaves it in its last-error slot; nothing reaches the GPU.
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(1);
+  cfg.blockDim = dim3(2048);
+  cfg.stream = st;
+  const cudaError_t le = cudaLaunchKernelEx(&cfg, selftest_noop_kernel);
+  return le == cudaSuccess ? TGEMM_OK : TGEMM_ECUDA;
 }
 
 size_t tgemm_workspace_size(int op, int M, int N, int K, int r) {

@@ -161,14 +161,15 @@ class Workload:
         return self.N * self.K // 4 + self.N * (self.K // 128) * 2
 
 
+# Seeds: one per workload family (0 tiny, 1 GEMV, 2 MMDiT, 3 branch, 4 encoder); every shape
+# of a family draws its own problem from a fresh generator with the family's seed.
 TINY = [Workload("tiny", "q2", 16, 128, 256, seed=0, out_f32=True)]
-GEMV = [Workload(f"gemv_m{m}", "q2", m, 3072, 3072, seed=(1, i),
-                 code_probs=(0.3, 0.4, 0.3)) for i, m in enumerate((1, 4, 16))]
-MMDIT = [Workload(f"mmdit_{n}x{k}", "q2", 1536, n, k, seed=(2, i))
-         for i, (n, k) in enumerate(((9216, 3072), (3072, 12288), (12288, 3072)))]
-LORA = [Workload(f"lora_r{r}", "q2_lora", 1536, 9216, 3072, seed=(3, i), r=r)
-        for i, r in enumerate((4, 32, 64))]
-ENCODER = [Workload("encoder_up", "q4", 512, 9728, 2560, seed=(4, 0)),
-           Workload("encoder_down", "q4", 512, 2560, 9728, seed=(4, 1))]
+GEMV = [Workload(f"gemv_m{m}", "q2", m, 3072, 3072, seed=1,
+                 code_probs=(0.3, 0.4, 0.3)) for m in (1, 4, 16)]
+MMDIT = [Workload(f"mmdit_{n}x{k}", "q2", 1536, n, k, seed=2)
+         for n, k in ((9216, 3072), (3072, 12288), (12288, 3072))]
+LORA = [Workload(f"lora_r{r}", "q2_lora", 1536, 9216, 3072, seed=3, r=r) for r in (4, 32, 64)]
+ENCODER = [Workload("encoder_up", "q4", 512, 9728, 2560, seed=4),
+           Workload("encoder_down", "q4", 512, 2560, 9728, seed=4)]
 
 ALL = {w.name: w for w in TINY + GEMV + MMDIT + LORA + ENCODER}

@@ -159,6 +159,16 @@ int q4_dequant(const uint8_t* wq, const uint16_t* sz, float* w, int N, int K, vo
 int tgemm_selftest_wait_timeout(void* stream);
 
 /*
+ * tgemm_selftest_bad_launch -- test hook for launch-error reporting.  Asks the CUDA
+ * runtime for a launch it refuses on the host (2048 threads in one block) and returns
+ * TGEMM_ECUDA; nothing reaches the GPU.  The refused launch's error is left in the
+ * runtime's last-error slot, as an unrelated caller's failed launch would leave it: the
+ * next matmul call must still return TGEMM_OK, since every call of this library reports
+ * only its own launches' results.  The pages have no counterpart.
+ */
+int tgemm_selftest_bad_launch(void* stream);
+
+/*
  * tgemm_workspace_size -- bytes of workspace the matmul `op` (TGEMM_OP_*) needs for
  * these sizes under the current path setting to run its fastest schedule (0 when it
  * needs none).  On the tensor-core path that schedule may split tiles between CTAs
@@ -248,7 +258,9 @@ int tgemm_q2_lora_bt(const uint16_t* x, const uint8_t* wq, const uint16_t* d, co
  *   TGEMM_ETOOLARGE before launching anything.  The small-M path (M <= 16) needs none.
  *   The first call on a device looks up that device's address of the buffer
  *   (cudaGetSymbolAddress, with that device current); make that first call before any
- *   stream capture.  All calls share the one buffer and it keeps the last call's
+ *   stream capture.  The address is kept per device and context: after a device reset
+ *   (a new primary context, with a new context id) the next call looks it up again, so
+ *   make that call before any capture too.  All calls share the one buffer and it keeps the last call's
  *   contents (nothing in it has to start at zero: every call rewrites what it reads).
  *   Calls that overlap on the GPU -- on different streams, or from different threads --
  *   race on the buffer: serialize them.  Arguments, layouts and errors as tgemm_q2.

@@ -77,3 +77,29 @@ def nan_filled(shape, dtype, pad: int = 64):
 def canary_intact(buf: torch.Tensor, n: int) -> bool:
     tail = buf[n:].float().cpu().numpy()
     return bool(np.all(tail == np.float32(12288.0)))
+
+
+def worst_blocks(got: np.ndarray, ref: np.ndarray, tok: int = 256, rows: int = 32, top: int = 3):
+    """The `top` output blocks (token tile of `tok` x weight rows of `rows`) with the largest
+    relative Frobenius error, as (token tile, row block, rel error) -- a striped failure
+    (one TMEM lane quarter of a tile, one CTA's rows) then shows up by name."""
+    M, N = ref.shape
+    out = []
+    for m0 in range(0, M, tok):
+        for n0 in range(0, N, rows):
+            r = ref[m0:m0 + tok, n0:n0 + rows]
+            e = got[m0:m0 + tok, n0:n0 + rows] - r
+            nr = np.linalg.norm(r)
+            out.append((m0 // tok, n0 // rows, float(np.linalg.norm(e) / nr if nr > 0 else np.linalg.norm(e))))
+    out.sort(key=lambda t: -t[2])
+    return out[:top]
+
+
+def gate_full(got: np.ndarray, ref: np.ndarray, what: str = ""):
+    """gate() over a whole output matrix [M, N]; on failure the message names the worst
+    (256-token tile, 32-row block) pieces."""
+    try:
+        return gate(got, ref, what)
+    except AssertionError as e:
+        blocks = worst_blocks(np.asarray(got, np.float64), np.asarray(ref, np.float64))
+        raise AssertionError(f"{e}; worst (token tile, 32-row block, rel err): {blocks}") from None

@@ -38,3 +38,23 @@ def test_bounded_wait_reports_timeout_and_context_survives(oracle):
             tg.set_path(prev)
         gate_output(y, oracle.q2_gemm(prob.x, wq, d, prob.N), oracle, f"after the timeout, path {path}")
     assert tg.device_error() == 0
+
+
+def test_launch_errors_are_reported_by_the_call_that_made_them(oracle):
+    """A launch the runtime refuses on the host returns TGEMM_ECUDA from that call; the
+    error it leaves behind in the runtime's last-error slot is not charged to the next,
+    valid call, which returns TGEMM_OK and computes correctly."""
+    st = tg.lib().tgemm_selftest_bad_launch(torch.cuda.current_stream().cuda_stream)
+    assert st == tg.ECUDA
+    prob = synth.q2_problem(43, 40, 136, 256)
+    wq, d, _ = oracle.q2_pack(prob.codes, prob.scale)
+    prev = tg.set_path(tg.PATH_AUTO)
+    try:
+        # raises on any status other than TGEMM_OK
+        y = tg.gemm_q2(dev(prob.x, torch.bfloat16), dev(wq, torch.uint8), dev(d, torch.float16),
+                       out_dtype=tg.OUT_F32)
+        torch.cuda.synchronize()
+    finally:
+        tg.set_path(prev)
+    gate_output(y, oracle.q2_gemm(prob.x, wq, d, prob.N), oracle, "after a refused launch")
+    assert tg.device_error() == 0

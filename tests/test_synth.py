@@ -94,3 +94,14 @@ def test_block_size_rules():
         synth.q2_problem(0, 1, 1, 192)
     with pytest.raises(ValueError):
         synth.q4_problem(0, 1, 1, 96)
+
+
+def test_named_workload_seeds():
+    # one seed per family: tiny 0, GEMV 1, MMDiT 2, branch 3, encoder 4
+    want = {"tiny": 0, "gemv_m1": 1, "gemv_m4": 1, "gemv_m16": 1, "mmdit_9216x3072": 2,
+            "mmdit_3072x12288": 2, "mmdit_12288x3072": 2, "lora_r4": 3, "lora_r32": 3,
+            "lora_r64": 3, "encoder_up": 4, "encoder_down": 4}
+    for name, seed in want.items():
+        assert synth.ALL[name].seed == seed, name
+    # the 1-token GEMV input is the first row of the 16-token one (same generator, same order)
+    assert np.array_equal(synth.ALL["gemv_m1"].make().x[0], synth.ALL["gemv_m16"].make().x[0])
