@@ -59,6 +59,8 @@ def parse_args():
                     help="comma-separated subset of the step's matmuls (profiling runs)")
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the end-to-end leg, the small-M stream and the CPU baseline")
+    ap.add_argument("--parts", default="",
+                    help="comma-separated subset of the extra parts to run (default: all)")
     return ap.parse_args()
 
 
@@ -560,8 +562,11 @@ def ours(args, world, rank, local):
     # ---- small-M stream: 64 distinct 3072x3072 weights (160 MB > L2), one graph of 64 GEMVs
     parts = {}
     if extras:
-        for key, fn in (("gemv_stream", gemv_stream), ("dual_out_projection", dual_out_projection),
+        for key, fn in (("gemv_stream", gemv_stream), ("gemv_branch", gemv_branch),
+                        ("dual_out_projection", dual_out_projection),
                         ("token_sweep", token_sweep), ("mmdit_sequence", mmdit_sequence)):
+            if args.parts and key not in args.parts.split(","):
+                continue
             try:
                 parts[key] = fn(tg, torch, stream)
             except Exception as exc:  # report, do not hide
@@ -569,13 +574,22 @@ def ours(args, world, rank, local):
 
     # the small-M roofline proper: back-to-back calls over weights that do not fit in L2
     gs = parts.get("gemv_stream", {})
-    if all(f"m{m}" in gs for m in (1, 4, 16)):
-        us = sum(gs[f"m{m}"]["us_per_call"] for m in (1, 4, 16))
-        wb = 3 * (3072 * 3072 // 4 + 3072 * 24 * 2)
-        roofline_small_m["achieved"] = wb / (us * 1e-6) / 1e9
+    by_shape = {}
+    for key, res in gs.items():
+        if not isinstance(res, dict) or not all(f"m{m}" in res for m in (1, 4, 16)):
+            continue
+        us = sum(res[f"m{m}"]["stream"]["us_per_call"] for m in (1, 4, 16))
+        gbs = 3 * res["weight_mb"] * 1e6 / (us * 1e-6) / 1e9
+        by_shape[key] = {"achieved": gbs, "frac": gbs / peaks["hbm_gbs"],
+                         **{f"m{m}_frac": res[f"m{m}"]["stream"]["weight_gbs"] / peaks["hbm_gbs"]
+                            for m in (1, 4, 16)}}
+    if "q2_3072x3072" in by_shape:
+        roofline_small_m["kernel"] = "gemv_stream_kernel<Q2> (M=1,4,16; 3072x3072), packed-weight bytes"
+        roofline_small_m["achieved"] = by_shape["q2_3072x3072"]["achieved"]
         roofline_small_m["how"] = ("CUDA graph of back-to-back calls at M = 1, 4 and 16, each over its "
                                    "own weight copy (working set >= 4x L2): packed-weight bytes of the "
                                    "three calls / their summed per-call time")
+        roofline_small_m["by_shape"] = by_shape
     if roofline_small_m["achieved"]:
         roofline_small_m["frac"] = roofline_small_m["achieved"] / peaks["hbm_gbs"]
 
@@ -733,53 +747,121 @@ def mmdit_sequence(tg, torch, stream):
     return out
 
 
-def gemv_stream(tg, torch, stream):
-    """Back-to-back small-M calls, replayed from a CUDA graph, rotating through distinct
-    weight copies whose total is at least 4x the L2 size (so weights come from HBM)."""
-    N = K = 3072
-    wbytes = N * K // 4 + N * (K // 128) * 2
-    l2 = torch.cuda.get_device_properties(0).L2_cache_size
-    ncopies = max(64, -(-4 * l2 // wbytes))
-    copies = []
-    g = torch.Generator(device="cuda").manual_seed(123)
-    for _ in range(ncopies):
+def _device_weights(tg, torch, fmt, N, K, g):
+    """One packed weight matrix drawn on the device (codes uniform, scales as the recipe)."""
+    if fmt == 0:
         codes = torch.randint(0, 3, (N, K), dtype=torch.uint8, device="cuda", generator=g)
         scale = (torch.rand(N, K // 128, device="cuda", generator=g) * 0.02).half().float()
-        wq, d, _ = tg.q2_pack(codes, scale)
-        copies.append((wq, d))
-    out = {}
+        wq, sc, _ = tg.q2_pack(codes, scale)
+    else:
+        codes = torch.randint(0, 16, (N, K), dtype=torch.uint8, device="cuda", generator=g)
+        s = (torch.rand(N, K // 64, device="cuda", generator=g) * 0.01).half().float()
+        z = (7 + torch.rand(N, K // 64, device="cuda", generator=g)).half().float()
+        wq, sc, _ = tg.q4_pack(codes, s, z)
+    return wq, sc
+
+
+def _graph_per_call(tg, torch, calls, fn):
+    """Seconds per call of `calls` (argument tuples for fn) replayed from one CUDA graph."""
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        for c in calls[:4]:
+            assert fn(*c, s.cuda_stream) == 0
+        s.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=s):
+            for c in calls:
+                fn(*c, s.cuda_stream)
+    torch.cuda.synchronize()
+    for _ in range(3):
+        graph.replay()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    reps = 10
+    a.record()
+    for _ in range(reps):
+        graph.replay()
+    b.record()
+    torch.cuda.synchronize()
+    del graph
+    return a.elapsed_time(b) / (reps * len(calls)) * 1e-3
+
+
+# Small-M shapes (format, N, K): the GEMV workload's 3072^2, the MMDiT step's large
+# linears, and the 4-bit encoder's up and down projections.
+GEMV_SHAPES = [(0, 3072, 3072), (0, 12288, 3072), (0, 3072, 12288), (0, 21504, 3072),
+               (1, 9728, 2560), (1, 2560, 9728)]
+
+
+def gemv_stream(tg, torch, stream):
+    """Back-to-back small-M calls (M = 1, 4, 16), replayed from a CUDA graph, each call over
+    its own weight copy; the copies total at least 4x the L2 size, so every call reads its
+    weights from HBM.  Per shape: the streaming kernel, and for comparison the per-pass
+    kernel (PATH_SMALL_M_PASS); weight GB/s = packed-weight bytes / time per call."""
+    l2 = torch.cuda.get_device_properties(0).L2_cache_size
     L = tg.lib()
-    for M in (1, 4, 16):
-        x = torch.randn(M, K, device="cuda").bfloat16()
-        y = torch.empty(M, N, device="cuda", dtype=torch.bfloat16)
-        s = torch.cuda.Stream()
-        s.wait_stream(torch.cuda.current_stream())
-        with torch.cuda.stream(s):
-            sh = s.cuda_stream
-            calls = [(x.data_ptr(), wq.data_ptr(), d.data_ptr(), y.data_ptr(), M, N, K,
-                      tg.OUT_BF16, None, 0, sh) for (wq, d) in copies]
-            for c in calls[:4]:
-                assert L.tgemm_q2(*c) == 0
-            s.synchronize()
-            graph = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(graph, stream=s):
-                for c in calls:
-                    L.tgemm_q2(*c)
-        torch.cuda.synchronize()
-        for _ in range(3):
-            graph.replay()
-        torch.cuda.synchronize()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        reps = 10
-        a.record()
-        for _ in range(reps):
-            graph.replay()
-        b.record()
-        torch.cuda.synchronize()
-        per_call = a.elapsed_time(b) / (reps * len(calls)) * 1e-3
-        out[f"m{M}"] = {"us_per_call": per_call * 1e6, "weight_gbs": wbytes / per_call / 1e9,
-                        "copies": ncopies, "working_set_mb": ncopies * wbytes / 1e6}
-        del graph
+    out = {}
+    for fmt, N, K in GEMV_SHAPES:
+        wbytes = N * K // 4 + N * (K // 128) * 2 if fmt == 0 else N * K // 2 + N * (K // 64) * 4
+        ncopies = max(24, -(-4 * l2 // wbytes))
+        g = torch.Generator(device="cuda").manual_seed(123 + N + K)
+        copies = [_device_weights(tg, torch, fmt, N, K, g) for _ in range(ncopies)]
+        fn = L.tgemm_q2 if fmt == 0 else L.tgemm_q4
+        key = f"{'q2' if fmt == 0 else 'q4'}_{N}x{K}"
+        res = {"copies": ncopies, "working_set_mb": ncopies * wbytes / 1e6, "weight_mb": wbytes / 1e6}
+        for M in (1, 4, 16):
+            x = torch.randn(M, K, device="cuda").bfloat16()
+            y = torch.empty(M, N, device="cuda", dtype=torch.bfloat16)
+            calls = [(x.data_ptr(), wq.data_ptr(), sc.data_ptr(), y.data_ptr(), M, N, K,
+                      tg.OUT_BF16, None, 0) for (wq, sc) in copies]
+            row = {}
+            for label, path in (("stream", tg.PATH_AUTO), ("pass", tg.PATH_SMALL_M_PASS)):
+                if label == "pass" and (fmt, N, K) not in ((0, 3072, 3072), (0, 21504, 3072), (1, 9728, 2560)):
+                    continue
+                prev = tg.set_path(path)
+                try:
+                    t = _graph_per_call(tg, torch, calls, fn)
+                finally:
+                    tg.set_path(prev)
+                row[label] = {"us_per_call": t * 1e6, "weight_gbs": wbytes / t / 1e9}
+            pl = tg.gemv_plan(fmt, M, N, K, torch.cuda.get_device_properties(0).multi_processor_count)
+            if pl:
+                row["plan"] = {"C": pl["C"], "clusters": pl["nclus"], "ring": pl["S"]}
+            res[f"m{M}"] = row
+        out[key] = res
+        del copies
+        torch.cuda.empty_cache()
+    return out
+
+
+def gemv_branch(tg, torch, stream):
+    """Small-M calls with the rank-r branch (M = 1, 4, 16 on 9216 x 3072, r = 4, 32, 64):
+    the branch's two preparation kernels plus the per-pass kernel, back to back from a
+    CUDA graph over weight copies totalling >= 4x L2."""
+    N, K = 9216, 3072
+    wbytes = N * K // 4 + N * (K // 128) * 2
+    l2 = torch.cuda.get_device_properties(0).L2_cache_size
+    ncopies = max(24, -(-4 * l2 // wbytes))
+    g = torch.Generator(device="cuda").manual_seed(321)
+    copies = [_device_weights(tg, torch, 0, N, K, g) for _ in range(ncopies)]
+    L = tg.lib()
+    out = {}
+    for r in (4, 32, 64):
+        a = (torch.randn(r, K, device="cuda") * 1e-3).bfloat16()
+        b = (torch.randn(N, r, device="cuda") * 1e-3).bfloat16()
+        for M in (1, 4, 16):
+            x = torch.randn(M, K, device="cuda").bfloat16()
+            y = torch.empty(M, N, device="cuda", dtype=torch.bfloat16)
+            ws = torch.empty(max(tg.workspace_size(tg.OP_Q2_LORA, M, N, K, r), 256),
+                             dtype=torch.uint8, device="cuda")
+            calls = [(x.data_ptr(), wq.data_ptr(), d.data_ptr(), a.data_ptr(), b.data_ptr(), r,
+                      y.data_ptr(), M, N, K, tg.OUT_BF16, ws.data_ptr(), ws.numel())
+                     for (wq, d) in copies]
+            t = _graph_per_call(tg, torch, calls, L.tgemm_q2_lora)
+            out[f"r{r}_m{M}"] = {"us_per_call": t * 1e6, "weight_gbs": wbytes / t / 1e9}
+    del copies
+    torch.cuda.empty_cache()
     return out
 
 

@@ -21,7 +21,7 @@ OK, EINVAL, EALIGN, ECUDA, EARCH, EWORKSPACE, ETOOLARGE = 0, -1, -2, -3, -4, -5,
 NOALLOC_SCRATCH_BYTES = 40 * 1024 * 1024
 OUT_F32, OUT_BF16 = 0, 1
 OP_Q2, OP_Q2_LORA, OP_Q4 = 0, 1, 2
-PATH_AUTO, PATH_SMALL_M, PATH_TENSOR = 0, 1, 2
+PATH_AUTO, PATH_SMALL_M, PATH_TENSOR, PATH_SMALL_M_PASS = 0, 1, 2, 3
 PACK_BAD_CODE, PACK_INEXACT, PACK_NONFINITE = 1, 2, 4
 PACK_ZERO_MISMATCH, PACK_GROUP_MISMATCH = 8, 16
 DEVERR_TIMEOUT = 1
@@ -39,6 +39,7 @@ _SIGS = {
     "q4_dequant": (_i, [_P, _P, _P, _i, _i, _P]),
     "tgemm_selftest_wait_timeout": (_i, [_P]),
     "tgemm_selftest_bad_launch": (_i, [_P]),
+    "tgemm_gemv_plan": (_i, [_i, _i, _i, _i, _i, _P]),
     "tgemm_workspace_size": (_sz, [_i, _i, _i, _i, _i]),
     "tgemm_workspace_size_min": (_sz, [_i, _i, _i, _i, _i]),
     "tgemm_q2_dual_workspace_size": (_sz, [_i, _i, _i, _i]),
@@ -215,6 +216,21 @@ def tc_plan(op: int, M: int, N: int, K: int, r: int = 0, K2: int = 0, sms: int =
     out = (ctypes.c_int * len(TC_PLAN_KEYS))()
     _check(lib().tgemm_tc_plan(op, M, N, K, r, K2, sms, out), "tgemm_tc_plan")
     return dict(zip(TC_PLAN_KEYS, out))
+
+
+GEMV_PLAN_KEYS = ("C", "nclus", "grid", "S", "U", "uq_max", "j_max", "smem", "row_stride",
+                  "xs_stride", "off_x", "off_corr", "off_sc", "off_ring", "off_red", "off_bar")
+
+
+def gemv_plan(fmt: int, M: int, N: int, K: int, sms: int = 148):
+    """The small-M streaming kernel's launch plan (tgemm_gemv_plan), or None when no
+    layout fits and the per-pass kernel serves the call."""
+    out = (ctypes.c_int * len(GEMV_PLAN_KEYS))()
+    st = lib().tgemm_gemv_plan(fmt, M, N, K, sms, out)
+    if st == ETOOLARGE:
+        return None
+    _check(st, "tgemm_gemv_plan")
+    return dict(zip(GEMV_PLAN_KEYS, out))
 
 
 _ws_cache = {}

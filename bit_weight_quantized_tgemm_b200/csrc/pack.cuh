@@ -41,7 +41,9 @@ __global__ void __launch_bounds__(256) q2_pack_kernel(const uint8_t* __restrict_
                                                       uint8_t* __restrict__ wq,
                                                       uint16_t* __restrict__ d, int64_t n_units,
                                                       int64_t n_scales, uint32_t* status) {
-  pdl_trigger_and_wait();
+  // no early trigger: kernels after this one on the stream start only once it has
+  // finished, so they may read the packed weights before their own dependency wait
+  pdl_wait();
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
   const int64_t tid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   const int64_t iters = (n_units > n_scales ? n_units : n_scales);
@@ -89,7 +91,9 @@ __global__ void __launch_bounds__(256) q2_from_gemlite_kernel(
     const float* __restrict__ zero, uint8_t* __restrict__ wq, uint16_t* __restrict__ d, int N,
     int K, int g, int tiles_n, uint32_t* status) {
   __shared__ uint8_t tile[kGlTileI][kGlTileN + 4];
-  pdl_trigger_and_wait();
+  // no early trigger: kernels after this one on the stream start only once it has
+  // finished, so they may read the packed weights before their own dependency wait
+  pdl_wait();
   const int kq = K / 4;
   const int i0 = (static_cast<int>(blockIdx.x) / tiles_n) * kGlTileI;
   const int n0 = (static_cast<int>(blockIdx.x) % tiles_n) * kGlTileN;
@@ -154,7 +158,9 @@ __global__ void __launch_bounds__(256) q4_pack_kernel(const uint8_t* __restrict_
                                                       uint8_t* __restrict__ wq,
                                                       uint16_t* __restrict__ sz, int64_t n_units,
                                                       int64_t n_groups, uint32_t* status) {
-  pdl_trigger_and_wait();
+  // no early trigger: kernels after this one on the stream start only once it has
+  // finished, so they may read the packed weights before their own dependency wait
+  pdl_wait();
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
   const int64_t tid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   const int64_t iters = (n_units > n_groups ? n_units : n_groups);

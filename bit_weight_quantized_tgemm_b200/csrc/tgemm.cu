@@ -15,6 +15,7 @@
 #include "common.cuh"
 #include "gemm_tc.cuh"
 #include "gemv.cuh"
+#include "gemv_stream.cuh"
 #include "pack.cuh"
 
 namespace tgemm {
@@ -187,7 +188,7 @@ int tc_prepare() {
 
 int choose_path(int M) {
   const int p = g_path.load();
-  if (p == TGEMM_PATH_SMALL_M) return TGEMM_PATH_SMALL_M;
+  if (p == TGEMM_PATH_SMALL_M || p == TGEMM_PATH_SMALL_M_PASS) return TGEMM_PATH_SMALL_M;
   if (p == TGEMM_PATH_TENSOR) return TGEMM_PATH_TENSOR;
   return M <= kSmallM ? TGEMM_PATH_SMALL_M : TGEMM_PATH_TENSOR;
 }
@@ -361,6 +362,174 @@ int gemv_prepare() {
   return err == cudaSuccess ? TGEMM_OK : TGEMM_ECUDA;
 }
 
+// ---- small-M streaming kernel: plan and launch ------------------------------------------
+
+constexpr int kGsSmemMax = 232448;  // dynamic shared memory a CTA may use on sm_100
+
+// Clusters of C CTAs that can run at once, one CTA per SM (the launch asks for the whole
+// shared memory so the count reflects the GPCs' SM counts); 0 when unknown.
+template <int FMT, int T>
+int gs_max_clusters(int C) {
+  static std::mutex mu;
+  static int cache[kMaxDevices][kGsMaxCluster + 1] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 0;
+  std::lock_guard<std::mutex> lock(mu);
+  int& v = cache[dev][C];
+  if (v == 0) {
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = static_cast<unsigned>(C);
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(C));
+    cfg.blockDim = dim3(kGsThreads);
+    cfg.dynamicSmemBytes = kGsSmemMax;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, gemv_stream_kernel<FMT, T>, &cfg) != cudaSuccess || n < 1)
+      n = -1;
+    v = n;
+  }
+  return v > 0 ? v : 0;
+}
+
+struct GsPlan {
+  GsParams p;
+  int grid = 0, smem = 0;
+  bool ok = false;
+};
+
+// Shared-memory layout of the streaming kernel for a cluster size C; fills p and returns the
+// bytes (or a value above kGsSmemMax when it does not fit).
+int gs_layout(GsParams& p, int fmt, int T, int C, int nclus, int ring_slots) {
+  const int unit_bytes = fmt == 0 ? 32 : 64;
+  const int n8 = (p.N + 7) / 8;
+  p.C = C;
+  p.nclus = nclus;
+  p.uq_max = (p.U + C - 1) / C;
+  p.j_max = (8 * ((n8 + nclus - 1) / nclus) + kGsTile - 1) / kGsTile;
+  p.S = ring_slots;
+  p.row_stride = p.uq_max * unit_bytes + 16;   // an odd multiple of 16 modulo 128
+  p.xs_stride = p.uq_max * 2 * kGsUnit + 16;  // 16 modulo 128
+  size_t off = 0;
+  p.off_x = 0;
+  off += static_cast<size_t>(8 * T) * p.xs_stride;
+  off = round_up(off, 16);
+  p.off_corr = static_cast<int>(off);
+  off += static_cast<size_t>(p.uq_max) * (fmt == 0 ? 1 : 2) * 16 * 4;
+  off = round_up(off, 16);
+  p.off_sc = static_cast<int>(off);
+  off += static_cast<size_t>(p.j_max) * kGsTile * p.uq_max * (fmt == 0 ? 2 : 8);
+  off = round_up(off, 128);
+  p.off_ring = static_cast<int>(off);
+  off += static_cast<size_t>(p.S) * kGsTile * p.row_stride;
+  off = round_up(off, 16);
+  p.off_red = static_cast<int>(off);
+  if (C > 1)
+    off += static_cast<size_t>((kGsWarps + C - 1) / C) * kGsRedSlots * C * 32 * 16 * T;
+  off = round_up(off, 8);
+  p.off_bar = static_cast<int>(off);
+  off += static_cast<size_t>(2 * p.S + 2 * kGsWarps * kGsRedSlots) * 8 + 8;
+  return off > static_cast<size_t>(kGsSmemMax) ? kGsSmemMax + 1 : static_cast<int>(off);
+}
+
+// Choose the cluster size (K slices) and ring depth for M <= 16 tokens.  The estimate is
+// the longest warp's work, in (tile, unit) pairs, plus a charge for the cluster reduction;
+// shapes that fit no layout return ok = false (the per-pass kernel then runs).
+template <int FMT, int T>
+GsPlan gs_plan(const uint16_t* x, const uint8_t* wq, const uint16_t* scales, void* y, int M,
+               int N, int K, int out_f32, int sms) {
+  GsPlan best;
+  if (M < 1 || M > 8 * T) return best;
+  GsParams p = {};
+  p.x = x;
+  p.wq = wq;
+  p.scales = scales;
+  p.y = y;
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.out_f32 = out_f32;
+  p.U = (K + kGsUnit - 1) / kGsUnit;
+  int best_cost = 0;
+  for (int C = 1; C <= kGsMaxCluster && C <= p.U; ++C) {
+    int nclus = sms / C;
+    if (C > 1) {
+      const int mx = gs_max_clusters<FMT, T>(C);
+      if (mx > 0 && mx < nclus) nclus = mx;
+    }
+    if (nclus < 1) break;
+    for (int S : {16, 8}) {  // a multiple of the 8 compute warps: slot s has one consumer
+      GsParams q = p;
+      const int bytes = gs_layout(q, FMT, T, C, nclus, S);
+      if (bytes > kGsSmemMax) continue;
+      const int cost = (q.j_max + kGsWarps - 1) / kGsWarps * q.uq_max + (C > 1 ? 2 : 0);
+      if (!best.ok || cost < best_cost) {
+        best.p = q;
+        best.grid = nclus * C;
+        best.smem = bytes;
+        best.ok = true;
+        best_cost = cost;
+      }
+      break;
+    }
+  }
+  return best;
+}
+
+template <int FMT, int T>
+int launch_gemv_stream(const GsPlan& pl, cudaStream_t st) {
+  static std::once_flag once;
+  static cudaError_t err = cudaSuccess;
+  std::call_once(once, [] {
+    err = cudaFuncSetAttribute(gemv_stream_kernel<FMT, T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               kGsSmemMax);
+  });
+  if (err != cudaSuccess) return TGEMM_ECUDA;
+  return launch(FMT == 0 ? TGEMM_KIND_GEMV_Q2 : TGEMM_KIND_GEMV_Q4, st, [&] {
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = static_cast<unsigned>(pl.p.C);
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(pl.grid));
+    cfg.blockDim = dim3(kGsThreads);
+    cfg.dynamicSmemBytes = static_cast<size_t>(pl.smem);
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = pl.p.C > 1 ? 2 : 1;
+    return cudaLaunchKernelEx(&cfg, gemv_stream_kernel<FMT, T>, pl.p);
+  });
+}
+
+// The streaming kernel when it applies (M <= 16, one input, no branch, a layout that fits);
+// returns 1 when it does not apply.
+int try_gemv_stream(int fmt, const uint16_t* x, const uint8_t* wq, const uint16_t* scales, void* y,
+                    int M, int N, int K, int out_f32, int sms, cudaStream_t st) {
+  if (g_path.load() == TGEMM_PATH_SMALL_M_PASS || M > 16) return 1;
+  const bool t1 = M <= 8;
+  if (fmt == 0) {
+    if (t1) {
+      const GsPlan pl = gs_plan<0, 1>(x, wq, scales, y, M, N, K, out_f32, sms);
+      return pl.ok ? launch_gemv_stream<0, 1>(pl, st) : 1;
+    }
+    const GsPlan pl = gs_plan<0, 2>(x, wq, scales, y, M, N, K, out_f32, sms);
+    return pl.ok ? launch_gemv_stream<0, 2>(pl, st) : 1;
+  }
+  if (t1) {
+    const GsPlan pl = gs_plan<1, 1>(x, wq, scales, y, M, N, K, out_f32, sms);
+    return pl.ok ? launch_gemv_stream<1, 1>(pl, st) : 1;
+  }
+  const GsPlan pl = gs_plan<1, 2>(x, wq, scales, y, M, N, K, out_f32, sms);
+  return pl.ok ? launch_gemv_stream<1, 2>(pl, st) : 1;
+}
+
 // One small-M launch: T token tiles of 8 per pass over the weights.
 template <int FMT, int T, bool LORA, bool DUAL>
 int launch_gemv(int grid, size_t smem, cudaStream_t st, const uint16_t* x, const uint8_t* wq,
@@ -429,6 +598,10 @@ int run_gemm(int fmt, const uint16_t* x, const uint8_t* wq, const uint16_t* scal
     if (lora) {
       u32 = reinterpret_cast<float*>(ws + wl.u32);
       if (int e = launch_lora_down(x, la, M, K, r, ld, part, u32, nullptr, st, di.sms)) return e;
+    }
+    if (!lora && !dual) {
+      const int e = try_gemv_stream(fmt, x, wq, scales, y, M, N, K, out_f32, di.sms, st);
+      if (e <= 0) return e;  // launched (TGEMM_OK) or failed
     }
     const int grid = (N + kGvRows - 1) / kGvRows;
     const int mrows = M < 16 ? M : 16;
@@ -810,6 +983,25 @@ int tgemm_tc_plan(int op, int M, int N, int K, int r, int K2, int sms, int* plan
   return TGEMM_OK;
 }
 
+int tgemm_gemv_plan(int fmt, int M, int N, int K, int sms, int* plan) {
+  if (!plan || M < 1 || M > 16 || N < 1 || K < 1 || sms < 1) return TGEMM_EINVAL;
+  if ((fmt != 0 && fmt != 1) || K % (fmt == 0 ? 128 : 64)) return TGEMM_EINVAL;
+  GsPlan pl;
+  if (fmt == 0)
+    pl = M <= 8 ? gs_plan<0, 1>(nullptr, nullptr, nullptr, nullptr, M, N, K, 0, sms)
+                : gs_plan<0, 2>(nullptr, nullptr, nullptr, nullptr, M, N, K, 0, sms);
+  else
+    pl = M <= 8 ? gs_plan<1, 1>(nullptr, nullptr, nullptr, nullptr, M, N, K, 0, sms)
+                : gs_plan<1, 2>(nullptr, nullptr, nullptr, nullptr, M, N, K, 0, sms);
+  if (!pl.ok) return TGEMM_ETOOLARGE;
+  const GsParams& q = pl.p;
+  const int vals[16] = {q.C, q.nclus, pl.grid, q.S, q.U, q.uq_max, q.j_max, pl.smem,
+                        q.row_stride, q.xs_stride, q.off_x, q.off_corr, q.off_sc, q.off_ring,
+                        q.off_red, q.off_bar};
+  for (int i = 0; i < 16; ++i) plan[i] = vals[i];
+  return TGEMM_OK;
+}
+
 int tgemm_q2(const uint16_t* x, const uint8_t* wq, const uint16_t* d, void* y, int M, int N,
              int K, int out_dtype, void* workspace, size_t ws_bytes, void* stream) {
   return run_gemm(0, x, wq, d, nullptr, nullptr, 0, y, M, N, K, out_dtype, workspace, ws_bytes,
@@ -889,7 +1081,8 @@ const char* tgemm_strerror(int status) {
 }
 
 int tgemm_set_path(int path) {
-  if (path != TGEMM_PATH_AUTO && path != TGEMM_PATH_SMALL_M && path != TGEMM_PATH_TENSOR)
+  if (path != TGEMM_PATH_AUTO && path != TGEMM_PATH_SMALL_M && path != TGEMM_PATH_TENSOR &&
+      path != TGEMM_PATH_SMALL_M_PASS)
     return TGEMM_EINVAL;
   return g_path.exchange(path);
 }

@@ -89,6 +89,8 @@ extern "C" {
 #define TGEMM_PATH_AUTO    0 /* M <= 16: small-M kernel; otherwise the tensor-core kernel */
 #define TGEMM_PATH_SMALL_M 1 /* always the small-M (HBM-bound, mma.sync) kernel */
 #define TGEMM_PATH_TENSOR  2 /* always the tcgen05 tensor-core kernel */
+#define TGEMM_PATH_SMALL_M_PASS 3 /* always the small-M path, in its per-pass form only (the
+                                     streaming form is skipped; for comparisons) */
 
 /*
  * q2_pack -- Q2_0 packing ("We're Teaching...", "The lucky break that wasn't luck").
@@ -169,6 +171,18 @@ int tgemm_selftest_wait_timeout(void* stream);
 int tgemm_selftest_bad_launch(void* stream);
 
 /*
+ * tgemm_gemv_plan -- introspection of the small-M streaming kernel's launch plan for a
+ * matmul of format `fmt` (0 Q2_0, 1 4-bit) with M <= 16 tokens on a GPU of `sms` SMs:
+ * plan[0..15] = cluster size C (CTAs splitting K), clusters, grid, ring slots, units of
+ * 128 along K, most units of a CTA, most 16-row tiles of a cluster, shared-memory bytes,
+ * ring row stride, activation row stride, then the offsets of the activations,
+ * correction sums, scales, ring, reduction slots and barriers in shared memory.  The
+ * cluster count is the one a device would run when a device is current, else sms / C.
+ * TGEMM_ETOOLARGE when no layout fits (the per-pass kernel then serves the call).
+ */
+int tgemm_gemv_plan(int fmt, int M, int N, int K, int sms, int* plan);
+
+/*
  * tgemm_workspace_size -- bytes of workspace the matmul `op` (TGEMM_OP_*) needs for
  * these sizes under the current path setting to run its fastest schedule (0 when it
  * needs none).  On the tensor-core path that schedule may split tiles between CTAs
@@ -217,6 +231,13 @@ int tgemm_tc_plan(int op, int M, int N, int K, int r, int K2, int sms, int* plan
  *   at least tgemm_workspace_size_min() (256-byte aligned; may be NULL when that is 0).
  *   The call overwrites it; calls sharing a workspace must not overlap on the GPU.
  *   Requires M, N >= 1, K % 128 == 0.
+ *   Packed weights are read early: for M <= 16 (one input, no branch) the kernel starts
+ *   copying wq and its scales before it waits for the kernels ahead of it on the stream
+ *   (programmatic dependent launch), so that the fetch overlaps their end.  wq and the
+ *   scales must therefore not be written by a matmul call of this library that is still
+ *   ahead on the stream.  Weights written by q2_pack, q4_pack or q2_from_gemlite (which
+ *   let no later kernel start before they finish), by host copies or by other libraries'
+ *   kernels are safe.  x is read only after that wait.
  */
 int tgemm_q2(const uint16_t* x, const uint8_t* wq, const uint16_t* d, void* y, int M, int N,
              int K, int out_dtype, void* workspace, size_t ws_bytes, void* stream);
@@ -294,7 +315,8 @@ size_t tgemm_q2_dual_workspace_size_min(int M, int N, int K1, int K2);
  * "We're Teaching...", "What's left").  Dispatch as for tgemm_q2.
  *   x [M][K] bf16 (16-byte aligned), wq [N][K/2] (16-byte aligned), sz [N][K/64][2] f16
  *   (4-byte aligned), y [M][N] (16-byte aligned), workspace as for tgemm_q2 with
- *   TGEMM_OP_Q4.  Requires M, N >= 1, K % 64 == 0.
+ *   TGEMM_OP_Q4.  Requires M, N >= 1, K % 64 == 0.  For M <= 16, wq and sz are read
+ *   before the wait for the kernels ahead on the stream, under the same rule as tgemm_q2.
  */
 int tgemm_q4(const uint16_t* x, const uint8_t* wq, const uint16_t* sz, void* y, int M, int N,
              int K, int out_dtype, void* workspace, size_t ws_bytes, void* stream);
