@@ -578,13 +578,15 @@ def ours(args, world, rank, local):
     for key, res in gs.items():
         if not isinstance(res, dict) or not all(f"m{m}" in res for m in (1, 4, 16)):
             continue
-        us = sum(res[f"m{m}"]["stream"]["us_per_call"] for m in (1, 4, 16))
+        us = sum(res[f"m{m}"]["auto"]["us_per_call"] for m in (1, 4, 16))
         gbs = 3 * res["weight_mb"] * 1e6 / (us * 1e-6) / 1e9
         by_shape[key] = {"achieved": gbs, "frac": gbs / peaks["hbm_gbs"],
-                         **{f"m{m}_frac": res[f"m{m}"]["stream"]["weight_gbs"] / peaks["hbm_gbs"]
+                         **{f"m{m}_frac": res[f"m{m}"]["auto"]["weight_gbs"] / peaks["hbm_gbs"]
                             for m in (1, 4, 16)}}
     if "q2_3072x3072" in by_shape:
-        roofline_small_m["kernel"] = "gemv_stream_kernel<Q2> (M=1,4,16; 3072x3072), packed-weight bytes"
+        roofline_small_m["kernel"] = ("small-M path as dispatched (gemv_kernel; gemv_stream_kernel for "
+                                      "<= 8 tokens on large one-pass linears), Q2 M=1,4,16 on "
+                                      "3072x3072, packed-weight bytes")
         roofline_small_m["achieved"] = by_shape["q2_3072x3072"]["achieved"]
         roofline_small_m["how"] = ("CUDA graph of back-to-back calls at M = 1, 4 and 16, each over its "
                                    "own weight copy (working set >= 4x L2): packed-weight bytes of the "
@@ -797,8 +799,8 @@ GEMV_SHAPES = [(0, 3072, 3072), (0, 12288, 3072), (0, 3072, 12288), (0, 21504, 3
 def gemv_stream(tg, torch, stream):
     """Back-to-back small-M calls (M = 1, 4, 16), replayed from a CUDA graph, each call over
     its own weight copy; the copies total at least 4x the L2 size, so every call reads its
-    weights from HBM.  Per shape: the streaming kernel, and for comparison the per-pass
-    kernel (PATH_SMALL_M_PASS); weight GB/s = packed-weight bytes / time per call."""
+    weights from HBM.  Per shape: the library's own choice ("auto"), and each form forced
+    (per-pass and streaming kernels); weight GB/s = packed-weight bytes / time per call."""
     l2 = torch.cuda.get_device_properties(0).L2_cache_size
     L = tg.lib()
     out = {}
@@ -816,9 +818,8 @@ def gemv_stream(tg, torch, stream):
             calls = [(x.data_ptr(), wq.data_ptr(), sc.data_ptr(), y.data_ptr(), M, N, K,
                       tg.OUT_BF16, None, 0) for (wq, sc) in copies]
             row = {}
-            for label, path in (("stream", tg.PATH_AUTO), ("pass", tg.PATH_SMALL_M_PASS)):
-                if label == "pass" and (fmt, N, K) not in ((0, 3072, 3072), (0, 21504, 3072), (1, 9728, 2560)):
-                    continue
+            for label, path in (("auto", tg.PATH_AUTO), ("pass", tg.PATH_SMALL_M_PASS),
+                                ("stream", tg.PATH_SMALL_M_STREAM)):
                 prev = tg.set_path(path)
                 try:
                     t = _graph_per_call(tg, torch, calls, fn)
@@ -827,7 +828,7 @@ def gemv_stream(tg, torch, stream):
                 row[label] = {"us_per_call": t * 1e6, "weight_gbs": wbytes / t / 1e9}
             pl = tg.gemv_plan(fmt, M, N, K, torch.cuda.get_device_properties(0).multi_processor_count)
             if pl:
-                row["plan"] = {"C": pl["C"], "clusters": pl["nclus"], "ring": pl["S"]}
+                row["stream_plan"] = {"passes": pl["passes"], "ring": pl["S"], "tiles": pl["j_max"]}
             res[f"m{M}"] = row
         out[key] = res
         del copies

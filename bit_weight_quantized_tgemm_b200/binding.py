@@ -21,7 +21,7 @@ OK, EINVAL, EALIGN, ECUDA, EARCH, EWORKSPACE, ETOOLARGE = 0, -1, -2, -3, -4, -5,
 NOALLOC_SCRATCH_BYTES = 40 * 1024 * 1024
 OUT_F32, OUT_BF16 = 0, 1
 OP_Q2, OP_Q2_LORA, OP_Q4 = 0, 1, 2
-PATH_AUTO, PATH_SMALL_M, PATH_TENSOR, PATH_SMALL_M_PASS = 0, 1, 2, 3
+PATH_AUTO, PATH_SMALL_M, PATH_TENSOR, PATH_SMALL_M_PASS, PATH_SMALL_M_STREAM = 0, 1, 2, 3, 4
 PACK_BAD_CODE, PACK_INEXACT, PACK_NONFINITE = 1, 2, 4
 PACK_ZERO_MISMATCH, PACK_GROUP_MISMATCH = 8, 16
 DEVERR_TIMEOUT = 1
@@ -40,6 +40,7 @@ _SIGS = {
     "tgemm_selftest_wait_timeout": (_i, [_P]),
     "tgemm_selftest_bad_launch": (_i, [_P]),
     "tgemm_gemv_plan": (_i, [_i, _i, _i, _i, _i, _P]),
+    "tgemm_mma_rate": (_i, [_i, _i, _i, _P, _i, _P]),
     "tgemm_workspace_size": (_sz, [_i, _i, _i, _i, _i]),
     "tgemm_workspace_size_min": (_sz, [_i, _i, _i, _i, _i]),
     "tgemm_q2_dual_workspace_size": (_sz, [_i, _i, _i, _i]),
@@ -218,8 +219,8 @@ def tc_plan(op: int, M: int, N: int, K: int, r: int = 0, K2: int = 0, sms: int =
     return dict(zip(TC_PLAN_KEYS, out))
 
 
-GEMV_PLAN_KEYS = ("C", "nclus", "grid", "S", "U", "uq_max", "j_max", "smem", "row_stride",
-                  "xs_stride", "off_x", "off_corr", "off_sc", "off_ring", "off_red", "off_bar")
+GEMV_PLAN_KEYS = ("T", "kp", "passes", "grid", "S", "U", "j_max", "smem", "nbox", "xs_stride",
+                  "off_x", "off_corr", "off_red", "off_acc", "off_sc", "off_ring", "off_bar")
 
 
 def gemv_plan(fmt: int, M: int, N: int, K: int, sms: int = 148):
@@ -231,6 +232,15 @@ def gemv_plan(fmt: int, M: int, N: int, K: int, sms: int = 148):
         return None
     _check(st, "tgemm_gemv_plan")
     return dict(zip(GEMV_PLAN_KEYS, out))
+
+
+def mma_rate(mode: int, n: int = 16, iters: int = 4096) -> float:
+    """Cycles per operation of tgemm_mma_rate's `mode` (averaged over the SMs)."""
+    sms = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+    out = torch.zeros(sms, dtype=torch.int64, device="cuda")
+    _check(lib().tgemm_mma_rate(mode, n, iters, _ptr(out), sms, _stream()), "tgemm_mma_rate")
+    torch.cuda.synchronize()
+    return float(out.double().mean().item()) / iters
 
 
 _ws_cache = {}

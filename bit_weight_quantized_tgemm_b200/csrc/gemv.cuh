@@ -135,23 +135,78 @@ __global__ void __launch_bounds__(256, 2) gemv_kernel(
     fence_mbar_init();
   }
   pdl_trigger();
-  {
-    // the first pass's packed rows and scales -> L2 while the previous kernel finishes
-    // (no data reaches the SM before the wait below)
-    const int64_t rb = FMT == 0 ? K / 4 : K / 2;
-    const int pass_bytes = static_cast<int>(rb < (FMT == 0 ? kp / 4 : kp / 2) ? rb : (FMT == 0 ? kp / 4 : kp / 2));
-    const int lines = (pass_bytes + 127) / 128;
-    for (int i = tid; i < kGvRows * lines; i += blockDim.x) {
-      const int row = n0 + i / lines;
-      if (row < N) prefetch_l2(wq + static_cast<int64_t>(row) * rb + (i % lines) * 128);
+  // Every packed-code load of a pass goes straight into registers: lane (g, c) takes rows g
+  // and g + 8, bytes [8c, 8c + 8) of each of its 32-byte Q2 row-units (or [8c, 8c + 8) and
+  // [32 + 8c, 32 + 8c + 8) of its 64-byte 4-bit row-units).
+  uint32_t wreg[F::kMaxU][2][F::kWords];
+  auto load_codes = [&](const uint8_t* wqq, int64_t row_bytes, int Kq, int u_base, int u_end) {
+#pragma unroll
+    for (int i = 0; i < F::kMaxU; ++i) {
+      const int unit = u_base + warp + kGvWarps * i;
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const int row = n0 + 8 * j + g;
+        const bool ok = unit < u_end && row < N;
+        const uint8_t* base = wqq + static_cast<int64_t>(row) * row_bytes +
+                              static_cast<int64_t>(unit) * F::kUnitBytes;
+        if (FMT == 0) {
+          // codes 32c..32c+31 of the unit (code 1 = weight 0 where there is no row)
+          uint2 a = make_uint2(0x55555555u, 0x55555555u);
+          if (ok) a = __ldg(reinterpret_cast<const uint2*>(base + 8 * c));
+          wreg[i][j][0] = a.x;
+          wreg[i][j][1] = a.y;
+        } else {
+          // codes 16c..16c+15 and 64+16c..64+16c+15; the unit's second 64 codes exist
+          // only where K reaches them
+          const bool ok2 = ok && static_cast<int64_t>(unit) * kGvUnit + 64 < Kq;
+          uint2 a = make_uint2(0u, 0u), b = make_uint2(0u, 0u);
+          if (ok) a = __ldg(reinterpret_cast<const uint2*>(base + 8 * c));
+          if (ok2) b = __ldg(reinterpret_cast<const uint2*>(base + 32 + 8 * c));
+          wreg[i][j][0] = a.x;
+          wreg[i][j][1] = a.y;
+          wreg[i][j][2] = b.x;
+          wreg[i][j][3] = b.y;
+        }
+      }
     }
-    if (tid < kGvRows && n0 + tid < N)
-      prefetch_l2(scales + static_cast<int64_t>(n0 + tid) * (FMT == 0 ? K / 128 : K / 32));
+  };
+  // The pass's scales of the CTA's rows (consecutive threads, consecutive scales) -> shared.
+  auto stage_scales = [&](const uint16_t* sq, int nscale, int u_base, int u_end) {
+    const int s_base = FMT == 0 ? u_base : 2 * u_base;
+    const int s_cnt = FMT == 0 ? u_end - u_base : min(nscale - s_base, 2 * (u_end - u_base));
+    uint32_t sv[kSclPerThread];
+#pragma unroll
+    for (int e = 0; e < kSclPerThread; ++e) {
+      const int it = tid + 256 * e;
+      const int rl = it / s_cnt, si = it - rl * s_cnt;
+      const int n = n0 + rl;
+      sv[e] = 0u;
+      if (rl < kGvRows && n < N) {
+        const int64_t idx = static_cast<int64_t>(n) * nscale + s_base + si;
+        sv[e] = FMT == 0 ? static_cast<uint32_t>(__ldg(sq + idx))
+                         : __ldg(reinterpret_cast<const uint32_t*>(sq) + idx);
+      }
+    }
+#pragma unroll
+    for (int e = 0; e < kSclPerThread; ++e) {
+      const int it = tid + 256 * e;
+      const int rl = it / s_cnt, si = it - rl * s_cnt;
+      if (rl < kGvRows) scl[rl][si] = sv[e];
+    }
+  };
+  // The first pass's codes and scales load before the dependency wait: the packed weights
+  // are not an output of the kernels ahead on the stream, so their trip to memory overlaps
+  // the end of those kernels; only the activations are fetched after the wait.
+  {
+    const int u_end0 = (min(kp, K) + kGvUnit - 1) / kGvUnit;
+    load_codes(wq, FMT == 0 ? K / 4 : K / 2, K, 0, u_end0);
+    stage_scales(scales, FMT == 0 ? K / 128 : K / 64, 0, u_end0);
   }
-  __syncthreads();  // the barrier's initialisation is visible to every thread
+  __syncthreads();  // the barrier's initialisation and the first scales are visible
   pdl_wait();
 
   uint32_t phase = 0;  // completed activation copies (the mbarrier's phase parity)
+  bool first = true;   // the first (token pass, input, k pass) has its weights loaded
   for (int m0 = 0; m0 < M; m0 += kTok) {
     const int mt = min(kTok, M - m0);  // tokens in this pass over the weights
     float acc[T][4];
@@ -192,61 +247,12 @@ __global__ void __launch_bounds__(256, 2) gemv_kernel(
                           (FMT == 0 ? (k0 + kp) / 4 : (k0 + kp) / 2) + (i % lines) * 128);
           }
         }
-        // ---- every packed-code load of this pass, straight into registers
-        uint32_t wreg[F::kMaxU][2][F::kWords];
-#pragma unroll
-        for (int i = 0; i < F::kMaxU; ++i) {
-          const int unit = u_base + warp + kGvWarps * i;
-#pragma unroll
-          for (int j = 0; j < 2; ++j) {
-            const int row = n0 + 8 * j + g;
-            const bool ok = unit < u_end && row < N;
-            const uint8_t* base = wqq + static_cast<int64_t>(row) * row_bytes +
-                                  static_cast<int64_t>(unit) * F::kUnitBytes;
-            if (FMT == 0) {
-              // codes 32c..32c+31 of the unit (code 1 = weight 0 where there is no row)
-              uint2 a = make_uint2(0x55555555u, 0x55555555u);
-              if (ok) a = __ldg(reinterpret_cast<const uint2*>(base + 8 * c));
-              wreg[i][j][0] = a.x;
-              wreg[i][j][1] = a.y;
-            } else {
-              // codes 16c..16c+15 and 64+16c..64+16c+15; the unit's second 64 codes exist
-              // only where K reaches them
-              const bool ok2 = ok && static_cast<int64_t>(unit) * kGvUnit + 64 < Kq;
-              uint2 a = make_uint2(0u, 0u), b = make_uint2(0u, 0u);
-              if (ok) a = __ldg(reinterpret_cast<const uint2*>(base + 8 * c));
-              if (ok2) b = __ldg(reinterpret_cast<const uint2*>(base + 32 + 8 * c));
-              wreg[i][j][0] = a.x;
-              wreg[i][j][1] = a.y;
-              wreg[i][j][2] = b.x;
-              wreg[i][j][3] = b.y;
-            }
-          }
+        // ---- this pass's codes and scales (the very first pass's are already loaded)
+        if (!first) {
+          load_codes(wqq, row_bytes, Kq, u_base, u_end);
+          stage_scales(sq, nscale, u_base, u_end);
         }
-        // ---- the pass's scales (consecutive threads, consecutive scales), then to shared
-        {
-          const int s_base = FMT == 0 ? u_base : 2 * u_base;
-          const int s_cnt = FMT == 0 ? u_end - u_base : min(nscale - s_base, 2 * (u_end - u_base));
-          uint32_t sv[kSclPerThread];
-#pragma unroll
-          for (int e = 0; e < kSclPerThread; ++e) {
-            const int it = tid + 256 * e;
-            const int rl = it / s_cnt, si = it - rl * s_cnt;
-            const int n = n0 + rl;
-            sv[e] = 0u;
-            if (rl < kGvRows && n < N) {
-              const int64_t idx = static_cast<int64_t>(n) * nscale + s_base + si;
-              sv[e] = FMT == 0 ? static_cast<uint32_t>(__ldg(sq + idx))
-                               : __ldg(reinterpret_cast<const uint32_t*>(sq) + idx);
-            }
-          }
-#pragma unroll
-          for (int e = 0; e < kSclPerThread; ++e) {
-            const int it = tid + 256 * e;
-            const int rl = it / s_cnt, si = it - rl * s_cnt;
-            if (rl < kGvRows) scl[rl][si] = sv[e];
-          }
-        }
+        first = false;
         // ---- wait for the activations (bounded); every thread must agree before going on
         const bool got = mbar_wait(bar, phase, abort_flag);
         phase ^= 1u;

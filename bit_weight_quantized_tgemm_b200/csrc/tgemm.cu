@@ -16,6 +16,7 @@
 #include "gemm_tc.cuh"
 #include "gemv.cuh"
 #include "gemv_stream.cuh"
+#include "mma_rate.cuh"
 #include "pack.cuh"
 
 namespace tgemm {
@@ -188,7 +189,8 @@ int tc_prepare() {
 
 int choose_path(int M) {
   const int p = g_path.load();
-  if (p == TGEMM_PATH_SMALL_M || p == TGEMM_PATH_SMALL_M_PASS) return TGEMM_PATH_SMALL_M;
+  if (p == TGEMM_PATH_SMALL_M || p == TGEMM_PATH_SMALL_M_PASS || p == TGEMM_PATH_SMALL_M_STREAM)
+    return TGEMM_PATH_SMALL_M;
   if (p == TGEMM_PATH_TENSOR) return TGEMM_PATH_TENSOR;
   return M <= kSmallM ? TGEMM_PATH_SMALL_M : TGEMM_PATH_TENSOR;
 }
@@ -366,84 +368,55 @@ int gemv_prepare() {
 
 constexpr int kGsSmemMax = 232448;  // dynamic shared memory a CTA may use on sm_100
 
-// Clusters of C CTAs that can run at once, one CTA per SM (the launch asks for the whole
-// shared memory so the count reflects the GPCs' SM counts); 0 when unknown.
-template <int FMT, int T>
-int gs_max_clusters(int C) {
-  static std::mutex mu;
-  static int cache[kMaxDevices][kGsMaxCluster + 1] = {};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 0;
-  std::lock_guard<std::mutex> lock(mu);
-  int& v = cache[dev][C];
-  if (v == 0) {
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = static_cast<unsigned>(C);
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(C));
-    cfg.blockDim = dim3(kGsThreads);
-    cfg.dynamicSmemBytes = kGsSmemMax;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, gemv_stream_kernel<FMT, T>, &cfg) != cudaSuccess || n < 1)
-      n = -1;
-    v = n;
-  }
-  return v > 0 ? v : 0;
-}
-
 struct GsPlan {
   GsParams p;
-  int grid = 0, smem = 0;
+  int smem = 0;
   bool ok = false;
 };
 
-// Shared-memory layout of the streaming kernel for a cluster size C; fills p and returns the
-// bytes (or a value above kGsSmemMax when it does not fit).
-int gs_layout(GsParams& p, int fmt, int T, int C, int nclus, int ring_slots) {
-  const int unit_bytes = fmt == 0 ? 32 : 64;
+// Shared-memory layout of the streaming kernel for `passes` passes over K and `S` ring
+// slots; fills p and returns the bytes.
+size_t gs_layout(GsParams& p, int fmt, int T, int passes, int S) {
+  const int upass = (p.U + passes - 1) / passes;
   const int n8 = (p.N + 7) / 8;
-  p.C = C;
-  p.nclus = nclus;
-  p.uq_max = (p.U + C - 1) / C;
-  p.j_max = (8 * ((n8 + nclus - 1) / nclus) + kGsTile - 1) / kGsTile;
-  p.S = ring_slots;
-  p.row_stride = p.uq_max * unit_bytes + 16;   // an odd multiple of 16 modulo 128
-  p.xs_stride = p.uq_max * 2 * kGsUnit + 16;  // 16 modulo 128
+  p.kp = upass * kGsUnit;
+  p.passes = (p.U + upass - 1) / upass;
+  p.j_max = (8 * ((n8 + p.grid - 1) / p.grid) + kGsRows - 1) / kGsRows;
+  p.S = S;
+  p.nbox = (p.kp / (fmt == 0 ? 4 : 2) + 127) / 128;
+  p.xs_stride = p.kp * 2 + 16;  // 16 modulo 128: ldmatrix rows hit distinct banks
   size_t off = 0;
   p.off_x = 0;
   off += static_cast<size_t>(8 * T) * p.xs_stride;
   off = round_up(off, 16);
   p.off_corr = static_cast<int>(off);
-  off += static_cast<size_t>(p.uq_max) * (fmt == 0 ? 1 : 2) * 16 * 4;
-  off = round_up(off, 16);
-  p.off_sc = static_cast<int>(off);
-  off += static_cast<size_t>(p.j_max) * kGsTile * p.uq_max * (fmt == 0 ? 2 : 8);
-  off = round_up(off, 128);
-  p.off_ring = static_cast<int>(off);
-  off += static_cast<size_t>(p.S) * kGsTile * p.row_stride;
+  off += static_cast<size_t>(upass) * (fmt == 0 ? 1 : 2) * 16 * 4;
   off = round_up(off, 16);
   p.off_red = static_cast<int>(off);
-  if (C > 1)
-    off += static_cast<size_t>((kGsWarps + C - 1) / C) * kGsRedSlots * C * 32 * 16 * T;
+  off += static_cast<size_t>(2) * kGsWarps * 32 * 8 * T * 4;  // two buffers
+  off = round_up(off, 16);
+  p.off_acc = static_cast<int>(off);
+  if (p.passes > 1) off += static_cast<size_t>(p.j_max) * kGsRows * 8 * T * 4;
+  off = round_up(off, 16);
+  p.off_sc = static_cast<int>(off);  // every scale of the CTA's rows: Q2 d, 4-bit (s, z)
+  off += static_cast<size_t>(p.j_max) * kGsRows * p.U * (fmt == 0 ? 2 : 8);
+  off = round_up(off, 1024);
+  p.off_ring = static_cast<int>(off);
+  off += static_cast<size_t>(S) * p.nbox * kGsBoxBytes;
   off = round_up(off, 8);
   p.off_bar = static_cast<int>(off);
-  off += static_cast<size_t>(2 * p.S + 2 * kGsWarps * kGsRedSlots) * 8 + 8;
-  return off > static_cast<size_t>(kGsSmemMax) ? kGsSmemMax + 1 : static_cast<int>(off);
+  off += static_cast<size_t>(2 * S) * 8 + 8;
+  off += 1024;  // slack: the kernel aligns its shared memory to 1024 bytes
+  return off;
 }
 
-// Choose the cluster size (K slices) and ring depth for M <= 16 tokens.  The estimate is
-// the longest warp's work, in (tile, unit) pairs, plus a charge for the cluster reduction;
-// shapes that fit no layout return ok = false (the per-pass kernel then runs).
-template <int FMT, int T>
-GsPlan gs_plan(const uint16_t* x, const uint8_t* wq, const uint16_t* scales, void* y, int M,
-               int N, int K, int out_f32, int sms) {
+// One CTA per SM; the fewest passes over K (each at most 4096 weights, the activations of
+// a pass staged whole) whose layout fits with at least 2 ring slots, and up to 4 slots.
+GsPlan gs_plan(int fmt, const uint16_t* x, const uint8_t* wq, const uint16_t* scales, void* y,
+               int M, int N, int K, int out_f32, int sms) {
   GsPlan best;
-  if (M < 1 || M > 8 * T) return best;
+  if (M < 1 || M > 16) return best;
+  const int T = M <= 8 ? 1 : 2;
   GsParams p = {};
   p.x = x;
   p.wq = wq;
@@ -454,27 +427,17 @@ GsPlan gs_plan(const uint16_t* x, const uint8_t* wq, const uint16_t* scales, voi
   p.K = K;
   p.out_f32 = out_f32;
   p.U = (K + kGsUnit - 1) / kGsUnit;
-  int best_cost = 0;
-  for (int C = 1; C <= kGsMaxCluster && C <= p.U; ++C) {
-    int nclus = sms / C;
-    if (C > 1) {
-      const int mx = gs_max_clusters<FMT, T>(C);
-      if (mx > 0 && mx < nclus) nclus = mx;
-    }
-    if (nclus < 1) break;
-    for (int S : {16, 8}) {  // a multiple of the 8 compute warps: slot s has one consumer
+  p.grid = sms;
+  const int min_passes = (p.U + kGsMaxUW * kGsWarps - 1) / (kGsMaxUW * kGsWarps);
+  for (int passes = min_passes; passes <= p.U; ++passes) {
+    for (int S = 4; S >= 2; --S) {
       GsParams q = p;
-      const int bytes = gs_layout(q, FMT, T, C, nclus, S);
-      if (bytes > kGsSmemMax) continue;
-      const int cost = (q.j_max + kGsWarps - 1) / kGsWarps * q.uq_max + (C > 1 ? 2 : 0);
-      if (!best.ok || cost < best_cost) {
-        best.p = q;
-        best.grid = nclus * C;
-        best.smem = bytes;
-        best.ok = true;
-        best_cost = cost;
-      }
-      break;
+      const size_t bytes = gs_layout(q, fmt, T, passes, S);
+      if (bytes > static_cast<size_t>(kGsSmemMax)) continue;
+      best.p = q;
+      best.smem = static_cast<int>(bytes);
+      best.ok = true;
+      return best;
     }
   }
   return best;
@@ -482,6 +445,12 @@ GsPlan gs_plan(const uint16_t* x, const uint8_t* wq, const uint16_t* scales, voi
 
 template <int FMT, int T>
 int launch_gemv_stream(const GsPlan& pl, cudaStream_t st) {
+  // packed weights as a [N][row bytes] u8 tensor, boxes of 32 rows x 128 bytes, 128-byte swizzle
+  CUtensorMap tm_w;
+  const uint64_t row_bytes = FMT == 0 ? static_cast<uint64_t>(pl.p.K) / 4 : static_cast<uint64_t>(pl.p.K) / 2;
+  if (int e = make_map_2d(&tm_w, pl.p.wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, row_bytes, pl.p.N, 128,
+                          kGsRows, CU_TENSOR_MAP_SWIZZLE_128B))
+    return e;
   static std::once_flag once;
   static cudaError_t err = cudaSuccess;
   std::call_once(once, [] {
@@ -490,44 +459,27 @@ int launch_gemv_stream(const GsPlan& pl, cudaStream_t st) {
   });
   if (err != cudaSuccess) return TGEMM_ECUDA;
   return launch(FMT == 0 ? TGEMM_KIND_GEMV_Q2 : TGEMM_KIND_GEMV_Q4, st, [&] {
-    cudaLaunchAttribute attr[2];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    attr[1].id = cudaLaunchAttributeClusterDimension;
-    attr[1].val.clusterDim.x = static_cast<unsigned>(pl.p.C);
-    attr[1].val.clusterDim.y = 1;
-    attr[1].val.clusterDim.z = 1;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(pl.grid));
-    cfg.blockDim = dim3(kGsThreads);
-    cfg.dynamicSmemBytes = static_cast<size_t>(pl.smem);
-    cfg.stream = st;
-    cfg.attrs = attr;
-    cfg.numAttrs = pl.p.C > 1 ? 2 : 1;
-    return cudaLaunchKernelEx(&cfg, gemv_stream_kernel<FMT, T>, pl.p);
+    return pdl_launch(gemv_stream_kernel<FMT, T>, dim3(static_cast<unsigned>(pl.p.grid)), kGsThreads,
+                      static_cast<size_t>(pl.smem), st, tm_w, pl.p);
   });
 }
 
-// The streaming kernel when it applies (M <= 16, one input, no branch, a layout that fits);
-// returns 1 when it does not apply.
+// The streaming kernel when it applies (M <= 16, one input, no branch, a layout that fits)
+// and is the faster form; returns 1 when it does not apply.  Measured (chained calls over
+// weights larger than L2): it beats the per-pass kernel for up to 8 tokens with all of K
+// in one pass on the large linears (12288 x 3072: 9.5 against 11.3 us; 21504 x 3072: 13.7
+// against 18.7 us; 4-bit 9728 x 2560: 10.4 against 11.7 us), and loses on 3072 x 3072
+// (4.8 against 3.9 us), with several passes, and at 9..16 tokens.
 int try_gemv_stream(int fmt, const uint16_t* x, const uint8_t* wq, const uint16_t* scales, void* y,
                     int M, int N, int K, int out_f32, int sms, cudaStream_t st) {
-  if (g_path.load() == TGEMM_PATH_SMALL_M_PASS || M > 16) return 1;
+  const int path = g_path.load();
+  if (path == TGEMM_PATH_SMALL_M_PASS || M > 16) return 1;
+  const GsPlan pl = gs_plan(fmt, x, wq, scales, y, M, N, K, out_f32, sms);
+  if (!pl.ok) return 1;
+  if (path != TGEMM_PATH_SMALL_M_STREAM && (M > 8 || pl.p.passes > 1 || N < 6144)) return 1;
   const bool t1 = M <= 8;
-  if (fmt == 0) {
-    if (t1) {
-      const GsPlan pl = gs_plan<0, 1>(x, wq, scales, y, M, N, K, out_f32, sms);
-      return pl.ok ? launch_gemv_stream<0, 1>(pl, st) : 1;
-    }
-    const GsPlan pl = gs_plan<0, 2>(x, wq, scales, y, M, N, K, out_f32, sms);
-    return pl.ok ? launch_gemv_stream<0, 2>(pl, st) : 1;
-  }
-  if (t1) {
-    const GsPlan pl = gs_plan<1, 1>(x, wq, scales, y, M, N, K, out_f32, sms);
-    return pl.ok ? launch_gemv_stream<1, 1>(pl, st) : 1;
-  }
-  const GsPlan pl = gs_plan<1, 2>(x, wq, scales, y, M, N, K, out_f32, sms);
-  return pl.ok ? launch_gemv_stream<1, 2>(pl, st) : 1;
+  if (fmt == 0) return t1 ? launch_gemv_stream<0, 1>(pl, st) : launch_gemv_stream<0, 2>(pl, st);
+  return t1 ? launch_gemv_stream<1, 1>(pl, st) : launch_gemv_stream<1, 2>(pl, st);
 }
 
 // One small-M launch: T token tiles of 8 per pass over the weights.
@@ -937,6 +889,29 @@ int tgemm_selftest_wait_timeout(void* stream) {
   return launch(TGEMM_KIND_PREP, st, [&] { return pdl_launch(selftest_wait_kernel, 1, 32, 0, st); });
 }
 
+int tgemm_mma_rate(int mode, int n, int iters, unsigned long long* out, int nout, void* stream) {
+  if (!out || mode < 0 || mode > 5 || iters < 1 || iters > (1 << 20)) return TGEMM_EINVAL;
+  if (mode <= 2 && (n < 16 || n > 256 || n % 16)) return TGEMM_EINVAL;
+  if (!aligned(out, 8)) return TGEMM_EALIGN;
+  DeviceInfo di;
+  if (int st = current_device_info(&di)) return st;
+  if (nout < di.sms) return TGEMM_EINVAL;
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [] {
+    attr_err = cudaFuncSetAttribute(mma_rate_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kRateSmem);
+  });
+  if (attr_err != cudaSuccess) return TGEMM_ECUDA;
+  const cudaStream_t st = as_stream(stream);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(di.sms));
+  cfg.blockDim = dim3(128);
+  cfg.dynamicSmemBytes = kRateSmem;
+  cfg.stream = st;
+  return cudaLaunchKernelEx(&cfg, mma_rate_kernel, mode, n, iters, out) == cudaSuccess ? TGEMM_OK
+                                                                                       : TGEMM_ECUDA;
+}
+
 int tgemm_selftest_bad_launch(void* stream) {
   DeviceInfo di;
   if (int st = current_device_info(&di)) return st;
@@ -986,19 +961,13 @@ int tgemm_tc_plan(int op, int M, int N, int K, int r, int K2, int sms, int* plan
 int tgemm_gemv_plan(int fmt, int M, int N, int K, int sms, int* plan) {
   if (!plan || M < 1 || M > 16 || N < 1 || K < 1 || sms < 1) return TGEMM_EINVAL;
   if ((fmt != 0 && fmt != 1) || K % (fmt == 0 ? 128 : 64)) return TGEMM_EINVAL;
-  GsPlan pl;
-  if (fmt == 0)
-    pl = M <= 8 ? gs_plan<0, 1>(nullptr, nullptr, nullptr, nullptr, M, N, K, 0, sms)
-                : gs_plan<0, 2>(nullptr, nullptr, nullptr, nullptr, M, N, K, 0, sms);
-  else
-    pl = M <= 8 ? gs_plan<1, 1>(nullptr, nullptr, nullptr, nullptr, M, N, K, 0, sms)
-                : gs_plan<1, 2>(nullptr, nullptr, nullptr, nullptr, M, N, K, 0, sms);
+  const GsPlan pl = gs_plan(fmt, nullptr, nullptr, nullptr, nullptr, M, N, K, 0, sms);
   if (!pl.ok) return TGEMM_ETOOLARGE;
   const GsParams& q = pl.p;
-  const int vals[16] = {q.C, q.nclus, pl.grid, q.S, q.U, q.uq_max, q.j_max, pl.smem,
-                        q.row_stride, q.xs_stride, q.off_x, q.off_corr, q.off_sc, q.off_ring,
-                        q.off_red, q.off_bar};
-  for (int i = 0; i < 16; ++i) plan[i] = vals[i];
+  const int vals[17] = {M <= 8 ? 1 : 2, q.kp, q.passes, q.grid, q.S, q.U, q.j_max, pl.smem,
+                        q.nbox, q.xs_stride, q.off_x, q.off_corr, q.off_red, q.off_acc,
+                        q.off_sc, q.off_ring, q.off_bar};
+  for (int i = 0; i < 17; ++i) plan[i] = vals[i];
   return TGEMM_OK;
 }
 
@@ -1082,7 +1051,7 @@ const char* tgemm_strerror(int status) {
 
 int tgemm_set_path(int path) {
   if (path != TGEMM_PATH_AUTO && path != TGEMM_PATH_SMALL_M && path != TGEMM_PATH_TENSOR &&
-      path != TGEMM_PATH_SMALL_M_PASS)
+      path != TGEMM_PATH_SMALL_M_PASS && path != TGEMM_PATH_SMALL_M_STREAM)
     return TGEMM_EINVAL;
   return g_path.exchange(path);
 }

@@ -86,11 +86,12 @@ extern "C" {
 #define TGEMM_OP_Q4      2
 
 /* ---- kernel path selection (tgemm_set_path) --------------------------------------- */
-#define TGEMM_PATH_AUTO    0 /* M <= 16: small-M kernel; otherwise the tensor-core kernel */
-#define TGEMM_PATH_SMALL_M 1 /* always the small-M (HBM-bound, mma.sync) kernel */
+#define TGEMM_PATH_AUTO    0 /* M <= 16: small-M path; otherwise the tensor-core kernel */
+#define TGEMM_PATH_SMALL_M 1 /* always the small-M (mma.sync) path, its form chosen per shape */
 #define TGEMM_PATH_TENSOR  2 /* always the tcgen05 tensor-core kernel */
-#define TGEMM_PATH_SMALL_M_PASS 3 /* always the small-M path, in its per-pass form only (the
-                                     streaming form is skipped; for comparisons) */
+#define TGEMM_PATH_SMALL_M_PASS 3   /* small-M path, per-pass form only (for comparisons) */
+#define TGEMM_PATH_SMALL_M_STREAM 4 /* small-M path, streaming form wherever its layout fits
+                                       (M <= 16, one input, no branch; for tests) */
 
 /*
  * q2_pack -- Q2_0 packing ("We're Teaching...", "The lucky break that wasn't luck").
@@ -171,14 +172,31 @@ int tgemm_selftest_wait_timeout(void* stream);
 int tgemm_selftest_bad_launch(void* stream);
 
 /*
+ * tgemm_mma_rate -- measurement hook behind two design choices (the small-M tile width
+ * and the 8-bit-activation variant); the pages have no counterpart.  One CTA per SM
+ * issues `iters` back-to-back operations of one kind and writes the cycles they took to
+ * out[cta] (device, 8-byte aligned, nout >= the SM count); read after synchronizing.
+ *   mode 0: tcgen05.mma kind::f16 (f16 x f16 -> f32), M = 128, N = n, K = 16, A and B in
+ *           shared memory;  1: the same with A in tensor memory;
+ *   mode 2: tcgen05.mma kind::i8 (s8 x s8 -> s32), M = 128, N = n, K = 32, both in shared
+ *           memory;
+ *   mode 3: tcgen05.ld of 32 lanes x 16 columns per warp (4 warps), each waited for;
+ *   mode 4: warp mma.sync m16n8k16 bf16 -> f32, 5: mma.sync m16n8k32 s8 -> s32, each of
+ *           4 warps running 8 independent accumulator chains (`iters` per warp).
+ * n: 16..256, a multiple of 16 (modes 0-2).  Operands are zeros (or TMEM contents); the
+ * results are not read.
+ */
+int tgemm_mma_rate(int mode, int n, int iters, unsigned long long* out, int nout, void* stream);
+
+/*
  * tgemm_gemv_plan -- introspection of the small-M streaming kernel's launch plan for a
  * matmul of format `fmt` (0 Q2_0, 1 4-bit) with M <= 16 tokens on a GPU of `sms` SMs:
- * plan[0..15] = cluster size C (CTAs splitting K), clusters, grid, ring slots, units of
- * 128 along K, most units of a CTA, most 16-row tiles of a cluster, shared-memory bytes,
- * ring row stride, activation row stride, then the offsets of the activations,
- * correction sums, scales, ring, reduction slots and barriers in shared memory.  The
- * cluster count is the one a device would run when a device is current, else sms / C.
- * TGEMM_ETOOLARGE when no layout fits (the per-pass kernel then serves the call).
+ * plan[0..16] = token tiles of 8 (T), weights per pass over K, passes, grid (one CTA per
+ * SM), ring slots, units of 128 along K, most 32-row tiles of a CTA, shared-memory bytes,
+ * weight boxes (32 rows x 128 bytes) per ring slot, activation row stride, then the
+ * offsets of the activations, correction sums, warp partial sums (two buffers), pass
+ * partial sums, staged scales, ring and barriers in shared memory.  TGEMM_ETOOLARGE when no layout fits (the per-pass
+ * kernel then serves the call).
  */
 int tgemm_gemv_plan(int fmt, int M, int N, int K, int sms, int* plan);
 
@@ -231,9 +249,9 @@ int tgemm_tc_plan(int op, int M, int N, int K, int r, int K2, int sms, int* plan
  *   at least tgemm_workspace_size_min() (256-byte aligned; may be NULL when that is 0).
  *   The call overwrites it; calls sharing a workspace must not overlap on the GPU.
  *   Requires M, N >= 1, K % 128 == 0.
- *   Packed weights are read early: for M <= 16 (one input, no branch) the kernel starts
- *   copying wq and its scales before it waits for the kernels ahead of it on the stream
- *   (programmatic dependent launch), so that the fetch overlaps their end.  wq and the
+ *   Packed weights are read early: for M <= 16 the small-M kernels start loading wq and
+ *   its scales before they wait for the kernels ahead of them on the stream (programmatic
+ *   dependent launch), so that the fetch overlaps the end of those kernels.  wq and the
  *   scales must therefore not be written by a matmul call of this library that is still
  *   ahead on the stream.  Weights written by q2_pack, q4_pack or q2_from_gemlite (which
  *   let no later kernel start before they finish), by host copies or by other libraries'

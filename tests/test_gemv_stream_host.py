@@ -11,9 +11,9 @@ the kernel's description:
   (g+8, 2c), (g+8, 2c+1)) and ldmatrix (lane (g, c) gets row g, columns 2c, 2c+1);
 and checks that the emulated products, minus the correction sums the kernel forms, give
 sum_k (q - 1) d x (Q2_0) and sum_k (q - z) s x (4-bit) for random codes and activations,
-exactly (small integers).  It also checks the launch plan: the clusters' row ranges and
-the CTAs' K slices cover everything once, the ring depth is a multiple of the 8 compute
-warps, and the shared-memory layout fits and does not overlap.
+exactly (small integers).  It also checks the launch plan: the CTAs' row ranges and the
+passes over K cover everything once, the swizzled code reads are conflict-free, and the
+shared-memory layout fits and does not overlap.
 """
 import itertools
 
@@ -139,7 +139,8 @@ def test_fragments_give_the_dequantized_product(fmt):
 
 SHAPES = [(0, 1, 3072, 3072), (0, 4, 3072, 3072), (0, 16, 3072, 3072), (0, 16, 21504, 3072),
           (0, 16, 3072, 12288), (0, 1, 12288, 3072), (1, 16, 9728, 2560), (1, 1, 2560, 9728),
-          (1, 9, 2560, 9728), (0, 3, 136, 256), (1, 5, 100, 320), (0, 16, 1, 128), (1, 2, 7, 64)]
+          (1, 16, 2560, 9728), (1, 9, 2560, 9728), (0, 3, 136, 256), (1, 5, 100, 320),
+          (0, 16, 1, 128), (1, 2, 7, 64), (0, 16, 520, 65536)]
 
 
 @pytest.mark.parametrize("fmt,M,N,K", SHAPES)
@@ -147,40 +148,75 @@ SHAPES = [(0, 1, 3072, 3072), (0, 4, 3072, 3072), (0, 16, 3072, 3072), (0, 16, 2
 def test_plan_covers_rows_and_k_once(fmt, M, N, K, sms):
     pl = tg.gemv_plan(fmt, M, N, K, sms)
     if pl is None:
-        # no layout fits (a whole K slice per CTA is too large on very few SMs): the
-        # per-pass kernel serves the call; never on a full B200
+        # no layout fits (on very few SMs a CTA's rows carry too many scales to stage):
+        # the per-pass kernel serves the call; never on a full B200
         assert sms < 100, (fmt, M, N, K, sms)
         return
-    C, nclus = pl["C"], pl["nclus"]
-    assert 1 <= C <= 8 and pl["grid"] == C * nclus and pl["grid"] <= sms
-    assert pl["S"] in (8, 16)
+    assert pl["grid"] == sms and pl["T"] == (1 if M <= 8 else 2)
+    assert 2 <= pl["S"] <= 4
     U = (K + 127) // 128
-    assert pl["U"] == U and C <= U
-    # K slices: CTA q owns units [q U / C, (q + 1) U / C)
-    slices = [(q * U // C, (q + 1) * U // C) for q in range(C)]
-    assert slices[0][0] == 0 and slices[-1][1] == U
-    assert all(a < b and b == slices[i + 1][0] for i, (a, b) in enumerate(slices[:-1]))
-    assert max(b - a for a, b in slices) <= pl["uq_max"]
-    # row ranges: 8-row aligned, contiguous, covering [0, N)
+    assert pl["U"] == U
+    # passes: kp a multiple of 128 (whole units), at most 4096; the passes cover K once
+    kp, P = pl["kp"], pl["passes"]
+    assert kp % 128 == 0 and kp <= 4096 and P == -(-U // (kp // 128))
+    assert (P - 1) * kp < 128 * U <= P * kp
+    # row ranges: 8-row aligned, contiguous, covering [0, N), at most j_max tiles of 32
     n8 = (N + 7) // 8
-    rows = [(8 * (gi * n8 // nclus), min(N, 8 * ((gi + 1) * n8 // nclus))) for gi in range(nclus)]
+    grid = pl["grid"]
+    rows = [(8 * (c * n8 // grid), min(N, 8 * ((c + 1) * n8 // grid))) for c in range(grid)]
     assert rows[0][0] == 0 and rows[-1][1] == N
     for (a0, a1), (b0, _) in zip(rows, rows[1:]):
         assert a1 == b0 or (a1 == N and b0 >= N)
-    assert max(-(-(b - a) // 16) for a, b in rows) <= pl["j_max"]
+    assert max(-(-max(b - a, 0) // 32) for a, b in rows) <= pl["j_max"]
     # shared memory: regions in order, aligned, inside the budget
-    T = 1 if M <= 8 else 2
-    offs = [pl["off_x"], pl["off_corr"], pl["off_sc"], pl["off_ring"], pl["off_red"], pl["off_bar"]]
-    assert offs == sorted(offs) and pl["off_ring"] % 128 == 0 and pl["off_bar"] % 8 == 0
-    assert pl["off_corr"] >= 8 * T * pl["xs_stride"]
-    assert pl["off_ring"] + pl["S"] * 16 * pl["row_stride"] <= pl["off_red"]
-    assert pl["smem"] <= 232448
-    assert pl["row_stride"] % 32 == 16 and pl["xs_stride"] % 128 == 16
-    unit_bytes = 32 if fmt == 0 else 64
-    assert pl["row_stride"] >= pl["uq_max"] * unit_bytes
-    # bulk copies: 16-byte aligned sources and sizes for every row's slice
+    T = pl["T"]
+    offs = [pl["off_x"], pl["off_corr"], pl["off_red"], pl["off_acc"], pl["off_sc"], pl["off_ring"],
+            pl["off_bar"]]
+    assert offs == sorted(offs) and pl["off_ring"] % 1024 == 0 and pl["off_bar"] % 8 == 0
+    assert pl["off_corr"] >= 8 * T * pl["xs_stride"] and pl["xs_stride"] >= 2 * kp
+    assert pl["off_red"] - pl["off_corr"] >= (kp // 128) * (1 if fmt == 0 else 2) * 16 * 4
+    assert pl["off_acc"] - pl["off_red"] >= 2 * 8 * 32 * 8 * T * 4
+    if P > 1:
+        assert pl["off_sc"] - pl["off_acc"] >= pl["j_max"] * 32 * 8 * T * 4
+    assert pl["off_ring"] - pl["off_sc"] >= pl["j_max"] * 32 * U * (2 if fmt == 0 else 8)
+    code_bytes = kp // 4 if fmt == 0 else kp // 2
+    assert pl["nbox"] == -(-code_bytes // 128)
+    assert pl["off_ring"] + pl["S"] * pl["nbox"] * 32 * 128 <= pl["off_bar"]
+    assert pl["smem"] <= 232448 and pl["smem"] >= pl["off_bar"] + 2 * pl["S"] * 8 + 8 + 1024
+    assert pl["xs_stride"] % 128 == 16
+    # TMA boxes: every box's x coordinate is a multiple of 16 bytes
     row_bytes = K // 4 if fmt == 0 else K // 2
-    for a, b in slices:
-        kend = min(K, 128 * b)
-        size = (kend - 128 * a) // (4 if fmt == 0 else 2)
-        assert size % 16 == 0 and (a * unit_bytes) % 16 == 0 and row_bytes % 16 == 0
+    assert row_bytes % 16 == 0
+    for p_ in range(P):
+        assert all((p_ * code_bytes + 128 * b) % 16 == 0 for b in range(pl["nbox"]))
+
+
+def code_addr(r, w):
+    """Byte offset of 32-bit word w of row r in a slot of 128-byte-swizzled 32 x 128 boxes."""
+    b, o = w >> 5, (w & 31) * 4
+    return b * 4096 + r * 128 + ((((o >> 4) ^ (r & 7)) << 4) | (o & 15))
+
+
+def test_swizzled_code_reads_are_conflict_free_and_in_place():
+    # the 128-byte swizzle moves 16-byte chunk i of row r to chunk i ^ (r % 8)
+    for r in range(32):
+        for w in range(64):
+            a = code_addr(r, w)
+            b, o = w >> 5, (w & 31) * 4
+            assert a // 4096 == b and (a % 4096) // 128 == r
+            assert ((a % 128) >> 4) == ((o >> 4) ^ (r & 7)) and a % 16 == o % 16
+    # one warp's word reads (lane (g, c): row g + 8 r, words uw + c + 4 hw (Q2) or uw + word
+    # (4-bit)) touch 32 distinct banks
+    for fmt in (0, 1):
+        for u in range(8):
+            uw = u * (8 if fmt == 0 else 16)
+            for half, r in itertools.product(range(2 if fmt == 0 else 4), range(4)):
+                addrs = []
+                for g in range(8):
+                    for c in range(4):
+                        w = uw + c + 4 * half
+                        addrs.append(code_addr(g + 8 * r, w))
+                banks = {}
+                for a in addrs:
+                    banks.setdefault((a // 4) % 32, set()).add(a)
+                assert all(len(v) == 1 for v in banks.values()), (fmt, u, half)
