@@ -3,7 +3,7 @@
 // slots while its warps run the products.
 //
 // Work split.  The rows of W are cut into contiguous ranges (multiples of 8 rows), one per
-// CTA, and each range into tiles of 32 rows (two m16 halves of mma.sync m16n8k16).  K is
+// CTA (one or, up to 8 tokens, two CTAs per SM), and each range into tiles of 32 rows (two m16 halves of mma.sync m16n8k16).  K is
 // cut into units of 128 weights and, when the activations of all of K do not fit in
 // shared memory, into passes of `kp` weights.  For each (pass, tile) item every compute
 // warp takes the units u = w, w + 8, ... of the pass, so one warp's products form 2T
@@ -151,11 +151,11 @@ __device__ __forceinline__ void gs_q4_pairs(uint32_t w, uint32_t (&p)[4]) {
 }
 
 // T: token tiles of 8 (1 for up to 8 tokens, 2 for up to 16).
+// Up to 8 tokens two CTAs share an SM (more warps to hide the MMA and load latencies).
 template <int FMT, int T>
-__global__ void __launch_bounds__(kGsThreads, 1)
+__global__ void __launch_bounds__(kGsThreads, T == 1 ? 2 : 1)
     gemv_stream_kernel(const __grid_constant__ CUtensorMap tm_w, const GsParams p) {
   using F = GsFmt<FMT>;
-  constexpr int kTok = 8 * T;
   extern __shared__ __align__(128) uint8_t gs_smem_raw[];
   // 1024-byte alignment: the swizzle pattern of the weight boxes follows address bits 7-9
   uint8_t* gs_smem = reinterpret_cast<uint8_t*>(
@@ -223,10 +223,13 @@ __global__ void __launch_bounds__(kGsThreads, 1)
   const uint32_t slot_bytes = static_cast<uint32_t>(p.nbox * kGsBoxBytes);
   const uint32_t xs = sb + p.off_x;
   float* corr = reinterpret_cast<float*>(gs_smem + p.off_corr);  // [unit of pass][16 tokens]
-  float* red = reinterpret_cast<float*>(gs_smem + p.off_red);    // [warp][lane][2 T 4]
-  float* accs = reinterpret_cast<float*>(gs_smem + p.off_acc);   // [tile][32 rows][kTok]
+  float* red = reinterpret_cast<float*>(gs_smem + p.off_red);    // 2 x [warp][8T values][32 lanes]
+  float* accs = reinterpret_cast<float*>(gs_smem + p.off_acc);   // [tile][8T values][32 lanes]
   // ldmatrix row addresses: lane l -> matrix l / 8 (token block l / 16, slot half (l / 8) % 2)
-  const uint32_t lm_addr = xs + ((lane >> 4) * 8 + (lane & 7)) * p.xs_stride + ((lane >> 3) & 1) * 16;
+  // (only the M real token rows are staged: rows of absent tokens read the last real row,
+  // and the outputs they feed are never stored)
+  const uint32_t lm_addr = xs + min((lane >> 4) * 8 + (lane & 7), p.M - 1) * p.xs_stride +
+                           ((lane >> 3) & 1) * 16;
   const int upass = p.kp / kGsUnit;  // units of a (full) pass
 
   // ---- every scale of this CTA's rows -> shared memory (zero past the rows), before the
@@ -368,11 +371,25 @@ __global__ void __launch_bounds__(kGsThreads, 1)
             for (int e = 0; e < 4; ++e) pacc[hf][tt][e] = 0.f;
 #pragma unroll
         for (int hw = 0; hw < 2; ++hw) {  // the lane's words c and c + 4
-          uint32_t pr[4][8];              // rows g, g + 8, g + 16, g + 24
+          uint32_t wd[4][3];              // rows g, g + 8, g + 16, g + 24: the word >> 0, 6, 12
 #pragma unroll
-          for (int r = 0; r < 4; ++r) gs_q2_pairs(ld_shared_u32(gs_code_addr(slot, g + 8 * r, uw + c + 4 * hw)), pr[r]);
+          for (int r = 0; r < 4; ++r) {
+            wd[r][0] = ld_shared_u32(gs_code_addr(slot, g + 8 * r, uw + c + 4 * hw));
+            wd[r][1] = wd[r][0] >> 6;
+            wd[r][2] = wd[r][0] >> 12;
+          }
 #pragma unroll
           for (int sp = 0; sp < 4; ++sp) {
+            // pairs 2 sp and 2 sp + 1 of each row's word (see gs_q2_pairs)
+            uint32_t pr[4][8];
+#pragma unroll
+            for (int r = 0; r < 4; ++r)
+#pragma unroll
+              for (int q = 2 * sp; q < 2 * sp + 2; ++q) {
+                constexpr uint32_t kMask[3] = {0x00030003u, 0x000C000Cu, 0x00300030u};
+                constexpr uint32_t kMagic[3] = {0x43004300u, 0x42004200u, 0x41004100u};
+                pr[r][q] = lop3_and_or(wd[r][q / 3], kMask[q % 3], kMagic[q % 3]);
+              }
             const uint32_t baddr = lm_addr + (u * kGsUnit + 16 * (4 * hw + sp)) * 2;
             uint32_t b[4];
             if (T == 1) {
@@ -466,33 +483,34 @@ __global__ void __launch_bounds__(kGsThreads, 1)
     __syncwarp();
     if (lane == 0) mbar_arrive(empty_bar(s));
 
-    // ---- add the 8 warps' partial sums (warp order), over the passes; store after the last
+    // ---- add the 8 warps' partial sums (warp order), over the passes; store after the last.
+    // Value i of lane l of warp w sits at redb[(w * 8T + i) * 32 + l]: each store and each
+    // load of a warp touches 32 consecutive words (no bank conflicts).  Thread (i, l) adds
+    // value i of lane l over the warps: for i = (hf T + tt) 4 + e that is row-in-tile
+    // rr = 16 hf + g + 8 (e >> 1) and token m = 8 tt + 2 c + (e & 1), with (g, c) of lane l.
     float* redb = red + (it & 1) * (kGsWarps * 32 * 8 * T);  // two buffers, alternating
-    {
-      float* mine = redb + (warp * 32 + lane) * (8 * T);
 #pragma unroll
-      for (int hf = 0; hf < 2; ++hf)
+    for (int hf = 0; hf < 2; ++hf)
 #pragma unroll
-        for (int tt = 0; tt < T; ++tt)
+      for (int tt = 0; tt < T; ++tt)
 #pragma unroll
-          for (int e = 0; e < 4; ++e) mine[(hf * T + tt) * 4 + e] = acc[hf][tt][e];
-    }
+        for (int e = 0; e < 4; ++e)
+          redb[(warp * 8 * T + (hf * T + tt) * 4 + e) * 32 + lane] = acc[hf][tt][e];
     named_barrier_sync(1, kGsWarps * 32);
     const bool last = pass == p.passes - 1;
-    for (int o = tid; o < kGsRows * kTok; o += kGsWarps * 32) {
-      // output o: token m, row-in-tile rr (rows fastest: consecutive threads store
-      // consecutive n); held by lane (g, c) of each warp at (hf, tt, e) with
-      // rr = 16 hf + g + 8 (e >> 1), m = 8 tt + 2 c + (e & 1)
-      const int m = o / kGsRows, rr = o - m * kGsRows;
-      const int hf = rr >> 4, gg = rr & 7, e = ((rr >> 3) & 1) * 2 + (m & 1);
-      const int tt = m >> 3, cc = (m & 7) >> 1;
-      const int ln = gg * 4 + cc;
-      float v = pass > 0 ? accs[(t * kGsRows + rr) * kTok + m] : 0.f;
 #pragma unroll
-      for (int w = 0; w < kGsWarps; ++w) v += redb[(w * 32 + ln) * (8 * T) + (hf * T + tt) * 4 + e];
+    for (int rep = 0; rep < T; ++rep) {
+      const int o = tid + rep * kGsWarps * 32;  // (value i, lane l) = (o / 32, o % 32)
+      const int i = o >> 5, l = o & 31;
+      float v = pass > 0 ? accs[(t * 8 * T + i) * 32 + l] : 0.f;
+#pragma unroll
+      for (int w = 0; w < kGsWarps; ++w) v += redb[(w * 8 * T + i) * 32 + l];
+      const int hf = i / (4 * T), tt = (i >> 2) % T, e = i & 3;
+      const int rr = 16 * hf + (l >> 2) + 8 * (e >> 1);
+      const int m = 8 * tt + 2 * (l & 3) + (e & 1);
       const int n = row0 + rr;
       if (!last) {
-        accs[(t * kGsRows + rr) * kTok + m] = v;
+        accs[(t * 8 * T + i) * 32 + l] = v;
       } else if (n < r1 && m < p.M) {
         if (p.out_f32)
           reinterpret_cast<float*>(p.y)[static_cast<int64_t>(m) * p.N + n] = v;

@@ -367,6 +367,7 @@ int gemv_prepare() {
 // ---- small-M streaming kernel: plan and launch ------------------------------------------
 
 constexpr int kGsSmemMax = 232448;  // dynamic shared memory a CTA may use on sm_100
+constexpr int kGsSmemHalf = 115712; // the most each of two CTAs on one SM may use
 
 struct GsPlan {
   GsParams p;
@@ -387,7 +388,7 @@ size_t gs_layout(GsParams& p, int fmt, int T, int passes, int S) {
   p.xs_stride = p.kp * 2 + 16;  // 16 modulo 128: ldmatrix rows hit distinct banks
   size_t off = 0;
   p.off_x = 0;
-  off += static_cast<size_t>(8 * T) * p.xs_stride;
+  off += static_cast<size_t>(p.M) * p.xs_stride;  // the M real token rows
   off = round_up(off, 16);
   p.off_corr = static_cast<int>(off);
   off += static_cast<size_t>(upass) * (fmt == 0 ? 1 : 2) * 16 * 4;
@@ -410,6 +411,22 @@ size_t gs_layout(GsParams& p, int fmt, int T, int passes, int S) {
   return off;
 }
 
+// Whether two CTAs of the one-token-tile streaming kernel fit on an SM with `smem` bytes
+// each (true without a device: the layout already fits half the shared memory).
+bool gs_two_fit(int fmt, int smem) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return true;
+  int n = 0;
+  const cudaError_t e = fmt == 0
+      ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, gemv_stream_kernel<0, 1>, kGsThreads, smem)
+      : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, gemv_stream_kernel<1, 1>, kGsThreads, smem);
+  if (e != cudaSuccess) {
+    cudaGetLastError();  // the query's own error, not a pending one of another call
+    return false;
+  }
+  return n >= 2;
+}
+
 // One CTA per SM; the fewest passes over K (each at most 4096 weights, the activations of
 // a pass staged whole) whose layout fits with at least 2 ring slots, and up to 4 slots.
 GsPlan gs_plan(int fmt, const uint16_t* x, const uint8_t* wq, const uint16_t* scales, void* y,
@@ -427,17 +444,23 @@ GsPlan gs_plan(int fmt, const uint16_t* x, const uint8_t* wq, const uint16_t* sc
   p.K = K;
   p.out_f32 = out_f32;
   p.U = (K + kGsUnit - 1) / kGsUnit;
-  p.grid = sms;
   const int min_passes = (p.U + kGsMaxUW * kGsWarps - 1) / (kGsMaxUW * kGsWarps);
-  for (int passes = min_passes; passes <= p.U; ++passes) {
-    for (int S = 4; S >= 2; --S) {
-      GsParams q = p;
-      const size_t bytes = gs_layout(q, fmt, T, passes, S);
-      if (bytes > static_cast<size_t>(kGsSmemMax)) continue;
-      best.p = q;
-      best.smem = static_cast<int>(bytes);
-      best.ok = true;
-      return best;
+  // up to 8 tokens, two CTAs per SM when a one-pass layout fits in half the shared memory
+  // (and, with a device current, the occupancy calculator confirms two fit)
+  for (int per_sm = T == 1 ? 2 : 1; per_sm >= 1; --per_sm) {
+    const int limit = per_sm == 2 ? kGsSmemHalf : kGsSmemMax;
+    p.grid = per_sm * sms;
+    for (int passes = min_passes; passes <= (per_sm == 2 ? min_passes : p.U); ++passes) {
+      for (int S = 4; S >= 2; --S) {
+        GsParams q = p;
+        const size_t bytes = gs_layout(q, fmt, T, passes, S);
+        if (bytes > static_cast<size_t>(limit)) continue;
+        if (per_sm == 2 && !gs_two_fit(fmt, static_cast<int>(bytes))) continue;
+        best.p = q;
+        best.smem = static_cast<int>(bytes);
+        best.ok = true;
+        return best;
+      }
     }
   }
   return best;
@@ -467,9 +490,9 @@ int launch_gemv_stream(const GsPlan& pl, cudaStream_t st) {
 // The streaming kernel when it applies (M <= 16, one input, no branch, a layout that fits)
 // and is the faster form; returns 1 when it does not apply.  Measured (chained calls over
 // weights larger than L2): it beats the per-pass kernel for up to 8 tokens with all of K
-// in one pass on the large linears (12288 x 3072: 9.5 against 11.3 us; 21504 x 3072: 13.7
-// against 18.7 us; 4-bit 9728 x 2560: 10.4 against 11.7 us), and loses on 3072 x 3072
-// (4.8 against 3.9 us), with several passes, and at 9..16 tokens.
+// in one pass on the large linears (M = 1: 12288 x 3072 8.5 against 10.1 us, 21504 x 3072
+// 11.7 against 16.8 us, 4-bit 9728 x 2560 9.3 against 10.4 us), and loses on 3072 x 3072
+// (5.6 against 3.1 us) and with several passes; at 9..16 tokens the two are close.
 int try_gemv_stream(int fmt, const uint16_t* x, const uint8_t* wq, const uint16_t* scales, void* y,
                     int M, int N, int K, int out_f32, int sms, cudaStream_t st) {
   const int path = g_path.load();
