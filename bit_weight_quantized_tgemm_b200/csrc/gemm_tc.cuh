@@ -275,7 +275,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  pdl_trigger_and_wait();  // everything above touched only shared and tensor memory
+  // Let the next kernel be scheduled.  Only the warps that touch memory the kernels ahead
+  // may write wait for them: the activation producer (x, or the branch's u, come from the
+  // preparation kernel) and the epilogue (y; the split-tile counters that kernel zeroes).
+  // The packed-weight producer, the dequantizers (codes, scales, the branch's B) and the
+  // MMA issuer (shared and tensor memory only) start at once: the packed weights are not
+  // written by the kernels ahead, so the first stages fill while those finish.
+  pdl_trigger();
+  if (warp == 0 || (warp >= kTcEpiWarp0 && warp < kTcWProdWarp)) pdl_wait();
   const uint32_t tmem_base = *tmem_slot;
   const int ksteps = p.ksteps;
   const int kt1 = DUAL ? p.kt1 : p.kt_main;  // stages of the first input
@@ -571,59 +578,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       }
       // Part of a tile shared with other CTAs.
       const int t_rel = sg.tile - p.sk_t0;  // the tile's place in the split region
-      if constexpr (FMT == 1 && !HYB) {
-        // Every tile split (the 4-bit encoder shapes): a CTA's last segment that holds a
-        // tile's first k part is also where it ends, so nothing waits for its accumulator.
-        // The later sharers write their slots in their first segment, before any wait of
-        // their own, so these waits form a chain towards higher CTAs that ends.  Wait
-        // (bounded) for them, add their slots to this accumulator in k order and store y:
-        // the same sum as the slot path below, without this CTA's slot.
-        if (u == ue && sg.ka == 0) {
-          const int c_lo = static_cast<int>(blockIdx.x);
-          const int c_hi = ((t_rel + 1) * ksteps - 1) / p.upc;
-          const int* cnt_p = p.cnt + t_rel * kTcEpiWarps + piece;
-          bool ready = false;
-          const uint64_t t0 = globaltimer_ns();
-          for (;;) {
-            int st = 0;  // 1: every later slot written, 2: gave up
-            if (lane == 0)
-              st = ld_acquire_gpu(cnt_p) == c_hi - c_lo ? 1 : (globaltimer_ns() - t0 > kWaitLimitNs ? 2 : 0);
-            st = __shfl_sync(0xFFFFFFFFu, st, 0);
-            if (st == 1) {
-              ready = true;
-              break;
-            }
-            if (st == 2) {
-              if (lane == 0) atomicOr(&g_device_error, kDevErrTimeout);
-              break;
-            }
-            __nanosleep(64);
-          }
-          if (ready) {
-            __threadfence();
-#pragma unroll 1
-            for (int cc = 0; cc < kChunks; ++cc) {
-              uint32_t v[32];
-              tmem_ld_32x32b_x32(tbase + cc * 32, v);
-              tmem_wait_ld();
-              if (cc == kChunks - 1) {
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(accempty_bar);
-              }
-#pragma unroll 1
-              for (int c = c_lo + 1; c <= c_hi; ++c) {
-                const float* src = p.part + static_cast<int64_t>(tc_slot(p, c, sg.tile)) * kTcSlotFloats +
-                                   piece * kPieceFloats + cc * 32 * 32 + lane;
-#pragma unroll
-                for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) + __ldcg(src + e * 32));
-              }
-              put(mbase + cc * 32, v);
-            }
-            continue;
-          }
-        }
-      }
       // Write this piece's f32 partial sum to the CTA's slot; the warp that completes the
       // piece's arrival count adds all slots of the tile in k order (deterministic) and
       // stores y.

@@ -249,9 +249,10 @@ int tgemm_tc_plan(int op, int M, int N, int K, int r, int K2, int sms, int* plan
  *   at least tgemm_workspace_size_min() (256-byte aligned; may be NULL when that is 0).
  *   The call overwrites it; calls sharing a workspace must not overlap on the GPU.
  *   Requires M, N >= 1, K % 128 == 0.
- *   Packed weights are read early: for M <= 16 the small-M kernels start loading wq and
- *   its scales before they wait for the kernels ahead of them on the stream (programmatic
- *   dependent launch), so that the fetch overlaps the end of those kernels.  wq and the
+ *   Packed weights are read early: every matmul kernel starts loading wq and its scales
+ *   (and the tensor-core kernel starts dequantizing them) before it waits for the kernels
+ *   ahead of it on the stream (programmatic dependent launch), so that the fetch overlaps
+ *   the end of those kernels.  wq and the
  *   scales must therefore not be written by a matmul call of this library that is still
  *   ahead on the stream.  Weights written by q2_pack, q4_pack or q2_from_gemlite (which
  *   let no later kernel start before they finish), by host copies or by other libraries'
@@ -333,8 +334,8 @@ size_t tgemm_q2_dual_workspace_size_min(int M, int N, int K1, int K2);
  * "We're Teaching...", "What's left").  Dispatch as for tgemm_q2.
  *   x [M][K] bf16 (16-byte aligned), wq [N][K/2] (16-byte aligned), sz [N][K/64][2] f16
  *   (4-byte aligned), y [M][N] (16-byte aligned), workspace as for tgemm_q2 with
- *   TGEMM_OP_Q4.  Requires M, N >= 1, K % 64 == 0.  For M <= 16, wq and sz are read
- *   before the wait for the kernels ahead on the stream, under the same rule as tgemm_q2.
+ *   TGEMM_OP_Q4.  Requires M, N >= 1, K % 64 == 0.  wq and sz are read before the wait for
+ *   the kernels ahead on the stream, under the same rule as tgemm_q2.
  */
 int tgemm_q4(const uint16_t* x, const uint8_t* wq, const uint16_t* sz, void* y, int M, int N,
              int K, int out_dtype, void* workspace, size_t ws_bytes, void* stream);

@@ -163,52 +163,3 @@ def test_plan_checker_catches_a_bad_schedule():
     bad = dict(pl, upc=pl["upc"] - 1)
     with pytest.raises(AssertionError):
         check_plan(bad)
-
-
-def _first_part_waits(pl):
-    """The 4-bit all-split kernel's first-part wait, restated: CTA c waits, at its last
-    segment, when that segment starts tile t's k range and the tile has later sharers.
-    Returns {c: (t, [later sharers])} and checks what makes the waits end: every later
-    sharer reaches the tile in a segment that is not such a wait (so it writes its slot
-    without waiting first), and every waiter waits only on higher-numbered CTAs."""
-    ks = pl["ksteps"]
-    waits = {}
-    segs = {c: _segments(pl, c) for c in range(pl["grid"])}
-    for c, ss in segs.items():
-        if not ss:
-            continue
-        t, ka, kb = ss[-1]
-        if ka == 0 and kb < ks:
-            lo, hi = (t - pl["sk_t0"]) * ks // pl["upc"], ((t - pl["sk_t0"] + 1) * ks - 1) // pl["upc"]
-            assert lo == c and hi > c, (c, t, lo, hi)
-            waits[c] = (t, list(range(c + 1, hi + 1)))
-    for c, (t, later) in waits.items():
-        for d in later:
-            assert d > c
-            mine = [s for s in segs[d] if s[0] == t]
-            assert len(mine) == 1 and mine[0][1] > 0, (c, d, mine)   # d's part starts mid-tile
-            assert segs[d].index(mine[0]) == 0, (c, d, segs[d])       # and is d's first segment
-    return waits
-
-
-@pytest.mark.parametrize("N,K", [(9728, 2560), (2560, 9728)])
-def test_first_part_waits_end_on_the_encoder_shapes(N, K):
-    pl = tg.tc_plan(tg.OP_Q4, 512, N, K, sms=148)
-    assert pl["split"] and pl["dpc"] == 0, pl
-    waits = _first_part_waits(pl)
-    assert waits, "the shape is expected to exercise the wait"
-
-
-def test_first_part_waits_end_random():
-    rng = random.Random(7)
-    n = 0
-    for _ in range(600):
-        M = rng.randint(1, 2000)
-        N = rng.randint(64, 20000)
-        K = 64 * rng.randint(1, 200)
-        sms = rng.choice([148, 148, 132, 100, 7])
-        pl = tg.tc_plan(tg.OP_Q4, M, N, K, sms=sms)
-        if pl["split"] and pl["dpc"] == 0:
-            _first_part_waits(pl)
-            n += 1
-    assert n > 50
