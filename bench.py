@@ -61,6 +61,9 @@ def parse_args():
                     help="skip the end-to-end leg, the small-M stream and the CPU baseline")
     ap.add_argument("--parts", default="",
                     help="comma-separated subset of the extra parts to run (default: all)")
+    ap.add_argument("--kernels", action="store_true",
+                    help="run every kernel of the library once on its workload inside an NVTX "
+                         "range named 'kernels' (for ncu --nvtx --nvtx-include kernels/), then exit")
     return ap.parse_args()
 
 
@@ -866,8 +869,94 @@ def gemv_branch(tg, torch, stream):
     return out
 
 
+def kernel_tour(tg, torch):
+    """Every kernel of the library once, each call inside an NVTX range 'kernels' after two
+    warm-up calls outside it; inputs are drawn outside the ranges and freed after each
+    workload (a small device footprint for profilers that replay kernels)."""
+    import torch.cuda.nvtx as nvtx
+    g = torch.Generator(device="cuda").manual_seed(99)
+    dev = "cuda"
+
+    def once(label, fn):
+        for _ in range(2):
+            fn()
+        torch.cuda.synchronize()
+        nvtx.range_push("kernels")
+        fn()
+        nvtx.range_pop()
+        torch.cuda.synchronize()
+        print(f"kernels: {label}", flush=True)
+
+    def codes(N, K, hi):
+        return torch.randint(0, hi, (N, K), dtype=torch.uint8, device=dev, generator=g)
+
+    # load-time packing and the dequantization hooks
+    c2, s2 = codes(9216, 3072, 3), (torch.rand(9216, 24, device=dev, generator=g) * 0.02).half().float()
+    once("q2_pack 9216x3072", lambda: tg.q2_pack(c2, s2))
+    c4 = codes(9728, 2560, 16)
+    s4 = (torch.rand(9728, 40, device=dev, generator=g) * 0.01).half().float()
+    z4 = (7 + torch.rand(9728, 40, device=dev, generator=g)).half().float()
+    once("q4_pack 9728x2560", lambda: tg.q4_pack(c4, s4, z4))
+    wgl = torch.randint(0, 256, (768, 3072), dtype=torch.uint8, device=dev, generator=g)
+    sgl = (torch.rand(3072, 48, device=dev, generator=g) * 0.02).half().float()
+    once("q2_from_gemlite 3072x3072 g=64", lambda: tg.q2_from_gemlite(wgl, sgl, -sgl, 64))
+    wq2, d2, _ = tg.q2_pack(c2, s2)
+    wq4, sz4, _ = tg.q4_pack(c4, s4, z4)
+    once("q2_dequant 9216x3072", lambda: tg.q2_dequant(wq2, d2))
+    once("q4_dequant 9728x2560", lambda: tg.q4_dequant(wq4, sz4))
+    del c2, s2, c4, s4, z4, wgl, sgl
+
+    def x(M, K):
+        return torch.randn(M, K, device=dev, generator=g).bfloat16()
+
+    prev = tg.set_path(tg.PATH_AUTO)
+    try:
+        # tensor-core path: activation prep + the tcgen05 kernel
+        x1 = x(1536, 3072)
+        once("tgemm_q2 1536x9216x3072", lambda: tg.gemm_q2(x1, wq2, d2))
+        a = (torch.randn(32, 3072, device=dev, generator=g) * 1e-3).bfloat16()
+        b = (torch.randn(9216, 32, device=dev, generator=g) * 1e-3).bfloat16()
+        once("tgemm_q2_lora r=32 1536x9216x3072", lambda: tg.gemm_q2_lora(x1, wq2, d2, a, b))
+        xe = x(512, 2560)
+        once("tgemm_q4 512x9728x2560", lambda: tg.gemm_q4(xe, wq4, sz4))
+        cw = codes(3072, 3072, 3)
+        cs = (torch.rand(3072, 24, device=dev, generator=g) * 0.02).half().float()
+        wa, da, _ = tg.q2_pack(cw, cs)
+        cw2 = codes(3072, 12288, 3)
+        cs2 = (torch.rand(3072, 96, device=dev, generator=g) * 0.02).half().float()
+        wb, db, _ = tg.q2_pack(cw2, cs2)
+        del cw, cs, cw2, cs2
+        xa, xb = x(1536, 3072), x(1536, 12288)
+        once("tgemm_q2_dual 1536x3072x(3072+12288)", lambda: tg.gemm_q2_dual(xa, wa, da, xb, wb, db))
+        # small-M path: the per-pass kernel (also with the branch and two inputs), the
+        # streaming kernel
+        tg.set_path(tg.PATH_SMALL_M_PASS)
+        x16 = x(16, 3072)
+        once("gemv pass Q2 M=16 3072x3072", lambda: tg.gemm_q2(x16, wa, da))
+        x4e = x(4, 2560)
+        once("gemv pass 4-bit M=4 9728x2560", lambda: tg.gemm_q4(x4e, wq4, sz4))
+        x4 = x(4, 3072)
+        once("gemv pass Q2 branch r=32 M=4 9216x3072", lambda: tg.gemm_q2_lora(x4, wq2, d2, a, b))
+        x4b = x(4, 12288)
+        once("gemv pass Q2 two inputs M=4 3072x(3072+12288)", lambda: tg.gemm_q2_dual(x4, wa, da, x4b, wb, db))
+        tg.set_path(tg.PATH_SMALL_M_STREAM)
+        x1q = x(1, 3072)
+        once("gemv stream Q2 M=1 9216x3072", lambda: tg.gemm_q2(x1q, wq2, d2))
+        x1e = x(1, 2560)
+        once("gemv stream 4-bit M=1 9728x2560", lambda: tg.gemm_q4(x1e, wq4, sz4))
+    finally:
+        tg.set_path(prev)
+    assert tg.device_error() == 0
+
+
 def main():
     args = parse_args()
+    if args.kernels:
+        import torch
+
+        import bit_weight_quantized_tgemm_b200 as tg
+        kernel_tour(tg, torch)
+        return 0
     world, rank, local = (1, 0, 0)
     if args.impl == "reference":
         world = int(os.environ.get("WORLD_SIZE", "1"))
