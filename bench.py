@@ -841,8 +841,8 @@ def gemv_stream(tg, torch, stream):
 
 def gemv_branch(tg, torch, stream):
     """Small-M calls with the rank-r branch (M = 1, 4, 16 on 9216 x 3072, r = 4, 32, 64):
-    the branch's two preparation kernels plus the per-pass kernel, back to back from a
-    CUDA graph over weight copies totalling >= 4x L2."""
+    the kernel computing u = x A^T plus the per-pass kernel, back to back from a CUDA graph
+    over weight copies totalling >= 4x L2; r0: the same calls without the branch."""
     N, K = 9216, 3072
     wbytes = N * K // 4 + N * (K // 128) * 2
     l2 = torch.cuda.get_device_properties(0).L2_cache_size
@@ -851,6 +851,13 @@ def gemv_branch(tg, torch, stream):
     copies = [_device_weights(tg, torch, 0, N, K, g) for _ in range(ncopies)]
     L = tg.lib()
     out = {}
+    for M in (1, 4, 16):  # the same calls without the branch
+        x = torch.randn(M, K, device="cuda").bfloat16()
+        y = torch.empty(M, N, device="cuda", dtype=torch.bfloat16)
+        calls = [(x.data_ptr(), wq.data_ptr(), d.data_ptr(), y.data_ptr(), M, N, K, tg.OUT_BF16, None, 0)
+                 for (wq, d) in copies]
+        t = _graph_per_call(tg, torch, calls, L.tgemm_q2)
+        out[f"r0_m{M}"] = {"us_per_call": t * 1e6, "weight_gbs": wbytes / t / 1e9}
     for r in (4, 32, 64):
         a = (torch.randn(r, K, device="cuda") * 1e-3).bfloat16()
         b = (torch.randn(N, r, device="cuda") * 1e-3).bfloat16()

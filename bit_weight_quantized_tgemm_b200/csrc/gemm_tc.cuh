@@ -862,93 +862,17 @@ __global__ void __launch_bounds__(256) prep_lora_kernel(const uint16_t* __restri
   }
 }
 
-// u = x A^T for the low-rank branch, in two deterministic phases (no atomics).
-// Phase 1 (lora_down_partial_kernel): CTA (token block of 16, K slice of kLoraKc, column
-// chunk of 64) accumulates its slice on mma.sync (bf16 in, f32 accumulate); its 8 warps
-// split the slice and reduce through shared memory; the partial lands in
-// part[slice][m][col] (f32, `rpad` columns per row).
-// Phase 2 (lora_finalize_kernel): sums the slices in a fixed order and writes u in f32
-// [M][r] (small-M path) and/or the concatenation ucat [M][wcat] =
-// [bf16(u) pad R | bf16(u - bf16(u)) pad R | 0] (tensor-core path).
-__global__ void __launch_bounds__(256) lora_down_partial_kernel(
-    const uint16_t* __restrict__ x, const uint16_t* __restrict__ a, int M, int K, int r,
-    int rpad, float* __restrict__ part) {
-  pdl_trigger_and_wait();
-  __shared__ float red[8][16][65];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int g = lane >> 2, c = lane & 3;
-  const int m0 = blockIdx.x * 16;
-  const int k_lo = blockIdx.y * kLoraKc;
-  const int k_hi = min(K, k_lo + kLoraKc);
-  const int col0 = blockIdx.z * 64;
-  float acc[8][4];
-#pragma unroll
-  for (int t = 0; t < 8; ++t)
-#pragma unroll
-    for (int e = 0; e < 4; ++e) acc[t][e] = 0.f;
-  const uint32_t* x32 = reinterpret_cast<const uint32_t*>(x);
-  const uint32_t* a32 = reinterpret_cast<const uint32_t*>(a);
-  const int kw = K / 2;  // 32-bit words per row
-  const bool r0 = m0 + g < M, r1 = m0 + g + 8 < M;
-#pragma unroll 2
-  for (int kb = k_lo / 16 + warp; kb < k_hi / 16; kb += 8) {
-    const int k2 = kb * 8 + c;  // word index of (k = 16kb + 2c, +1)
-    const uint32_t a0 = r0 ? __ldg(x32 + static_cast<int64_t>(m0 + g) * kw + k2) : 0u;
-    const uint32_t a1 = r1 ? __ldg(x32 + static_cast<int64_t>(m0 + g + 8) * kw + k2) : 0u;
-    const uint32_t a2 = r0 ? __ldg(x32 + static_cast<int64_t>(m0 + g) * kw + k2 + 4) : 0u;
-    const uint32_t a3 = r1 ? __ldg(x32 + static_cast<int64_t>(m0 + g + 8) * kw + k2 + 4) : 0u;
-    uint32_t b[8][2];
-#pragma unroll
-    for (int t = 0; t < 8; ++t) {
-      const int col = col0 + 8 * t + g;
-      const bool cv = col < r;
-      b[t][0] = cv ? __ldg(a32 + static_cast<int64_t>(col) * kw + k2) : 0u;
-      b[t][1] = cv ? __ldg(a32 + static_cast<int64_t>(col) * kw + k2 + 4) : 0u;
-    }
-#pragma unroll
-    for (int t = 0; t < 8; ++t)
-      asm volatile(
-          "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
-          "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
-          : "+f"(acc[t][0]), "+f"(acc[t][1]), "+f"(acc[t][2]), "+f"(acc[t][3])
-          : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b[t][0]), "r"(b[t][1]));
-  }
-#pragma unroll
-  for (int t = 0; t < 8; ++t) {
-    red[warp][g][8 * t + 2 * c] = acc[t][0];
-    red[warp][g][8 * t + 2 * c + 1] = acc[t][1];
-    red[warp][g + 8][8 * t + 2 * c] = acc[t][2];
-    red[warp][g + 8][8 * t + 2 * c + 1] = acc[t][3];
-  }
-  __syncthreads();
-  for (int o = threadIdx.x; o < 16 * 64; o += blockDim.x) {
-    const int mm = o >> 6, cc = o & 63;
-    const int m = m0 + mm, col = col0 + cc;
-    if (m >= M || col >= rpad) continue;
-    float v = 0.f;
-#pragma unroll
-    for (int w = 0; w < 8; ++w) v += red[w][mm][cc];
-    part[(static_cast<int64_t>(blockIdx.y) * M + m) * rpad + col] = v;
-  }
-}
-
+// Tensor-core path, second step of u = x A^T: sums prep_lora_kernel's K-slice partials in a
+// fixed order (no atomics) and writes the concatenation ucat [M][wcat] =
+// [bf16(u) pad R | bf16(u - bf16(u)) pad R | 0], the branch stages' activations.
 __global__ void __launch_bounds__(256) lora_finalize_kernel(const float* __restrict__ part,
                                                             int slices, int M, int r, int rpad,
                                                             int R, int wcat,
-                                                            float* __restrict__ u32,
                                                             uint16_t* __restrict__ ucat) {
   pdl_trigger_and_wait();
   const int64_t total = static_cast<int64_t>(M) * wcat;
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-       i < (ucat ? total : static_cast<int64_t>(M) * r); i += stride) {
-    if (ucat == nullptr) {
-      const int64_t m = i / r, col = i % r;
-      float v = 0.f;
-      for (int sl = 0; sl < slices; ++sl) v += part[(sl * static_cast<int64_t>(M) + m) * rpad + col];
-      u32[i] = v;
-      continue;
-    }
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total; i += stride) {
     const int64_t m = i / wcat;
     const int j = static_cast<int>(i % wcat);
     uint16_t out = 0;

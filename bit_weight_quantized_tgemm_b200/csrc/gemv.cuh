@@ -52,22 +52,41 @@ struct GvFmt {
   static constexpr int kUnitBytes = FMT == 0 ? 32 : 64;      // packed bytes of a row-unit
   static constexpr int kWords = FMT == 0 ? 2 : 4;             // 32-bit code words per lane
 };
-// Dynamic shared memory per CTA (the staged activations): two CTAs fit on one SM with 16
-// tokens x 3072 in one pass.
-constexpr int kGvXBudget = 104960;
+// Dynamic shared memory per CTA: the staged activations (whose space the warps' partial
+// sums reuse once the last pass is done) and, with the low-rank branch, u and B.  Two CTAs
+// fit on one SM at this size: 2 x (111360 + at most 4224 static + 1024 reserved) is within
+// the SM's 233472 bytes.  16 tokens x 3072 (and, with the branch, up to r = 112) take one pass.
+constexpr int kGvXBudget = 111360;
 
 __host__ __device__ constexpr int gemv_row_stride_bytes(int kp) { return 2 * kp + 16; }
+__host__ __device__ constexpr int gemv_round16(int b) { return (b + 15) / 16 * 16; }
+// the warps' partial sums: f32 [warp][row][token], kTok + 1 tokens per row
+__host__ __device__ constexpr int gemv_red_bytes(int T) { return kGvWarps * kGvRows * (8 * T + 1) * 4; }
+// the activation rows of a pass, or the partial sums, whichever is larger
+__host__ __device__ constexpr int gemv_xreg_bytes(int mrows, int kp, int T) {
+  return gemv_round16(mrows * gemv_row_stride_bytes(kp) > gemv_red_bytes(T)
+                          ? mrows * gemv_row_stride_bytes(kp) : gemv_red_bytes(T));
+}
+// Branch operands in shared memory, bf16, the rank padded with zeros to a multiple of 16 and
+// rows gemv_lb_pitch(r) elements apart (= 8 mod 16, so a fragment's 32 words hit 32 banks):
+// the CTA's 16 rows of B, then u of the pass's 8 T tokens as u_hi = bf16(u) and
+// u_lo = bf16(u - u_hi).
+__host__ __device__ constexpr int gemv_lb_pitch(int r) { return (r + 15) / 16 * 16 + 8; }
+__host__ __device__ constexpr int gemv_lora_bytes(int T, int r) {
+  return r > 0 ? gemv_round16((kGvRows + 16 * T) * gemv_lb_pitch(r) * 2) : 0;
+}
 // K per pass: the largest multiple of 128 (at most the format's kKPMax) whose staged
-// activation rows (`mrows` tokens) fit kGvXBudget; never more than K needs.
-__host__ __device__ inline int gemv_pass_k(int fmt, int mrows, int K) {
+// activation rows (`mrows` tokens, token tiles of 8 T) fit kGvXBudget next to `extra`
+// bytes; never more than K needs.
+__host__ __device__ inline int gemv_pass_k(int fmt, int mrows, int K, int T = 2, int extra = 0) {
   const int kmax = fmt == 0 ? GvFmt<0>::kKPMax : GvFmt<1>::kKPMax;
   int kp = (K + kGvUnit - 1) / kGvUnit * kGvUnit;
   if (kp > kmax) kp = kmax;
-  while (kp > kGvUnit && mrows * gemv_row_stride_bytes(kp) > kGvXBudget) kp -= kGvUnit;
+  while (kp > kGvUnit && gemv_xreg_bytes(mrows, kp, T) + extra > kGvXBudget) kp -= kGvUnit;
   return kp;
 }
-__host__ __device__ constexpr int gemv_smem_bytes(int mrows, int kp) {
-  return mrows * gemv_row_stride_bytes(kp);
+__host__ __device__ constexpr int gemv_smem_bytes(int mrows, int kp, int T = 2, int r = 0) {
+  return gemv_xreg_bytes(mrows, kp, T) + gemv_lora_bytes(T, r);
 }
 
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
@@ -112,7 +131,6 @@ __global__ void __launch_bounds__(256, 2) gemv_kernel(
   using F = GvFmt<FMT>;
   constexpr int kTok = 8 * T;  // tokens per pass over the weights
   extern __shared__ __align__(128) uint8_t gv_smem[];
-  __shared__ float red[kGvWarps][kGvRows][kTok + 1];  // the warps' partial sums
   __shared__ __align__(8) uint64_t xbar;              // the activation copies of a pass
   __shared__ uint32_t abort_word;
   // the pass's scales of the CTA's rows: Q2 d per unit, 4-bit (s, z) per group
@@ -128,6 +146,13 @@ __global__ void __launch_bounds__(256, 2) gemv_kernel(
   const uint32_t xs = smem_u32(gv_smem);
   const uint32_t bar = smem_u32(&xbar);
   const int rs = gemv_row_stride_bytes(kp);
+  // the warps' partial sums [warp][row][token] reuse the activations' space after the last pass
+  float* red = reinterpret_cast<float*>(gv_smem);
+  // branch operands: the CTA's rows of B [row][lbp], u_hi and u_lo [token][lbp]
+  const int lbp = gemv_lb_pitch(r), r16 = lbp - 8;
+  uint16_t* bs = reinterpret_cast<uint16_t*>(gv_smem + gemv_xreg_bytes(min(M, kTok), kp, T));
+  uint16_t* uhs = bs + kGvRows * lbp;
+  uint16_t* uls = uhs + kTok * lbp;
   volatile uint32_t* abort_flag = &abort_word;
   if (tid == 0) {
     mbar_init(bar, 1);
@@ -202,6 +227,28 @@ __global__ void __launch_bounds__(256, 2) gemv_kernel(
     load_codes(wq, FMT == 0 ? K / 4 : K / 2, K, 0, u_end0);
     stage_scales(scales, FMT == 0 ? K / 128 : K / 64, 0, u_end0);
   }
+  if (LORA) {
+    // The CTA's rows of B (a weight, like the codes) -> shared memory, zero past r and N,
+    // in the order that keeps consecutive threads on consecutive addresses of its layout.
+    const bool by_row = lb_si == 1;
+    for (int i0 = tid; i0 < kGvRows * r16; i0 += 4 * 256) {
+      uint16_t v[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int i = i0 + e * 256;
+        const int nn = by_row ? i / r16 : i % kGvRows, k = by_row ? i % r16 : i / kGvRows;
+        v[e] = 0;
+        if (i < kGvRows * r16 && k < r && n0 + nn < N)
+          v[e] = __ldg(lb + static_cast<int64_t>(n0 + nn) * lb_sn + static_cast<int64_t>(k) * lb_si);
+      }
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int i = i0 + e * 256;
+        const int nn = by_row ? i / r16 : i % kGvRows, k = by_row ? i % r16 : i / kGvRows;
+        if (i < kGvRows * r16) bs[nn * lbp + k] = v[e];
+      }
+    }
+  }
   __syncthreads();  // the barrier's initialisation and the first scales are visible
   pdl_wait();
 
@@ -214,6 +261,29 @@ __global__ void __launch_bounds__(256, 2) gemv_kernel(
     for (int t = 0; t < T; ++t)
 #pragma unroll
       for (int e = 0; e < 4; ++e) acc[t][e] = 0.f;
+    if (LORA && warp > 0) {
+      // Warps 1-7 copy u of this pass's tokens to shared memory as (u_hi, u_lo), zero past
+      // r and the pass's tokens, while warp 0 starts the activation copies; they are read
+      // after the last pass.
+      const int nt = blockDim.x - 32;
+      for (int i0 = tid - 32; i0 < kTok * r16; i0 += 8 * nt) {
+        float v[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const int i = i0 + e * nt, mm = i / r16, k = i % r16;
+          v[e] = i < kTok * r16 && mm < mt && k < r ? __ldg(u + static_cast<int64_t>(m0 + mm) * r + k) : 0.f;
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const int i = i0 + e * nt, mm = i / r16, k = i % r16;
+          if (i < kTok * r16) {
+            const __nv_bfloat16 h = __float2bfloat16_rn(v[e]);
+            uhs[mm * lbp + k] = __bfloat16_as_ushort(h);
+            uls[mm * lbp + k] = __bfloat16_as_ushort(__float2bfloat16_rn(v[e] - __bfloat162float(h)));
+          }
+        }
+      }
+    }
 
     // one input, or two (a projection split along its input axis: their products add
     // into the same partial sums)
@@ -352,13 +422,35 @@ __global__ void __launch_bounds__(256, 2) gemv_kernel(
       }
     }
 
+    // ---- the branch: acc += B (u_hi + u_lo)^T, its rank's 16-wide steps spread over the
+    // warps (bf16 products are exact in the f32 accumulators)
+    if (LORA) {
+      for (int s = warp; s < r16 / 16; s += kGvWarps) {
+        // rank slots 2c, 2c+1 (word 0) and 2c+8, 2c+9 (word 4) of step s
+        const uint32_t* b0 = reinterpret_cast<const uint32_t*>(bs + g * lbp + 16 * s + 2 * c);
+        const uint32_t* b1 = reinterpret_cast<const uint32_t*>(bs + (g + 8) * lbp + 16 * s + 2 * c);
+        const uint32_t af[4] = {b0[0], b1[0], b0[4], b1[4]};
+#pragma unroll
+        for (int t = 0; t < T; ++t) {
+          const uint32_t* uh = reinterpret_cast<const uint32_t*>(uhs + (g + 8 * t) * lbp + 16 * s + 2 * c);
+          const uint32_t* ul = reinterpret_cast<const uint32_t*>(uls + (g + 8 * t) * lbp + 16 * s + 2 * c);
+          mma_bf16_16816(acc[t], af, uh[0], uh[4]);
+          mma_bf16_16816(acc[t], af, ul[0], ul[4]);
+        }
+      }
+    }
+
     // ---- reduce the warps' partial sums and write y ---------------------------------
+    // (the last pass ended with a barrier: nobody reads the activations any more)
+    auto red_at = [&](int w, int nn, int mm) -> float& {
+      return red[(w * kGvRows + nn) * (kTok + 1) + mm];
+    };
 #pragma unroll
     for (int t = 0; t < T; ++t) {
-      red[warp][g][2 * c + 8 * t] = acc[t][0];
-      red[warp][g][2 * c + 1 + 8 * t] = acc[t][1];
-      red[warp][g + 8][2 * c + 8 * t] = acc[t][2];
-      red[warp][g + 8][2 * c + 1 + 8 * t] = acc[t][3];
+      red_at(warp, g, 2 * c + 8 * t) = acc[t][0];
+      red_at(warp, g, 2 * c + 1 + 8 * t) = acc[t][1];
+      red_at(warp, g + 8, 2 * c + 8 * t) = acc[t][2];
+      red_at(warp, g + 8, 2 * c + 1 + 8 * t) = acc[t][3];
     }
     __syncthreads();
     for (int o = tid; o < kTok * kGvRows; o += blockDim.x) {
@@ -367,20 +459,87 @@ __global__ void __launch_bounds__(256, 2) gemv_kernel(
       if (mm >= mt || n >= N) continue;
       float v = 0.f;
 #pragma unroll
-      for (int w = 0; w < kGvWarps; ++w) v += red[w][nn][mm];
-      if (LORA) {
-        float br = 0.f;
-        for (int i = 0; i < r; ++i)
-          br = fmaf(bf16_bits_to_f32(lb[static_cast<int64_t>(n) * lb_sn + static_cast<int64_t>(i) * lb_si]),
-                    u[static_cast<int64_t>(m) * r + i], br);
-        v += br;
-      }
+      for (int w = 0; w < kGvWarps; ++w) v += red_at(w, nn, mm);
       if (out_f32)
         reinterpret_cast<float*>(y)[static_cast<int64_t>(m) * N + n] = v;
       else
         reinterpret_cast<__nv_bfloat16*>(y)[static_cast<int64_t>(m) * N + n] = __float2bfloat16_rn(v);
     }
+    // the next token pass's bulk copies (the async proxy) overwrite the partial sums
+    fence_proxy_async_smem();
     __syncthreads();
+  }
+}
+
+// u = x A^T for the low-rank branch on the small-M path, in one launch.  CTA (16 tokens, 8
+// columns of u = 8 rows of A) runs over the whole of K: its 16 warps take interleaved k16
+// steps on mma.sync (A operand: the token rows of x; B operand: the rows of A; bf16 in, f32
+// accumulate), and the warps' sums are added in warp order through shared memory -- a fixed
+// order, no atomics and no second kernel.  The CTA's rows of A (a weight) are prefetched
+// into L2 before the dependency wait.  Lane (g, c) feeds the k slots {2c, 2c+1, 2c+8, 2c+9}
+// of a step with its elements 4c..4c+3 (one 8-byte load per row); both operands use that
+// map, so the contraction is unchanged.  A8: A is 8-byte aligned (else two 4-byte loads).
+constexpr int kLdWarps = 16;
+constexpr int kLdBatch = 12;  // k16 steps a warp loads before their mma (one trip when K <= 3072)
+template <bool A8>
+__global__ void __launch_bounds__(kLdWarps * 32) lora_down_small_kernel(
+    const uint16_t* __restrict__ x, const uint16_t* __restrict__ a, int M, int K, int r,
+    float* __restrict__ u) {
+  __shared__ float red[kLdWarps][16][8];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, c = lane & 3;
+  const int j0 = blockIdx.x * 8, m0 = blockIdx.y * 16;
+  const int64_t row_bytes = static_cast<int64_t>(K) * 2;
+  pdl_trigger();
+  {
+    const int lines = static_cast<int>((row_bytes + 127) / 128);
+    for (int i = threadIdx.x; i < 8 * lines; i += blockDim.x) {
+      const int j = j0 + i / lines;
+      if (j < r) prefetch_l2(reinterpret_cast<const uint8_t*>(a) + j * row_bytes + (i % lines) * 128);
+    }
+  }
+  pdl_wait();
+  const bool ok0 = m0 + g < M, ok1 = m0 + g + 8 < M, okb = j0 + g < r;
+  // rows clamped into range (a row that does not exist contributes zeros); element 4c
+  const uint2* x0 = reinterpret_cast<const uint2*>(x + static_cast<int64_t>(min(m0 + g, M - 1)) * K) + c;
+  const uint2* x1 = reinterpret_cast<const uint2*>(x + static_cast<int64_t>(min(m0 + g + 8, M - 1)) * K) + c;
+  const uint16_t* arow = a + static_cast<int64_t>(min(j0 + g, r - 1)) * K + 4 * c;
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  const int steps = K / 16;
+  for (int kb0 = warp; kb0 < steps; kb0 += kLdWarps * kLdBatch) {
+    uint2 f0[kLdBatch], f1[kLdBatch], fb[kLdBatch];
+#pragma unroll
+    for (int i = 0; i < kLdBatch; ++i) {
+      const int kb = kb0 + i * kLdWarps;
+      const bool in = kb < steps;
+      const uint2 z = make_uint2(0u, 0u);
+      f0[i] = in && ok0 ? __ldg(x0 + 4 * kb) : z;
+      f1[i] = in && ok1 ? __ldg(x1 + 4 * kb) : z;
+      if (A8) {
+        fb[i] = in && okb ? __ldg(reinterpret_cast<const uint2*>(arow + 16 * kb)) : z;
+      } else {
+        const uint32_t* p = reinterpret_cast<const uint32_t*>(arow + 16 * kb);
+        fb[i] = in && okb ? make_uint2(__ldg(p), __ldg(p + 1)) : z;
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < kLdBatch; ++i) {
+      const uint32_t af[4] = {f0[i].x, f1[i].x, f0[i].y, f1[i].y};
+      mma_bf16_16816(acc, af, fb[i].x, fb[i].y);
+    }
+  }
+  // acc: u[m0 + g (+8)][j0 + 2c (+1)]
+  red[warp][g][2 * c] = acc[0];
+  red[warp][g][2 * c + 1] = acc[1];
+  red[warp][g + 8][2 * c] = acc[2];
+  red[warp][g + 8][2 * c + 1] = acc[3];
+  __syncthreads();
+  if (threadIdx.x < 128) {
+    const int mm = threadIdx.x >> 3, jj = threadIdx.x & 7;
+    float v = 0.f;
+#pragma unroll
+    for (int w = 0; w < kLdWarps; ++w) v += red[w][mm][jj];
+    if (m0 + mm < M && j0 + jj < r) u[static_cast<int64_t>(m0 + mm) * r + j0 + jj] = v;
   }
 }
 

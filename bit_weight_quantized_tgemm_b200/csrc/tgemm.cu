@@ -304,7 +304,7 @@ Workspace workspace_layout(int op, int M, int N, int K, int r, int path, int sms
     w.u32_bytes = static_cast<size_t>(M) * r * 4;
     off = round_up(off + w.u32_bytes, 256);
   }
-  if (lora) {
+  if (lora && path == TGEMM_PATH_TENSOR) {
     const LoraDims ld = lora_dims(r, K);
     w.part = off;
     w.part_bytes = static_cast<size_t>(ld.slices) * M * ld.rpad * 4;
@@ -326,20 +326,14 @@ Workspace workspace_layout(int op, int M, int N, int K, int r, int path, int sms
   return w;
 }
 
-// u = x A^T into u32 (f32 [M][r]) and/or ucat, through the partial-sum workspace.
-int launch_lora_down(const uint16_t* x, const uint16_t* la, int M, int K, int r,
-                     const LoraDims& ld, float* part, float* u32, uint16_t* ucat,
-                     cudaStream_t st, int sms) {
-  const dim3 grid((M + 15) / 16, ld.slices, ld.rpad / 64);
-  if (int e = launch(TGEMM_KIND_PREP, st, [&] {
-        return pdl_launch(lora_down_partial_kernel, grid, 256, 0, st, x, la, M, K, r, ld.rpad, part);
-      }))
-    return e;
-  const int64_t items = ucat ? static_cast<int64_t>(M) * ld.wcat : static_cast<int64_t>(M) * r;
-  const int fgrid = grid_for(items, 256, sms);
+// Small-M path: u = x A^T into u32 (f32 [M][r]), one launch.
+int launch_lora_down_small(const uint16_t* x, const uint16_t* la, int M, int K, int r, float* u32,
+                           cudaStream_t st) {
+  const dim3 grid((r + 7) / 8, (M + 15) / 16);
   return launch(TGEMM_KIND_PREP, st, [&] {
-    return pdl_launch(lora_finalize_kernel, fgrid, 256, 0, st, part, ld.slices, M, r, ld.rpad, ld.R, ld.wcat,
-                                                u32, ucat);
+    if (aligned(la, 8))
+      return pdl_launch(lora_down_small_kernel<true>, grid, kLdWarps * 32, 0, st, x, la, M, K, r, u32);
+    return pdl_launch(lora_down_small_kernel<false>, grid, kLdWarps * 32, 0, st, x, la, M, K, r, u32);
   });
 }
 
@@ -572,7 +566,7 @@ int run_gemm(int fmt, const uint16_t* x, const uint8_t* wq, const uint16_t* scal
     float* u32 = nullptr;
     if (lora) {
       u32 = reinterpret_cast<float*>(ws + wl.u32);
-      if (int e = launch_lora_down(x, la, M, K, r, ld, part, u32, nullptr, st, di.sms)) return e;
+      if (int e = launch_lora_down_small(x, la, M, K, r, u32, st)) return e;
     }
     if (!lora && !dual) {
       const int e = try_gemv_stream(fmt, x, wq, scales, y, M, N, K, out_f32, di.sms, st);
@@ -580,9 +574,10 @@ int run_gemm(int fmt, const uint16_t* x, const uint8_t* wq, const uint16_t* scal
     }
     const int grid = (N + kGvRows - 1) / kGvRows;
     const int mrows = M < 16 ? M : 16;
-    const int kp = gemv_pass_k(fmt, mrows, K > K2 ? K : K2);
-    const size_t smem = gemv_smem_bytes(mrows, kp);
     const bool t1 = M <= 8;  // one token tile of 8, else two
+    const int T = t1 ? 1 : 2, rl = lora ? r : 0;
+    const int kp = gemv_pass_k(fmt, mrows, K > K2 ? K : K2, T, gemv_lora_bytes(T, rl));
+    const size_t smem = gemv_smem_bytes(mrows, kp, T, rl);
     const uint16_t* x2 = in2.x;
     const uint8_t* wq2 = in2.wq;
     const uint16_t* d2 = in2.d;
@@ -622,8 +617,8 @@ int run_gemm(int fmt, const uint16_t* x, const uint8_t* wq, const uint16_t* scal
       return e;
     const int fgrid = grid_for(static_cast<int64_t>(M) * ld.wcat, 256, di.sms);
     if (int e = launch(TGEMM_KIND_PREP, st, [&] {
-          return pdl_launch(lora_finalize_kernel, fgrid, 256, 0, st, part, ld.slices, M, r, ld.rpad, ld.R, ld.wcat,
-                                                      nullptr, ucat);
+          return pdl_launch(lora_finalize_kernel, fgrid, 256, 0, st, part, ld.slices, M, r, ld.rpad, ld.R,
+                            ld.wcat, ucat);
         }))
       return e;
   } else {

@@ -265,9 +265,10 @@ int tgemm_q2(const uint16_t* x, const uint8_t* wq, const uint16_t* d, void* y, i
  * tgemm_q2_lora -- y = x . W^T + (x . A^T) . B^T ("mindview-t2i-turbo", "One step").
  *   As tgemm_q2, plus a [r][K] bf16 (4-byte aligned) and b [N][r] bf16 (2-byte aligned),
  *   1 <= r <= 256, and workspace of tgemm_workspace_size(TGEMM_OP_Q2_LORA, M, N, K, r).
- *   The branch has no extra scale factor.  u = x . A^T is accumulated in f32; the
- *   tensor-core path feeds it to the MMA as a bf16 pair (hi + lo) so that its rounding
- *   error stays near 2^-16 relative.
+ *   The branch has no extra scale factor.  u = x . A^T is accumulated in f32; both
+ *   paths feed it to the MMA as a bf16 pair (hi + lo) so that its rounding error stays
+ *   near 2^-16 relative.  a and b are weights and are read early like wq (see tgemm_q2):
+ *   neither may be written by a matmul call of this library still ahead on the stream.
  */
 int tgemm_q2_lora(const uint16_t* x, const uint8_t* wq, const uint16_t* d, const uint16_t* a,
                   const uint16_t* b, int r, void* y, int M, int N, int K, int out_dtype,

@@ -60,7 +60,7 @@ def test_workspace_sizes():
         # f16 x + [u_hi | u_lo] + f32 partial sums of u over 6 K-slices of 512
         assert lora == 1536 * 3072 * 2 + 1536 * 128 * 2 + 6 * 1536 * 64 * 4  # wcat = 128
         # small-M path: f32 u + the partial sums
-        assert tg.workspace_size(tg.OP_Q2_LORA, 4, 9216, 3072, 64) == 4 * 64 * 4 + 6 * 4 * 64 * 4
+        assert tg.workspace_size(tg.OP_Q2_LORA, 4, 9216, 3072, 64) == 4 * 64 * 4  # u only
         assert tg.workspace_size(tg.OP_Q2_LORA, 1536, 9216, 3072, 0) == 0  # invalid r
         # whole tiles fill 148 SMs evenly here: minimum == full size
         assert tg.workspace_size_min(tg.OP_Q2, 1536, 9216, 3072) == 1536 * 3072 * 2

@@ -64,3 +64,26 @@ def test_q2_lora_long_k(oracle, small_path):
     assert canary_intact(buf, M * N)
     gate_output(y, oracle.q2_lora_gemm(prob.x, wq, d, prob.a, prob.b, N), oracle,
                 f"q2 + branch small-M {M}x{N}x{K}")
+
+
+# The branch operands (u of a token pass, the CTA's rows of B) sit in shared memory next to
+# the activations: r = 256 at 16 tokens leaves less room for them (K is then cut into more
+# passes), r = 30 and r = 1 exercise the row pitches, 33 tokens three token passes (u
+# restaged per pass, the partial sums reusing the activations' space in between).
+@pytest.mark.parametrize("M,N,K,r", [(1, 77, 3072, 1), (8, 130, 3072, 30), (16, 520, 3072, 256),
+                                     (12, 200, 6144, 64), (33, 96, 1024, 6)])
+def test_q2_lora_operands_in_shared_memory(oracle, small_path, M, N, K, r):
+    prob = synth.q2_problem((34, M, N, K, r), M, N, K, r=r, ab_sigma=0.05)
+    wq, d, st = oracle.q2_pack(prob.codes, prob.scale)
+    assert st == 0
+    args = (dev(prob.x, torch.bfloat16), dev(wq, torch.uint8), dev(d, torch.float16),
+            dev(prob.a, torch.bfloat16), dev(prob.b, torch.bfloat16))
+    y, buf = nan_filled((M, N), torch.float32)
+    tg.gemm_q2_lora(*args, out_dtype=tg.OUT_F32, y=y)
+    y2 = tg.gemm_q2_lora(*args, out_dtype=tg.OUT_F32)
+    torch.cuda.synchronize()
+    assert canary_intact(buf, M * N)
+    gate_output(y, oracle.q2_lora_gemm(prob.x, wq, d, prob.a, prob.b, N), oracle,
+                f"q2 + branch small-M {M}x{N}x{K} r{r}")
+    assert torch.equal(y, y2), "two identical calls differ"
+    assert tg.device_error() == 0
