@@ -145,4 +145,146 @@ __global__ void __launch_bounds__(128, 1) mma_rate_kernel(int mode, int n, int i
   }
 }
 
+// Modes 6-8: the steady state of an 8-bit-activation design in which each 128-k block's
+// int32 products (M = 128 weight rows x N = 256 tokens, kind::i8, four K = 32 MMAs) are
+// drained from TMEM by 16 epilogue warps -- 4 per TMEM lane quarter, 64 token columns each,
+// read 16 at a time -- converted to f32 and added, times a per-row scale, into running sums held in
+// registers, while the next block's MMAs fill the other of two 256-column accumulators.
+//   mode 6: MMAs and drains together, int -> float by cvt;
+//   mode 7: the drains alone (no MMA; the same columns read each block), cvt;
+//   mode 8: as mode 6, int -> float by the exponent trick (i + 0x4B400000 read as a float
+//           is 12582912 + i for |i| < 2^22);
+//   mode 9: as mode 8 with the subtraction and the multiply-add on packed f32x2 pairs;
+//   mode 10: as mode 6 with the multiply-add on packed f32x2 pairs.
+// out[cta] = cycles for `iters` blocks, from the MMA-issuing thread (modes 6, 8: the last
+// block's drain included) or from epilogue warp 0 (mode 7).
+constexpr int kDrainWarps = 16;
+constexpr int kDrainThreads = (kDrainWarps + 1) * 32;
+__global__ void __launch_bounds__(kDrainThreads, 1) drain_rate_kernel(int mode, int iters,
+                                                                   unsigned long long* out) {
+  extern __shared__ uint8_t rate_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(rate_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  for (int i = tid; i < (kRateA + kRateB) / 16; i += blockDim.x)
+    reinterpret_cast<uint4*>(sm)[i] = make_uint4(0u, 0u, 0u, 0u);
+  const uint32_t sa = smem_u32(sm), sbx = sa + kRateA;
+  const uint32_t full0 = sa + kRateA + kRateB, empty0 = full0 + 16;  // two barriers each, 8 bytes apart
+  uint32_t* slot = reinterpret_cast<uint32_t*>(sm + kRateA + kRateB + 32);
+  volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(sm + kRateA + kRateB + 40);
+  if (tid == 0) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(full0 + 8 * i, 1);
+      mbar_init(empty0 + 8 * i, kDrainWarps);
+    }
+    *abort_flag = 0u;
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(slot), 512);
+    tmem_relinquish();
+  }
+  fence_proxy_async_smem();
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *slot;
+  const bool with_mma = mode != 7;
+  if (warp == kDrainWarps) {
+    if (lane == 0 && with_mma) {
+      const uint32_t idesc = make_idesc_i8(128u, 256u);
+      const uint64_t adesc = smem_desc_sw128(sa), bdesc = smem_desc_sw128(sbx);
+      const unsigned long long t0 = clock64();
+      bool ok = true;
+      for (int b = 0; b < iters && ok; ++b) {
+        const int p = b & 1;
+        if (b >= 2) ok = mbar_wait(empty0 + 8 * p, static_cast<uint32_t>(((b >> 1) - 1) & 1), abort_flag);
+        if (!ok) break;
+        tc_fence_after();
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          mma_i8_ss(tmem + 256u * p, adesc + 2u * k, bdesc + 2u * k, idesc, k > 0 ? 1u : 0u);
+        mma_commit(full0 + 8 * p);
+      }
+      if (ok) {
+        const int b = iters - 1;
+        ok = mbar_wait(empty0 + 8 * (b & 1), static_cast<uint32_t>((b >> 1) & 1), abort_flag);
+      }
+      out[blockIdx.x] = ok ? clock64() - t0 : 0ull;
+    }
+  } else {
+    const int lq = warp & 3, cs = warp >> 2;
+    const uint32_t taddr = tmem + (static_cast<uint32_t>(lq * 32) << 16) + 64u * cs;
+    const float d = 1.0f + 1e-3f * lane;
+    float acc[64];
+#pragma unroll
+    for (int i = 0; i < 64; ++i) acc[i] = 0.f;
+    const unsigned long long t0 = clock64();
+    for (int b = 0; b < iters; ++b) {
+      const int p = b & 1;
+      if (with_mma) {
+        if (!mbar_wait(full0 + 8 * p, static_cast<uint32_t>((b >> 1) & 1), abort_flag)) break;
+        tc_fence_after();
+      }
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {  // 16 columns at a time (registers: 64 sums + 16 loaded)
+        uint32_t v[16];
+        tmem_ld_32x32b_x16(taddr + 256u * p + 16u * h, v);
+        tmem_wait_ld();
+        if (h == 3 && with_mma) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(empty0 + 8 * p);
+        }
+        if (mode >= 9) {
+          // packed f32x2 arithmetic, two columns per instruction
+#pragma unroll
+          for (int i = 0; i < 16; i += 2) {
+            float f0, f1;
+            if (mode == 9) {
+              f0 = __uint_as_float(v[i] + 0x4B400000u);
+              f1 = __uint_as_float(v[i + 1] + 0x4B400000u);
+            } else {
+              f0 = static_cast<float>(static_cast<int>(v[i]));
+              f1 = static_cast<float>(static_cast<int>(v[i + 1]));
+            }
+            unsigned long long fv = (static_cast<unsigned long long>(__float_as_uint(f1)) << 32) | __float_as_uint(f0);
+            if (mode == 9) {
+              const unsigned long long mc = 0xCB400000CB400000ull;  // (-12582912, -12582912)
+              asm("add.rn.f32x2 %0, %1, %2;" : "=l"(fv) : "l"(fv), "l"(mc));
+            }
+            const unsigned long long dd = (static_cast<unsigned long long>(__float_as_uint(d)) << 32) | __float_as_uint(d);
+            unsigned long long ac = (static_cast<unsigned long long>(__float_as_uint(acc[16 * h + i + 1])) << 32) |
+                                    __float_as_uint(acc[16 * h + i]);
+            asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(ac) : "l"(dd), "l"(fv));
+            acc[16 * h + i] = __uint_as_float(static_cast<uint32_t>(ac));
+            acc[16 * h + i + 1] = __uint_as_float(static_cast<uint32_t>(ac >> 32));
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float f = mode == 8 ? __uint_as_float(v[i] + 0x4B400000u) - 12582912.f
+                                      : static_cast<float>(static_cast<int>(v[i]));
+            acc[16 * h + i] = fmaf(d, f, acc[16 * h + i]);
+          }
+        }
+      }
+    }
+    const unsigned long long t1 = clock64();
+    float keep = 0.f;
+#pragma unroll
+    for (int i = 0; i < 64; ++i) keep += acc[i];
+    if (keep == 12345.f) out[blockIdx.x] = 1ull;  // keeps the sums
+    if (mode == 7 && tid == 0) out[blockIdx.x] = t1 - t0;
+  }
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
 }  // namespace tgemm

@@ -908,7 +908,7 @@ int tgemm_selftest_wait_timeout(void* stream) {
 }
 
 int tgemm_mma_rate(int mode, int n, int iters, unsigned long long* out, int nout, void* stream) {
-  if (!out || mode < 0 || mode > 5 || iters < 1 || iters > (1 << 20)) return TGEMM_EINVAL;
+  if (!out || mode < 0 || mode > 10 || iters < 1 || iters > (1 << 20)) return TGEMM_EINVAL;
   if (mode <= 2 && (n < 16 || n > 256 || n % 16)) return TGEMM_EINVAL;
   if (!aligned(out, 8)) return TGEMM_EALIGN;
   DeviceInfo di;
@@ -918,16 +918,19 @@ int tgemm_mma_rate(int mode, int n, int iters, unsigned long long* out, int nout
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(once, [] {
     attr_err = cudaFuncSetAttribute(mma_rate_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kRateSmem);
+    if (attr_err == cudaSuccess)
+      attr_err = cudaFuncSetAttribute(drain_rate_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kRateSmem);
   });
   if (attr_err != cudaSuccess) return TGEMM_ECUDA;
   const cudaStream_t st = as_stream(stream);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(di.sms));
-  cfg.blockDim = dim3(128);
+  cfg.blockDim = dim3(mode >= 6 ? kDrainThreads : 128);
   cfg.dynamicSmemBytes = kRateSmem;
   cfg.stream = st;
-  return cudaLaunchKernelEx(&cfg, mma_rate_kernel, mode, n, iters, out) == cudaSuccess ? TGEMM_OK
-                                                                                       : TGEMM_ECUDA;
+  const cudaError_t le = mode >= 6 ? cudaLaunchKernelEx(&cfg, drain_rate_kernel, mode, iters, out)
+                                   : cudaLaunchKernelEx(&cfg, mma_rate_kernel, mode, n, iters, out);
+  return le == cudaSuccess ? TGEMM_OK : TGEMM_ECUDA;
 }
 
 int tgemm_selftest_bad_launch(void* stream) {

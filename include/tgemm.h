@@ -182,7 +182,13 @@ int tgemm_selftest_bad_launch(void* stream);
  *           memory;
  *   mode 3: tcgen05.ld of 32 lanes x 16 columns per warp (4 warps), each waited for;
  *   mode 4: warp mma.sync m16n8k16 bf16 -> f32, 5: mma.sync m16n8k32 s8 -> s32, each of
- *           4 warps running 8 independent accumulator chains (`iters` per warp).
+ *           4 warps running 8 independent accumulator chains (`iters` per warp);
+ *   modes 6-8: `iters` 128-k blocks of an 8-bit-activation pipeline: four kind::i8 MMAs
+ *           (M = 128, N = 256) per block into one of two int32 accumulators, each block
+ *           drained by 16 warps (64 columns each) into f32 running sums in registers
+ *           (sum += d * float(int)); 6: MMAs and drains overlapped, int -> float by cvt;
+ *           7: drains alone; 8: as 6 with the exponent-trick conversion; 9: as 8 and
+ *           10: as 6, with packed f32x2 subtract and multiply-add.  n is ignored.
  * n: 16..256, a multiple of 16 (modes 0-2).  Operands are zeros (or TMEM contents); the
  * results are not read.
  */
