@@ -101,13 +101,18 @@ struct TcFmt {
   static constexpr int kWqRowBytes = FMT == 0 ? 32 : 64;  // packed bytes per row per stage
   // Packed weights reach the dequant warps through their own ring of shared-memory
   // stages (one TMA box of 128 rows per stage), filled this many stages ahead: deep
-  // enough to hide a DRAM miss, small enough to fit beside the activation stages.
-  static constexpr int kWStages = FMT == 0 ? 8 : 4;
+  // enough to hide a DRAM miss, small enough to fit beside the activation stages (and,
+  // for Q2, the output boxes).
+  static constexpr int kWStages = 4;
   static constexpr int kWBytes = kTcRows * kWqRowBytes;
   static constexpr int kXOff = 0;
   static constexpr int kWOff = kXOff + kTcStages * kTcXBytes;
-  static constexpr int kBarOff = kWOff + kWStages * kWBytes;
-  static constexpr int kNumBars = 2 * kTcStages + 3 + 2 * kWStages;
+  // Q2: two [32 tokens][128 rows] bf16 boxes, one per half of the accumulator's columns,
+  // through which a whole tile's bf16 output is turned around for coalesced stores
+  static constexpr int kYBoxBytes = 32 * kTcRows * 2;
+  static constexpr int kYOff = kWOff + kWStages * kWBytes;
+  static constexpr int kBarOff = kYOff + (FMT == 0 ? 2 * kYBoxBytes : 0);
+  static constexpr int kNumBars = 2 * kTcStages + 3 + 2 * kWStages + 4;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kSmemBytes = kMiscOff + 16 + 1024;  // + alignment slack
 };
@@ -136,6 +141,7 @@ struct TcParams {
   int sk_t0;               // first tile of the split region (tiles before it are whole per CTA)
   int dpc;                 // whole-tile region: CTA c owns units [c * dpc, (c + 1) * dpc) (0: none)
   int lb_sn, lb_si;        // B's element strides: (r, 1) for B [N][r], (1, N) for B^T [r][N]
+  int y_box;               // whole tiles leave through the output boxes (Q2, bf16 y, N % 4 == 0)
 };
 
 // One tile's share of a CTA's unit range [u, u1): tile `tile`, stages [ka, kb).
@@ -238,6 +244,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const uint32_t drain_bar = bar0 + 8u * (2 * kTcStages + 2);
   auto wfull_bar = [&](int w) { return bar0 + 8u * (2 * kTcStages + 3 + w); };
   auto wempty_bar = [&](int w) { return bar0 + 8u * (2 * kTcStages + 3 + F::kWStages + w); };
+  // output boxes (Q2, bf16): filled / read out by the 4 warps of a column half
+  auto yfull_bar = [&](int h) { return bar0 + 8u * (2 * kTcStages + 3 + 2 * F::kWStages + h); };
+  auto yfree_bar = [&](int h) { return bar0 + 8u * (2 * kTcStages + 5 + 2 * F::kWStages + h); };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + F::kMiscOff);
   volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + F::kMiscOff + 4);
 
@@ -254,6 +263,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     for (int w = 0; w < F::kWStages; ++w) {
       mbar_init(wfull_bar(w), 1);   // weight producer's expect_tx
       mbar_init(wempty_bar(w), kTcDeqWarps);  // every dequant warp has read its codes
+    }
+    for (int h = 0; h < 2; ++h) {
+      mbar_init(yfull_bar(h), 4);  // the column half's 4 epilogue warps have filled the box
+      mbar_init(yfree_bar(h), 4);  // ... and have read it out
     }
     *abort_flag = 0u;
     fence_mbar_init();
@@ -529,6 +542,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     constexpr int kChunks = kTcTok / 32 / 2;
     constexpr int kPieceFloats = kTcSlotFloats / kTcEpiWarps;
     uint32_t scount = 0;
+    uint32_t ycount = 0;  // output boxes this warp has filled
     bool ok = true;
     for (int r = 0; ok && r < (HYB ? 2 : 1); ++r)
     for (int u = r ? rg.b0 : rg.a0, ue = r ? rg.b1 : rg.a1; u < ue; ++scount) {
@@ -559,6 +573,59 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             if (m0 + e < p.M) dst[static_cast<int64_t>(e) * p.N] = __float2bfloat16_rn(__uint_as_float(v[e]));
         }
       };
+      if (FMT == 0 && p.y_box && sg.ka == 0 && sg.kb == ksteps) {
+        // The whole tile, bf16.  A thread holds one weight row, so its stores of y (one
+        // token row per store) land 2 bytes apart from its neighbours'; instead, each
+        // 32-token chunk of this half of the accumulator is turned around in a
+        // [32 tokens][128 rows] box in shared memory, and each of the half's 4 warps then
+        // writes 8 token rows of 256 contiguous bytes (8 bytes a lane).  The 4 warps meet
+        // twice per chunk: box filled (yfull), box read (yfree); both waits are bounded.
+        uint16_t* ybox = reinterpret_cast<uint16_t*>(smem + F::kYOff + eh * F::kYBoxBytes);
+        const int n4 = tn * kTcRows + 4 * lane;  // this lane's 4 rows in the copy-out
+#pragma unroll 1
+        for (int cc = 0; ok && cc < kChunks; ++cc, ++ycount) {
+          const uint32_t yph = ycount & 1u;
+          if (!mbar_wait_warp(yfree_bar(eh), yph ^ 1u, abort_flag)) {
+            ok = false;
+            break;
+          }
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            uint32_t v[16];
+            tmem_ld_32x32b_x16(tbase + cc * 32 + hh * 16, v);
+            tmem_wait_ld();
+            if (cc == kChunks - 1 && hh == 1) {
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(accempty_bar);
+            }
+#pragma unroll
+            for (int e = 0; e < 16; ++e)
+              ybox[(16 * hh + e) * kTcRows + q * 32 + lane] =
+                  __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(v[e])));
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(yfull_bar(eh));
+          if (!mbar_wait_warp(yfull_bar(eh), yph, abort_flag)) {
+            ok = false;
+            break;
+          }
+          {
+            // this warp's 8 token rows of the chunk
+            const int m0 = mbase + cc * 32 + 8 * q;
+            const int rows = n4 < p.N ? min(8, p.M - m0) : 0;
+            const uint2* src = reinterpret_cast<const uint2*>(ybox + 8 * q * kTcRows + 4 * lane);
+            uint2* dst = reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(p.y) +
+                                                  static_cast<int64_t>(m0) * p.N + n4);
+#pragma unroll
+            for (int e8 = 0; e8 < 8; ++e8)
+              if (e8 < rows) dst[static_cast<int64_t>(e8) * (p.N / 4)] = src[e8 * (kTcRows / 4)];
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(yfree_bar(eh));
+        }
+        continue;
+      }
       if (sg.ka == 0 && sg.kb == ksteps) {
         // the whole tile: accumulator -> y
 #pragma unroll 1

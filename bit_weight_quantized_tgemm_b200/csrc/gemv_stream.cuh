@@ -125,10 +125,6 @@ __device__ __forceinline__ uint32_t ld_shared_u32(uint32_t saddr) {
   return v;
 }
 
-__device__ __forceinline__ void named_barrier_sync(int id, int threads) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
-}
-
 // Q2: the 8 code pairs (i, i+8) of a word as bf16 pairs (base_i + q_i, base_i + q_{i+8}).
 __device__ __forceinline__ void gs_q2_pairs(uint32_t w, uint32_t (&p)[8]) {
   const uint32_t w6 = w >> 6, w12 = w >> 12;

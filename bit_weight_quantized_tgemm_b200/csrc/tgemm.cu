@@ -672,6 +672,8 @@ int run_gemm(int fmt, const uint16_t* x, const uint8_t* wq, const uint16_t* scal
       return e;
   }
   TcParams p;
+  // bf16 Q2 output of whole tiles goes through the output boxes when 4 rows are 8 bytes
+  p.y_box = fmt == 0 && !out_f32 && N % 4 == 0 ? 1 : 0;
   p.M = M;
   p.N = N;
   p.K = K;
