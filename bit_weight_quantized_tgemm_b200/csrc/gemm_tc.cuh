@@ -94,6 +94,10 @@ constexpr int kTcTmemCols = 512;
 constexpr int kTcAccCols = kTcTok;              // f32 accumulator columns
 constexpr int kTcACol0 = kTcAccCols;            // first A-stage column
 constexpr int kTcACols = kTcBK / 2;             // columns per A stage (2 f16 per column)
+// Past the A stages: where the epilogue parks half of a finished tile's bf16 output (32
+// columns per column half of the accumulator) so that the accumulator is released sooner.
+constexpr int kTcStashCol0 = kTcACol0 + kTcStages * kTcACols;
+static_assert(kTcStashCol0 + 64 <= kTcTmemCols, "the epilogue's stash must fit in TMEM");
 static_assert(kTcACol0 + kTcStages * kTcACols <= kTcTmemCols, "TMEM budget");
 
 template <int FMT>
@@ -575,34 +579,73 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       };
       if (FMT == 0 && p.y_box && sg.ka == 0 && sg.kb == ksteps) {
         // The whole tile, bf16.  A thread holds one weight row, so its stores of y (one
-        // token row per store) land 2 bytes apart from its neighbours'; instead, each
+        // token row per store) would land 2 bytes apart from its neighbours'; instead, each
         // 32-token chunk of this half of the accumulator is turned around in a
         // [32 tokens][128 rows] box in shared memory, and each of the half's 4 warps then
-        // writes 8 token rows of 256 contiguous bytes (8 bytes a lane).  The 4 warps meet
-        // twice per chunk: box filled (yfull), box read (yfree); both waits are bounded.
+        // writes 8 token rows of 256 contiguous bytes (8 bytes a lane).  The accumulator is
+        // released first: its 4 chunks are read and packed to bf16 pairs, chunks 0-1 kept
+        // in registers and chunks 2-3 parked in the TMEM stash.  The 4 warps meet twice per
+        // chunk: box filled (yfull), box read out (yfree); both waits are bounded.
         uint16_t* ybox = reinterpret_cast<uint16_t*>(smem + F::kYOff + eh * F::kYBoxBytes);
+        const uint32_t tstash = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + kTcStashCol0 + eh * 32;
         const int n4 = tn * kTcRows + 4 * lane;  // this lane's 4 rows in the copy-out
-#pragma unroll 1
-        for (int cc = 0; ok && cc < kChunks; ++cc, ++ycount) {
-          const uint32_t yph = ycount & 1u;
-          if (!mbar_wait_warp(yfree_bar(eh), yph ^ 1u, abort_flag)) {
-            ok = false;
-            break;
-          }
+        // chunk 0 goes into the box at once (its previous read-out ended with the last
+        // tile), chunk 1 stays in registers as packed bf16 pairs, chunks 2-3 are parked in
+        // the stash; then the accumulator is released
+        if (!mbar_wait_warp(yfree_bar(eh), (ycount & 1u) ^ 1u, abort_flag)) {
+          ok = false;
+          continue;
+        }
+        uint32_t pk1[16];  // pk1[i]: tokens 32 + 2i (low half), 33 + 2i of this row
+#pragma unroll
+        for (int cc = 0; cc < kChunks; ++cc)
 #pragma unroll
           for (int hh = 0; hh < 2; ++hh) {
             uint32_t v[16];
             tmem_ld_32x32b_x16(tbase + cc * 32 + hh * 16, v);
             tmem_wait_ld();
-            if (cc == kChunks - 1 && hh == 1) {
-              tc_fence_before();
-              __syncwarp();
-              if (lane == 0) mbar_arrive(accempty_bar);
+            if (cc == 0) {
+#pragma unroll
+              for (int e = 0; e < 16; ++e)
+                ybox[(16 * hh + e) * kTcRows + q * 32 + lane] =
+                    __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(v[e])));
+              continue;
+            }
+            uint32_t w[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) w[i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+            if (cc == 1) {
+#pragma unroll
+              for (int i = 0; i < 8; ++i) pk1[8 * hh + i] = w[i];
+            } else {
+              tmem_st_32x32b_x8(tstash + (cc - 2) * 16 + hh * 8, w);
+            }
+          }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(accempty_bar);
+#pragma unroll
+        for (int cc = 0; cc < kChunks; ++cc) {
+          const uint32_t yph = (ycount + cc) & 1u;
+          if (cc > 0) {
+            if (!mbar_wait_warp(yfree_bar(eh), yph ^ 1u, abort_flag)) {
+              ok = false;
+              break;
+            }
+            uint32_t w[16];
+            if (cc == 1) {
+#pragma unroll
+              for (int i = 0; i < 16; ++i) w[i] = pk1[i];
+            } else {
+              tmem_ld_32x32b_x16(tstash + (cc - 2) * 16, w);
+              tmem_wait_ld();
             }
 #pragma unroll
-            for (int e = 0; e < 16; ++e)
-              ybox[(16 * hh + e) * kTcRows + q * 32 + lane] =
-                  __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(v[e])));
+            for (int i = 0; i < 16; ++i) {
+              ybox[(2 * i) * kTcRows + q * 32 + lane] = static_cast<uint16_t>(w[i] & 0xFFFFu);
+              ybox[(2 * i + 1) * kTcRows + q * 32 + lane] = static_cast<uint16_t>(w[i] >> 16);
+            }
           }
           __syncwarp();
           if (lane == 0) mbar_arrive(yfull_bar(eh));
@@ -624,6 +667,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           __syncwarp();
           if (lane == 0) mbar_arrive(yfree_bar(eh));
         }
+        ycount += kChunks;
         continue;
       }
       if (sg.ka == 0 && sg.kb == ksteps) {
