@@ -583,10 +583,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         // 32-token chunk of this half of the accumulator is turned around in a
         // [32 tokens][128 rows] box in shared memory, and each of the half's 4 warps then
         // writes 8 token rows of 256 contiguous bytes (8 bytes a lane).  The accumulator is
-        // released first: its 4 chunks are read and packed to bf16 pairs, chunks 0-1 kept
-        // in registers and chunks 2-3 parked in the TMEM stash.  The 4 warps meet twice per
-        // chunk: box filled (yfull), box read out (yfree); both waits are bounded.
+        // released before any of that: chunk 0 goes into the box, chunk 1 is kept in
+        // registers and chunks 2-3 in the TMEM stash, as packed bf16 pairs.  The 4 warps
+        // meet twice per chunk: box filled (yfull), box read out (yfree); both waits are
+        // bounded.
         uint16_t* ybox = reinterpret_cast<uint16_t*>(smem + F::kYOff + eh * F::kYBoxBytes);
+        uint16_t* ymine = ybox + q * 32 + lane;  // this thread's row in the box
         const uint32_t tstash = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + kTcStashCol0 + eh * 32;
         const int n4 = tn * kTcRows + 4 * lane;  // this lane's 4 rows in the copy-out
         // chunk 0 goes into the box at once (its previous read-out ended with the last
@@ -607,8 +609,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             if (cc == 0) {
 #pragma unroll
               for (int e = 0; e < 16; ++e)
-                ybox[(16 * hh + e) * kTcRows + q * 32 + lane] =
-                    __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(v[e])));
+                ymine[(16 * hh + e) * kTcRows] = __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(v[e])));
               continue;
             }
             uint32_t w[8];
@@ -625,7 +626,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(accempty_bar);
-#pragma unroll
+#pragma unroll 1
         for (int cc = 0; cc < kChunks; ++cc) {
           const uint32_t yph = (ycount + cc) & 1u;
           if (cc > 0) {
@@ -643,8 +644,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             }
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
-              ybox[(2 * i) * kTcRows + q * 32 + lane] = static_cast<uint16_t>(w[i] & 0xFFFFu);
-              ybox[(2 * i + 1) * kTcRows + q * 32 + lane] = static_cast<uint16_t>(w[i] >> 16);
+              ymine[(2 * i) * kTcRows] = static_cast<uint16_t>(w[i] & 0xFFFFu);
+              ymine[(2 * i + 1) * kTcRows] = static_cast<uint16_t>(w[i] >> 16);
             }
           }
           __syncwarp();
