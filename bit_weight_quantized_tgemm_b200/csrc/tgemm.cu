@@ -219,7 +219,12 @@ LoraDims lora_dims(int r, int K) {
 // split form only when it saves more than the split tiles' charge over whole tiles alone
 // (a larger charge when the CTAs also run whole tiles).
 constexpr int kDefaultSms = 148;    // sizes workspaces when no device is visible (B200)
-constexpr int kSplitPenalty = 2;    // units a split tile is charged (partial sums + fixup)
+// Units a pure-split schedule is charged for its partial sums and fix-ups, which come at
+// the end of every CTA's work: measured against whole tiles, 1536 tokens x 3072 x
+// (3072 + 12288) ran 120 us split against 105 us whole (117 + 2 units against 120), and
+// 256 x 9216 x 3072 32 us against 30 us (12 against 24 units), while the 4-bit encoder
+// shapes stayed faster split (40 against 46 us at 21 against 40 units).
+constexpr int kSplitPenalty = 13;
 // Next to whole tiles a CTA's split share costs more: writing its partial sums and fixing
 // up shared tiles keeps the epilogue warps from draining the following whole tile, which
 // stalls the MMAs (measured: 4096 tokens x 9216 x 3072 ran 6 % slower split than whole at

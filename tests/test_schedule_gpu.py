@@ -53,9 +53,9 @@ def _check(outs, ref, oracle, what):
     assert rel < 1e-5, f"{what}: schedules differ by {rel:.2e}"
 
 
-# Q2: 8 tiles of 32 stages (upc 2: every tile split 16 ways); 3 tiles of 4 stages with a
-# ragged token edge; and 2 x 8 tiles of 14 stages.
-@pytest.mark.parametrize("M,N,K", [(256, 1024, 4096), (200, 300, 512), (300, 1000, 1792)])
+# Q2: 8 tiles of 32 stages (upc 2: every tile split 16 ways); 3 tiles of 64 stages with
+# ragged token and row edges; and 2 x 8 tiles of 32 stages.
+@pytest.mark.parametrize("M,N,K", [(256, 1024, 4096), (200, 300, 8192), (300, 1000, 4096)])
 def test_q2_split_vs_whole(oracle, M, N, K):
     prob = synth.q2_problem((11, M, N, K), M, N, K)
     wq, d, st = oracle.q2_pack(prob.codes, prob.scale)
@@ -82,11 +82,11 @@ def test_q4_split_vs_whole(oracle):
     _check(_both(run, M, N), oracle.q4_gemm(prob.x, wq, sz, N), oracle, f"q4 {M}x{N}x{K}")
 
 
-# Branch: 9 main + 1 branch stage per tile, upc 2, so some segments hold only the
-# branch stage (the MMA must start that accumulator from zero).
+# Branch: 32 main + 1 branch stage per tile, upc 4, so the segment [32, 36) holds only
+# tile 0's branch stage (the MMA must start that accumulator from zero).
 @pytest.mark.parametrize("r", [4, 64])
 def test_q2_lora_split_vs_whole(oracle, r):
-    M, N, K = 300, 1000, 1152
+    M, N, K = 300, 1000, 4096
     prob = synth.q2_problem((13, M, N, K, r), M, N, K, r=r)
     wq, d, st = oracle.q2_pack(prob.codes, prob.scale)
     assert st == 0

@@ -123,8 +123,9 @@ def _form(pl):
     (tg.OP_Q2, 1536, 21504, 3072, 0, 0, "whole"),    # 1008 tiles: 6 waves + 120, likewise
     (tg.OP_Q2, 300, 13300, 3072, 0, 0, "hybrid"),    # 208 tiles: 1 wave + 60, ragged edges
     (tg.OP_Q2_LORA, 1280, 9216, 3072, 32, 0, "hybrid"),
-    (tg.OP_Q2, 1536, 3072, 3072, 0, 12288, "split"),  # fused out projection: 144 tiles of 120 stages
-    (tg.OP_Q2, 256, 9216, 3072, 0, 0, "split"),      # 72 tiles
+    (tg.OP_Q2, 1536, 3072, 3072, 0, 12288, "whole"),  # fused out projection: 144 tiles of 120 stages
+    (tg.OP_Q2, 256, 9216, 3072, 0, 0, "whole"),      # 72 tiles: halving K saves 12 units, less than the charge
+    (tg.OP_Q2, 256, 1024, 4096, 0, 0, "split"),      # 8 tiles of 32 stages
 ])
 def test_plan_forms(op, M, N, K, r, K2, form):
     pl = tg.tc_plan(op, M, N, K, r, K2, sms=148)
