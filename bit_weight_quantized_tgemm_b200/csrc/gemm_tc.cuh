@@ -26,25 +26,30 @@
 //   columns [0, 256)             the f32 accumulator
 //   columns [256 + 64 s, +64)    A stage s (s < 3): 128 rows x 128 k of f16, element k of
 //                                a row in column k/2 (low half for even k)
+//   columns [448, 512)           the epilogue's stash: half of a finished tile's bf16
+//                                output (32 columns per half of the accumulator)
 // Stage s of the pipeline is the activation tile in shared memory plus A stage s; one
 // mbarrier says it is full (TMA bytes + the eight dequant warps) and one says it is
 // free (the MMA's commit), so the MMA thread waits once and commits once per stage.
-// With one accumulator the MMA waits while a finished tile is read out; eight epilogue
-// warps keep that short, and the stages keep filling meanwhile, so the next tile starts
-// with full queues.
+// With one accumulator the MMA waits while a finished tile is read out; the epilogue
+// releases it as soon as the tile is out of TMEM (into a shared-memory box, registers and
+// the stash), before any store to y, and the stages keep filling meanwhile.
 //
-// Warp roles (18 warps, one CTA per SM):
+// Warp roles (19 warps, one CTA per SM):
 //   warp 0      TMA producer: activation tile, 256 tokens x 128 k as two 64-k boxes (f16,
 //               128-byte swizzle)
 //   warp 1      TMEM allocator and MMA issuer (one thread): 8 x tcgen05.mma 128x256x16
 //   warps 2-9   dequantizers: warp w handles TMEM lanes 32*(w%4).. (weight rows), warps
-//               2-5 the first 64 k of a stage and warps 6-9 the second; codes and
-//               scales come straight from global memory (16 or 32 bytes per thread per
-//               stage, issued ahead into alternating register sets), are unpacked and
-//               scaled in f16 and stored with one tcgen05.st of 32 columns
+//               2-5 the first 64 k of a stage and warps 6-9 the second; codes come from
+//               a shared-memory ring that warp 18 fills by TMA (one 128-row box per
+//               stage), scales straight from global memory one item ahead; they are
+//               unpacked and scaled in f16 and stored with one tcgen05.st of 32 columns
 //   warps 10-17 epilogue: warp w reads TMEM lanes 32*(w%4).. and half of the columns
-//               (tcgen05.ld), converts and stores y (lanes write consecutive n of one
-//               token row: coalesced)
+//               (tcgen05.ld) and stores y.  A whole tile's bf16 output is turned around
+//               through a [32 tokens][128 rows] shared-memory box per column half, so
+//               that each warp store writes 256 contiguous bytes of one token row;
+//               otherwise lanes write consecutive rows n of one token row
+//   warp 18     TMA producer: packed codes, one box of the tile's 128 rows per stage
 //
 // Operand precision: kind::f16 with both operands f16.  Q2_0 weights (q - 1) * d are
 // exact in f16; 4-bit weights are computed as ((q - z) * s) in f16, exact up to the
