@@ -863,12 +863,28 @@ __global__ void __launch_bounds__(256) prep_lora_kernel(const uint16_t* __restri
                                                         float* __restrict__ part,
                                                         int* __restrict__ cnt, int ncnt,
                                                         int a_vec) {
-  pdl_trigger_and_wait();
   static_assert((kPlPitch * 2) % 16 == 0, "pitch");
   extern __shared__ __align__(16) uint16_t pl_smem[];
   uint16_t* xs = pl_smem;                     // [kPlTok][kPlPitch] bf16 x tile
   uint16_t* as = pl_smem + kPlTok * kPlPitch;  // [64][kPlPitch] bf16 rows of A
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int k0 = blockIdx.y * kLoraKc;
+  // Columns [c0, c0 + 64) of A's K slice -> `as` by cp.async (A 16-byte aligned): 64 rows x
+  // 32 pieces of 16 bytes, zeros past r and K.  The first chunk is a weight read and goes
+  // out before the dependency wait, so its trip to memory overlaps the kernels ahead.
+  auto a_async = [&](int c0) {
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      const int pi = tid + 256 * j;  // piece: row pi / 64, 8 elements at (pi % 64) * 8
+      const int row = pi >> 6, e = (pi & 63) * 8;
+      const int col = c0 + row, k = k0 + e;
+      const bool in = col < r && k < K;  // K is a multiple of 128: a piece is all in or out
+      cp_async16(smem_u32(as + row * kPlPitch + e), in ? a + static_cast<int64_t>(col) * K + k : a, in ? 16u : 0u);
+    }
+  };
+  pdl_trigger();
+  if (a_vec) a_async(0);
+  pdl_wait();
   {
     const int64_t stride = static_cast<int64_t>(gridDim.x) * gridDim.y * blockDim.x;
     for (int64_t i = (static_cast<int64_t>(blockIdx.y) * gridDim.x + blockIdx.x) * blockDim.x + tid;
@@ -876,7 +892,6 @@ __global__ void __launch_bounds__(256) prep_lora_kernel(const uint16_t* __restri
       cnt[i] = 0;
   }
   const int m0 = blockIdx.x * kPlTok;
-  const int k0 = blockIdx.y * kLoraKc;
   // x tile: 64 rows x 32 groups of 16 (thread -> group, a warp covers one row); each
   // thread's 8 groups are loaded 4 at a time before any is stored
 #pragma unroll 1
@@ -912,8 +927,12 @@ __global__ void __launch_bounds__(256) prep_lora_kernel(const uint16_t* __restri
   const int ksteps = min(kLoraKc, K - k0) / 16;
   for (int c0 = 0; c0 < rpad; c0 += 64) {
     __syncthreads();  // x tile written (first pass) / previous A chunk consumed
+    if (a_vec) {
+      if (c0 > 0) a_async(c0);
+      cp_async_wait_all();
+    }
 #pragma unroll 1
-    for (int half = 0; half < 2; ++half) {
+    for (int half = 0; half < (a_vec ? 0 : 2); ++half) {
       uint4 v[4][2];
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
@@ -922,16 +941,10 @@ __global__ void __launch_bounds__(256) prep_lora_kernel(const uint16_t* __restri
         const int col = c0 + row, k = k0 + 16 * g;
         v[j][0] = make_uint4(0, 0, 0, 0);
         v[j][1] = v[j][0];
-        if (col < r && k < K) {
-          if (a_vec) {
-            const uint4* src = reinterpret_cast<const uint4*>(a + static_cast<int64_t>(col) * K + k);
-            v[j][0] = __ldg(src);
-            v[j][1] = __ldg(src + 1);
-          } else {  // A only 4-byte aligned
-            const uint32_t* src = reinterpret_cast<const uint32_t*>(a + static_cast<int64_t>(col) * K + k);
-            v[j][0] = make_uint4(__ldg(src), __ldg(src + 1), __ldg(src + 2), __ldg(src + 3));
-            v[j][1] = make_uint4(__ldg(src + 4), __ldg(src + 5), __ldg(src + 6), __ldg(src + 7));
-          }
+        if (col < r && k < K) {  // A only 4-byte aligned
+          const uint32_t* src = reinterpret_cast<const uint32_t*>(a + static_cast<int64_t>(col) * K + k);
+          v[j][0] = make_uint4(__ldg(src), __ldg(src + 1), __ldg(src + 2), __ldg(src + 3));
+          v[j][1] = make_uint4(__ldg(src + 4), __ldg(src + 5), __ldg(src + 6), __ldg(src + 7));
         }
       }
 #pragma unroll
