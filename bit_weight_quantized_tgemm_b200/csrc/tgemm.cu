@@ -14,6 +14,7 @@
 #include "../../include/tgemm.h"
 #include "common.cuh"
 #include "gemm_tc.cuh"
+#include "prep.cuh"
 #include "gemv.cuh"
 #include "gemv_stream.cuh"
 #include "mma_rate.cuh"
